@@ -1,0 +1,424 @@
+"""Benchmark of the D-Quant compressed-KV hot path on B200.
+
+One step = append one new token per sequence (dq_append_kv: rotate,
+normalise, quantise, rANS-encode, drift into a container) + one decode step
+of attention over the whole compressed context (dq_decode_attention: split-K
+kernel decoding the containers in-kernel + combine kernel), on the serving
+shape batch 128, 8 KV heads, 32 query heads, head_dim 128, 8192-token context
+(the token appended each step is position 8191; the context is 8192 tokens).
+
+Metric: compressed-KV decode attention throughput in KV tokens/s (B x context
+per step); the HBM rate of the compressed bytes and the dominant kernel's
+roofline fraction are reported beside it.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dq|reference]
+Under torchrun every rank runs an independent replica (no data-path
+collective): value = all ranks' KV tokens / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode attention: KV tokens/s and HBM GB/s at B=128, 8K ctx"
+UNIT = "KV tokens/s"
+WORKLOAD = "serve_b128_t8k"
+# Algorithmic work per token-head (one K and one V container), fixed
+# convention: 128 symbols x 2 streams x (5.5 rANS decode ops + G multiply-adds)
+# + 8 G softmax ops, counted in lane-ops (issue slots x 32).
+RANS_OPS_PER_SYMBOL = 5.5
+SOFTMAX_OPS_PER_HEAD = 8
+
+
+def ops_per_token_head(G: int) -> float:
+    return 2 * 128 * (RANS_OPS_PER_SYMBOL + G) + SOFTMAX_OPS_PER_HEAD * G
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def run_dq(args):
+    import numpy as np
+    import torch
+
+    import decode_attention_dq_b200 as dq
+    from decode_attention_dq_b200 import synth
+
+    ws, rank, local = dist_setup(args)
+    dist = None
+    if ws > 1:
+        import torch.distributed as dist
+    w = synth.WORKLOADS[args.workload]
+    if rank:  # each replica its own sequences
+        w = synth.scaled(w, seed=w.seed + 1000 * rank, name=w.name)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
+    ck, cv = tab.k.container_bytes, tab.v.container_bytes
+    T = w.T
+    T_cap = (T + 15) // 16 * 16
+    G = w.Hq // w.Hkv
+    kc = torch.zeros((w.B, w.Hkv, T_cap, ck), dtype=torch.uint8, device=dev)
+    vc = torch.zeros((w.B, w.Hkv, T_cap, cv), dtype=torch.uint8, device=dev)
+    prefill_stats = dq.new_stats(dev)
+    t0 = time.time()
+    synth.prefill_cache(tab, w, kc, vc, T - 1, stats=prefill_stats, threads=args.threads)
+    torch.cuda.synchronize()
+    prefill_s = time.time() - t0
+    pstats = dq.stats_dict(prefill_stats)
+
+    # Per-step inputs: a distinct new token and q for each step (host, pinned).
+    nsteps_inputs = 4
+    rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    host_k, host_v, host_q = [], [], []
+    for s in range(nsteps_inputs):
+        host_k.append(torch.from_numpy(synth.kv_block(w, "k", rows, n=1, step=s, threads=args.threads))
+                      .to(w.torch_dtype).view(w.B, w.Hkv, 1, 128).pin_memory())
+        host_v.append(torch.from_numpy(synth.kv_block(w, "v", rows, n=1, step=s, threads=args.threads))
+                      .to(w.torch_dtype).view(w.B, w.Hkv, 1, 128).pin_memory())
+        host_q.append(torch.from_numpy(synth.q_block(w, step=s)).to(w.torch_dtype).pin_memory())
+    dev_k = [t.to(dev) for t in host_k]
+    dev_v = [t.to(dev) for t in host_v]
+    dev_q = [t.to(dev) for t in host_q]
+    start = torch.full((w.B,), T - 1, dtype=torch.int32, device=dev)
+    seq = torch.full((w.B,), T, dtype=torch.int32, device=dev)
+    nbytes = dq.dq_decode_workspace_bytes(tab, w.B, w.Hq, w.Hkv, T)
+    wsp = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=dev)
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    stats = dq.new_stats(dev)
+    stream = torch.cuda.current_stream()
+
+    def step(s, e_dec0=None, e_dec1=None):
+        i = s % nsteps_inputs
+        dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kc, vc, stats=stats, stream=stream)
+        if e_dec0 is not None:
+            e_dec0.record(stream)
+        dq.dq_decode_attention(tab, dev_q[i], kc, vc, seq, T, out, wsp, stats=stats, stream=stream)
+        if e_dec1 is not None:
+            e_dec1.record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+
+    # ---- timed region: device-resident inputs ----
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for s in range(args.steps):
+        step(s, *ev_dec[s])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    dec_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / args.steps
+    if dist is not None:
+        t = torch.tensor([elapsed_ms, dec_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, dec_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / args.steps
+    kv_tokens_step = w.B * T
+    value = kv_tokens_step * ws / (ms_per_step * 1e-3)
+
+    # ---- e2e: host buffers, copies inside the timed region ----
+    def step_e2e(s):
+        i = s % nsteps_inputs
+        dev_k[i].copy_(host_k[i], non_blocking=True)
+        dev_v[i].copy_(host_v[i], non_blocking=True)
+        dev_q[i].copy_(host_q[i], non_blocking=True)
+        dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kc, vc, stats=stats, stream=stream)
+        dq.dq_decode_attention(tab, dev_q[i], kc, vc, seq, T, out, wsp, stats=stats, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for s in range(2):
+        step_e2e(s)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for s in range(args.steps):
+        step_e2e(s)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = f0.elapsed_time(f1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = kv_tokens_step * ws / (e2e_ms / args.steps * 1e-3)
+    h2d = (host_k[0].numel() + host_v[0].numel() + host_q[0].numel()) * host_k[0].element_size()
+    d2h = out_host.numel() * out_host.element_size()
+    st = dq.stats_dict(stats)
+
+    result = None
+    if rank == 0:
+        peaks, src = measured_peaks()
+        sm_count = torch.cuda.get_device_properties(dev).multi_processor_count
+        clock_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        alu_peak = sm_count * 128 * clock_mhz * 1e6 / 1e12  # T lane-ops/s
+        token_heads = w.B * T * w.Hkv
+        ops = token_heads * ops_per_token_head(G)
+        achieved = ops / (dec_ms * 1e-3) / 1e12
+        comp_bytes = token_heads * (ck + cv)
+        hbm_gbs = comp_bytes / (dec_ms * 1e-3) / 1e9
+        splits = (nbytes // (w.B * w.Hq * 4 * 130)) if nbytes else 1
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
+                       "context": T, "appended_per_step": 1, "input_dtype": w.dtype,
+                       "k_bits_per_value": w.k_bits, "v_bits_per_value": w.v_bits,
+                       "k_container_bytes": ck, "v_container_bytes": cv,
+                       "l2": "inputs larger than L2 (%.0f MB of containers read per step)" % (comp_bytes / 1e6),
+                       "parallelism": "replicas x%d" % ws},
+            "hbm_gbs": hbm_gbs,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tlaneop/s",
+                         "frac": achieved / alu_peak, "traffic": None,
+                         "kernel": "decode_split_kernel + combine_kernel (dq_decode_attention)",
+                         "kernel_ms": dec_ms, "peak_source": "%s clock, %d SMs x 128 lanes" % (src, sm_count),
+                         "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": peaks.get("hbm_gbs"),
+                                 "frac": hbm_gbs / float(peaks.get("hbm_gbs", 6650.0))}},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk,
+            "drift": {"prefill_k_syms_pct": 100.0 * pstats["k_syms_drifted"] / (token_heads * 128),
+                      "prefill_v_syms_pct": 100.0 * pstats["v_syms_drifted"] / (token_heads * 128),
+                      "prefill_k_cont_pct": 100.0 * pstats["k_cont_drifted"] / token_heads,
+                      "prefill_v_cont_pct": 100.0 * pstats["v_cont_drifted"] / token_heads,
+                      "fallbacks": pstats["overflow_fallbacks"]},
+            "integrity_errors": st["integrity_errors"],
+            "prefill_s": prefill_s,
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(w, tab_seed=0, seconds=args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def oracle_sample_step(w, tabs, rows, cache_rows):
+    """One bounded sample of the step on the host oracle: append one token to
+    each sampled row and decode-attend over its full context."""
+    import numpy as np
+    from oracle import oracle as o
+
+    G = w.Hq // w.Hkv
+    for (b, h), (kc, vc) in zip(rows, cache_rows):
+        from decode_attention_dq_b200 import synth
+        k_new = synth.kv_row(w, "k", b, h, n=1, step=0)
+        v_new = synth.kv_row(w, "v", b, h, n=1, step=0)
+        kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, np.array([h], np.int32))
+        vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, np.array([h], np.int32))
+        kc[-1] = kk[0]
+        vc[-1] = vv[0]
+        q = synth.q_rows(w, b)[h * G:(h + 1) * G]
+        qb = np.zeros((1, w.Hkv * G, 128))
+        qb[0, h * G:(h + 1) * G] = q
+        kfull = np.zeros((1, w.Hkv) + kc.shape, np.uint8)
+        vfull = np.zeros((1, w.Hkv) + vc.shape, np.uint8)
+        kfull[0, h] = kc
+        vfull[0, h] = vc
+        o.attention_fp64(tabs, qb, kfull, vfull, [kc.shape[0]], rows=[(0, h)])
+
+
+def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=64):
+    """The oracle, as it stands, on the host: bounded sample of the step."""
+    import numpy as np
+    from decode_attention_dq_b200 import synth
+    from oracle import oracle as o
+
+    tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
+                    v_container_bytes=o.container_bytes(w.v_bits), sign_seed=tab_seed)
+    # Containers for a few sampled rows, encoded by the oracle (setup, untimed).
+    rng = np.random.default_rng(0)
+    cand = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, max_rows), rng.integers(0, w.Hkv, max_rows))]
+    prepared = []
+    t_setup = time.time()
+    for b, h in cand:
+        K = synth.kv_row(w, "k", b, h)
+        V = synth.kv_row(w, "v", b, h)
+        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
+        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+        prepared.append(((b, h), (kc, vc)))
+        if time.time() - t_setup > seconds:
+            break
+    done = 0
+    t0 = time.time()
+    for (bh, cc) in prepared:
+        oracle_sample_step(w, tabs, [bh], [cc])
+        done += 1
+        if time.time() - t0 > seconds:
+            break
+    dt = time.time() - t0
+    kv_tokens = done * w.T / w.Hkv  # one KV token = one position across all KV heads
+    return {"value": kv_tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d (sequence, KV head) rows of %s: append 1 token + fp64 decode attention "
+                      "over %d tokens each, single thread, %.1f s" % (done, w.name, w.T, dt)}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    from decode_attention_dq_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    import numpy as np
+    from oracle import oracle as o
+    tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
+                    v_container_bytes=o.container_bytes(w.v_bits))
+    rows = [(s % w.B, (s * 3) % w.Hkv) for s in range(args.warmup + args.steps)]
+    prepared = []
+    for b, h in rows:
+        K = synth.kv_row(w, "k", b, h)
+        V = synth.kv_row(w, "v", b, h)
+        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
+        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+        prepared.append(((b, h), (kc, vc)))
+    for i in range(args.warmup):
+        oracle_sample_step(w, tabs, [prepared[i][0]], [prepared[i][1]])
+    t0 = time.time()
+    for i in range(args.warmup, args.warmup + args.steps):
+        oracle_sample_step(w, tabs, [prepared[i][0]], [prepared[i][1]])
+    dt = time.time() - t0
+    kv_tokens = args.steps * w.T / w.Hkv
+    value = kv_tokens / dt
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
+                       "context": w.T, "sample_per_step": "one (sequence, KV head) row"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": "per step: one (sequence, KV head) row of %s, append 1 token "
+                                       "+ fp64 attention over %d tokens, single thread" % (w.name, w.T)},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="dq", choices=["dq", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--threads", type=int, default=max(4, min(32, os.cpu_count() or 8)))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    res = run_reference(args) if args.impl == "reference" else run_dq(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

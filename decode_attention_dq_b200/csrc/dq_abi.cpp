@@ -1,0 +1,396 @@
+// dq_abi.cpp -- the C-ABI of libdq: argument checks, table upload, workspace
+// sizing and kernel launches. Every entry point catches C++ exceptions and
+// reports a DQ_ERR_* code; nothing here allocates per call except
+// dq_build_tables.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "dq_internal.h"
+
+struct dq_tables {
+  dq_config cfg{};
+  int device = -1;
+  int sm_count = 0;
+  dqi::StreamDesign k, v;
+  std::vector<int8_t> signs;
+  void *d_block = nullptr;
+  dqi::DevTables *d_tabs = nullptr;
+  uint32_t *d_sign_bits = nullptr;
+};
+
+namespace {
+
+thread_local int g_last_cuda = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda = static_cast<int>(e);
+  return DQ_ERR_CUDA;
+}
+
+// Same device as the tables? (Device pointers from another device would be
+// read through peer mappings at best; refuse instead.)
+int check_device(const dq_tables *t) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return dev == t->device ? DQ_OK : DQ_ERR_DEVICE;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
+  std::memset(s, 0, sizeof(*s));
+  for (int sym = 0; sym < d.n_levels; ++sym)
+    for (uint32_t slot = d.cum[sym]; slot < d.cum[sym + 1]; ++slot)
+      s->lut[slot] = (slot - d.cum[sym]) | (d.freq[sym] << 12) | (static_cast<uint32_t>(sym) << 24);
+  for (int i = 0; i < dqi::kMaxLevels; ++i) {
+    s->levels[i] = i < d.n_levels ? d.levels[i] : 0.0f;
+    s->thresholds[i] = d.thresholds[i];
+    s->cost[i] = i < d.n_levels ? d.cost[i] : INFINITY;
+    s->freq[i] = i < d.n_levels ? d.freq[i] : 0u;
+    s->cum[i] = i < d.n_levels ? d.cum[i] : dqi::kM;
+  }
+  s->n_levels = d.n_levels;
+  s->container_bytes = d.container_bytes;
+  s->payload_bytes = d.payload_bytes;
+}
+
+const dqi::StreamDesign *stream_of(const dq_tables *t, int kind) {
+  if (!t) return nullptr;
+  if (kind == DQ_STREAM_K) return &t->k;
+  if (kind == DQ_STREAM_V) return &t->v;
+  return nullptr;
+}
+
+// Split-K plan: chunk of tokens per CTA (a multiple of 32) and number of
+// splits, chosen so the grid fills whole waves of the SMs.
+struct Plan {
+  int splits;
+  int64_t chunk;
+};
+
+Plan plan_splits(int sm_count, int B, int Hkv, int64_t T_max) {
+  const int ctas_per_sm = 2;  // residency of the split kernel
+  const int64_t slots = static_cast<int64_t>(sm_count) * ctas_per_sm;
+  const int64_t bh = static_cast<int64_t>(B) * Hkv;
+  const int64_t min_chunk = 256;
+  int64_t max_splits = std::max<int64_t>(1, (T_max + min_chunk - 1) / min_chunk);
+  max_splits = std::min<int64_t>(max_splits, 256);
+  Plan best{1, std::max<int64_t>(32, ((T_max + 31) / 32) * 32)};
+  double best_score = -1.0;
+  for (int64_t s = 1; s <= max_splits; ++s) {
+    int64_t chunk = ((T_max + s - 1) / s + 31) / 32 * 32;
+    if (chunk < 32) chunk = 32;
+    int64_t eff_splits = (T_max + chunk - 1) / chunk;
+    if (eff_splits != s) continue;
+    const int64_t ctas = bh * s;
+    const double waves = static_cast<double>(ctas) / slots;
+    const double fill = waves / std::ceil(waves);
+    // prefer fuller waves; among near-equal fills prefer fewer splits
+    const double score = fill - 0.002 * s;
+    if (score > best_score) {
+      best_score = score;
+      best = Plan{static_cast<int>(s), chunk};
+    }
+  }
+  if (T_max == 0) best = Plan{1, 32};
+  return best;
+}
+
+size_t workspace_bytes(const Plan &p, int B, int Hq) {
+  const size_t rows = static_cast<size_t>(B) * Hq * p.splits;
+  size_t o = rows * dqi::kD * sizeof(float);
+  o = (o + 255) / 256 * 256;
+  return o + rows * 2 * sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+void dq_config_default(dq_config *cfg) {
+  if (!cfg) return;
+  std::memset(cfg, 0, sizeof(*cfg));
+  cfg->head_dim = 128;
+  cfg->k_levels = 8;
+  cfg->v_levels = 6;
+  cfg->prob_bits = 12;
+  cfg->k_bits_per_value = 2.26f;
+  cfg->v_bits_per_value = 2.26f;
+  cfg->n_kv_heads = 8;
+  cfg->sign_seed = 0;
+}
+
+const char *dq_error_string(int status) {
+  switch (status) {
+    case DQ_OK: return "ok";
+    case DQ_ERR_NULL: return "a required pointer is NULL";
+    case DQ_ERR_CONFIG: return "invalid configuration (head_dim, prob_bits or level counts)";
+    case DQ_ERR_BUDGET: return "container too small (or too large) for the level design";
+    case DQ_ERR_SHAPE: return "invalid shape argument";
+    case DQ_ERR_WORKSPACE: return "workspace too small";
+    case DQ_ERR_ALIGN: return "misaligned pointer or T_cap not a multiple of 16";
+    case DQ_ERR_DTYPE: return "unknown dtype";
+    case DQ_ERR_CUDA: return "CUDA runtime error (see dq_last_cuda_error)";
+    case DQ_ERR_DEVICE: return "not an sm_100 device or not the device of the tables";
+    default: return "unknown status";
+  }
+}
+
+int dq_last_cuda_error(void) { return g_last_cuda; }
+
+// Host-only design of one stream (no device needed); arrays of 8 (9 for cum).
+int dq_design_stream(int32_t n_levels, int32_t container_bytes, double rate_offset,
+                     float *levels, float *thresholds, uint32_t *freq, uint32_t *cum,
+                     float *cost, double *lambda, double *entropy, double *mse) {
+  try {
+    dqi::StreamDesign d;
+    int rc = dqi::design_stream(n_levels, container_bytes, rate_offset, &d);
+    if (rc != DQ_OK) return rc;
+    for (int i = 0; i < dqi::kMaxLevels; ++i) {
+      if (levels) levels[i] = i < n_levels ? d.levels[i] : 0.0f;
+      if (thresholds && i < dqi::kMaxLevels - 1) thresholds[i] = d.thresholds[i];
+      if (freq) freq[i] = d.freq[i];
+      if (cost) cost[i] = i < n_levels ? d.cost[i] : 0.0f;
+    }
+    if (cum)
+      for (int i = 0; i <= dqi::kMaxLevels; ++i) cum[i] = i <= n_levels ? d.cum[i] : dqi::kM;
+    if (lambda) *lambda = d.lambda;
+    if (entropy) *entropy = d.entropy;
+    if (mse) *mse = d.mse;
+    return DQ_OK;
+  } catch (...) {
+    return DQ_ERR_CONFIG;
+  }
+}
+
+int dq_build_tables(const dq_config *cfg, dq_tables **out) {
+  if (!cfg || !out) return DQ_ERR_NULL;
+  *out = nullptr;
+  if (cfg->head_dim != dqi::kD || cfg->prob_bits != dqi::kProbBits || cfg->n_kv_heads < 1 ||
+      cfg->n_kv_heads > 4096 || cfg->reserved != 0)
+    return DQ_ERR_CONFIG;
+  dq_tables *t = nullptr;
+  try {
+    t = new dq_tables();
+    t->cfg = *cfg;
+    const int ck = cfg->k_container_bytes ? cfg->k_container_bytes
+                                          : dqi::container_bytes_for(cfg->k_bits_per_value);
+    const int cv = cfg->v_container_bytes ? cfg->v_container_bytes
+                                          : dqi::container_bytes_for(cfg->v_bits_per_value);
+    int rc = dqi::design_stream(cfg->k_levels, ck, cfg->k_rate_offset, &t->k);
+    if (rc == DQ_OK) rc = dqi::design_stream(cfg->v_levels, cv, cfg->v_rate_offset, &t->v);
+    if (rc != DQ_OK) {
+      delete t;
+      return rc;
+    }
+    t->signs.resize(static_cast<size_t>(cfg->n_kv_heads) * dqi::kD);
+    dqi::rotation_signs(cfg->sign_seed, cfg->n_kv_heads, t->signs.data());
+
+    cudaError_t e = cudaGetDevice(&t->device);
+    if (e != cudaSuccess) { delete t; return cuda_fail(e); }
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, t->device);
+    if (e != cudaSuccess) { delete t; return cuda_fail(e); }
+    if (prop.major != 10) { delete t; return DQ_ERR_DEVICE; }
+    t->sm_count = prop.multiProcessorCount;
+
+    std::vector<uint8_t> host(sizeof(dqi::DevTables) + t->signs.size() / 8);
+    auto *dt = reinterpret_cast<dqi::DevTables *>(host.data());
+    fill_dev_stream(t->k, &dt->k);
+    fill_dev_stream(t->v, &dt->v);
+    auto *bits = reinterpret_cast<uint32_t *>(host.data() + sizeof(dqi::DevTables));
+    for (int h = 0; h < cfg->n_kv_heads; ++h)
+      for (int w = 0; w < 4; ++w) {
+        uint32_t word = 0;
+        for (int l = 0; l < 32; ++l)
+          if (t->signs[h * dqi::kD + w * 32 + l] < 0) word |= 1u << l;
+        bits[h * 4 + w] = word;
+      }
+    e = cudaMalloc(&t->d_block, host.size());
+    if (e != cudaSuccess) { delete t; return cuda_fail(e); }
+    e = cudaMemcpy(t->d_block, host.data(), host.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(t->d_block); delete t; return cuda_fail(e); }
+    t->d_tabs = reinterpret_cast<dqi::DevTables *>(t->d_block);
+    t->d_sign_bits = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(t->d_block) + sizeof(dqi::DevTables));
+    *out = t;
+    return DQ_OK;
+  } catch (const std::bad_alloc &) {
+    delete t;
+    return DQ_ERR_CONFIG;
+  } catch (...) {
+    delete t;
+    return DQ_ERR_CONFIG;
+  }
+}
+
+void dq_free_tables(dq_tables *t) {
+  if (!t) return;
+  if (t->d_block) cudaFree(t->d_block);
+  delete t;
+}
+
+int dq_get_stream_table(const dq_tables *t, int stream_kind, int32_t *n_levels,
+                        int32_t *container_bytes, float *levels, float *thresholds,
+                        uint32_t *freq, uint32_t *cum, float *cost) {
+  const dqi::StreamDesign *d = stream_of(t, stream_kind);
+  if (!d) return t ? DQ_ERR_CONFIG : DQ_ERR_NULL;
+  if (n_levels) *n_levels = d->n_levels;
+  if (container_bytes) *container_bytes = d->container_bytes;
+  for (int i = 0; i < dqi::kMaxLevels; ++i) {
+    if (levels) levels[i] = i < d->n_levels ? d->levels[i] : 0.0f;
+    if (thresholds && i < dqi::kMaxLevels - 1) thresholds[i] = d->thresholds[i];
+    if (freq) freq[i] = d->freq[i];
+    if (cost) cost[i] = i < d->n_levels ? d->cost[i] : 0.0f;
+  }
+  if (cum)
+    for (int i = 0; i <= dqi::kMaxLevels; ++i) cum[i] = i <= d->n_levels ? d->cum[i] : dqi::kM;
+  return DQ_OK;
+}
+
+int dq_get_stream_design(const dq_tables *t, int stream_kind, double *lambda, double *entropy,
+                         double *rate, double *mse, int32_t *is_lloyd_max) {
+  const dqi::StreamDesign *d = stream_of(t, stream_kind);
+  if (!d) return t ? DQ_ERR_CONFIG : DQ_ERR_NULL;
+  if (lambda) *lambda = d->lambda;
+  if (entropy) *entropy = d->entropy;
+  if (rate) *rate = d->rate;
+  if (mse) *mse = d->mse;
+  if (is_lloyd_max) *is_lloyd_max = d->lloyd_max ? 1 : 0;
+  return DQ_OK;
+}
+
+int dq_get_signs(const dq_tables *t, int8_t *signs) {
+  if (!t || !signs) return DQ_ERR_NULL;
+  std::memcpy(signs, t->signs.data(), t->signs.size());
+  return DQ_OK;
+}
+
+int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv,
+                 int n_new, const int32_t *d_start_pos, uint8_t *d_kcache, uint8_t *d_vcache,
+                 int64_t T_cap, dq_stats *d_stats, void *stream) {
+  try {
+    if (!t || !k || !v || !d_start_pos || !d_kcache || !d_vcache) return DQ_ERR_NULL;
+    if (dtype != DQ_F32 && dtype != DQ_BF16) return DQ_ERR_DTYPE;
+    if (B < 0 || n_new < 0 || T_cap < 0 || Hkv != t->cfg.n_kv_heads) return DQ_ERR_SHAPE;
+    if (!aligned(k, 16) || !aligned(v, 16)) return DQ_ERR_ALIGN;
+    int rc = check_device(t);
+    if (rc != DQ_OK) return rc;
+    if (B == 0 || n_new == 0) return DQ_OK;
+    dqi::AppendArgs a{};
+    a.tabs = t->d_tabs;
+    a.sign_bits = t->d_sign_bits;
+    a.k = k;
+    a.v = v;
+    a.dtype = dtype;
+    a.B = B;
+    a.Hkv = Hkv;
+    a.n_new = n_new;
+    a.start_pos = d_start_pos;
+    a.kcache = d_kcache;
+    a.vcache = d_vcache;
+    a.T_cap = T_cap;
+    a.ck = t->k.container_bytes;
+    a.cv = t->v.container_bytes;
+    a.nk = t->k.n_levels;
+    a.nv = t->v.n_levels;
+    a.stats = d_stats;
+    int e = dqi::launch_append(a, stream);
+    return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
+  } catch (...) {
+    return DQ_ERR_CUDA;
+  }
+}
+
+size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv, int64_t T_max) {
+  if (!t || B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || T_max < 0) return 0;
+  const Plan p = plan_splits(t->sm_count, B, Hkv, T_max);
+  return workspace_bytes(p, B, Hq);
+}
+
+int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
+                        const uint8_t *d_vcache, const int32_t *d_seq_lens, int B, int Hq, int Hkv,
+                        int64_t T_cap, int64_t T_max, float sm_scale, void *out, int out_dtype,
+                        void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream) {
+  try {
+    if (!t || !q || !d_kcache || !d_vcache || !d_seq_lens || !out || !d_workspace) return DQ_ERR_NULL;
+    if ((q_dtype != DQ_F32 && q_dtype != DQ_BF16) || (out_dtype != DQ_F32 && out_dtype != DQ_BF16))
+      return DQ_ERR_DTYPE;
+    if (B < 0 || Hkv != t->cfg.n_kv_heads || Hq < Hkv || Hq % Hkv) return DQ_ERR_SHAPE;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return DQ_ERR_SHAPE;
+    if (T_cap < 0 || T_max < 0 || T_max > T_cap) return DQ_ERR_SHAPE;
+    if (T_cap % 16 || !aligned(d_kcache, 16) || !aligned(d_vcache, 16) || !aligned(d_workspace, 16) ||
+        !aligned(q, 4) || !aligned(out, 4))
+      return DQ_ERR_ALIGN;
+    if (!std::isfinite(sm_scale)) return DQ_ERR_SHAPE;
+    const Plan p = plan_splits(t->sm_count, B, Hkv, T_max);
+    if (ws_bytes < workspace_bytes(p, B, Hq)) return DQ_ERR_WORKSPACE;
+    int rc = check_device(t);
+    if (rc != DQ_OK) return rc;
+    if (B == 0) return DQ_OK;
+    dqi::DecodeArgs a{};
+    a.tabs = t->d_tabs;
+    a.sign_bits = t->d_sign_bits;
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.kcache = d_kcache;
+    a.vcache = d_vcache;
+    a.seq_lens = d_seq_lens;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = G;
+    a.T_cap = T_cap;
+    a.T_max = T_max;
+    a.sm_scale = sm_scale;
+    a.out = out;
+    a.out_dtype = out_dtype;
+    size_t o_bytes = static_cast<size_t>(B) * Hq * p.splits * dqi::kD * sizeof(float);
+    o_bytes = (o_bytes + 255) / 256 * 256;
+    a.ws_o = static_cast<float *>(d_workspace);
+    a.ws_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(d_workspace) + o_bytes);
+    a.splits = p.splits;
+    a.chunk = p.chunk;
+    a.ck = t->k.container_bytes;
+    a.cv = t->v.container_bytes;
+    a.stats = d_stats;
+    int e = dqi::launch_decode_attention(a, stream);
+    return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
+  } catch (...) {
+    return DQ_ERR_CUDA;
+  }
+}
+
+int dq_decode_symbols(const dq_tables *t, const uint8_t *d_cache, int stream_kind,
+                      int64_t n_containers, uint8_t *d_syms, uint16_t *d_norm16, int32_t *d_status,
+                      dq_stats *d_stats, void *stream) {
+  try {
+    if (!t || !d_cache || !d_syms || !d_norm16) return DQ_ERR_NULL;
+    if (stream_kind != DQ_STREAM_K && stream_kind != DQ_STREAM_V) return DQ_ERR_CONFIG;
+    if (n_containers < 0) return DQ_ERR_SHAPE;
+    if (!aligned(d_cache, 4)) return DQ_ERR_ALIGN;
+    int rc = check_device(t);
+    if (rc != DQ_OK) return rc;
+    if (n_containers == 0) return DQ_OK;
+    dqi::SymbolsArgs a{};
+    a.tab = stream_kind == DQ_STREAM_K ? &t->d_tabs->k : &t->d_tabs->v;
+    a.cache = d_cache;
+    a.n = n_containers;
+    a.c = stream_kind == DQ_STREAM_K ? t->k.container_bytes : t->v.container_bytes;
+    a.syms = d_syms;
+    a.norm16 = d_norm16;
+    a.status = d_status;
+    a.stats = d_stats;
+    int e = dqi::launch_decode_symbols(a, stream);
+    return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
+  } catch (...) {
+    return DQ_ERR_CUDA;
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,223 @@
+/*
+ * dq.h -- C-ABI of libdq, the B200 (sm_100a) D-Quant compressed-KV hot path.
+ *
+ * D-Quant stores each token's K or V head vector as a fixed-size byte
+ * container: the vector is rotated and normalised so its coordinates are close
+ * to N(0,1), quantised to a few levels, entropy-coded with rANS, and "drift"
+ * moves a few symbols one level to a cheaper neighbour until the stream fits.
+ * Attention then decodes the containers inside the attention kernel.
+ *   [news] "D-Quant: Entropy Coding Meets KV Cache at 2.26 Bits", sections
+ *          "Why Fixed Width Is a Ceiling" and "Drift: Bending Variable Back to
+ *          Fixed" (8 levels for K, 6 for V at 2.26 bits; no symbol moves more
+ *          than one level; analytic, calibration-free probability model).
+ *   [abstract] "D-Quant: Driftable Entropy Coding for KV Cache Quantization",
+ *          Abstract (fixed-size bitstreams; regular memory access and parallel
+ *          dequantisation within attention kernels).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* and the k/v/q/out buffers are DEVICE pointers on the
+ *     device the tables were built on; everything else is host memory.
+ *   - The caller owns every device buffer (inputs, caches, workspace, stats,
+ *     outputs). The library owns only what dq_build_tables allocates.
+ *   - Device work is enqueued on `stream` (a cudaStream_t, or NULL for the
+ *     legacy default stream) and is asynchronous; nothing is allocated and
+ *     nothing synchronises inside dq_append_kv, dq_decode_attention and
+ *     dq_decode_symbols.
+ *   - Return value: DQ_OK (0) or a negative DQ_ERR_* code. Argument errors are
+ *     detected on the host before anything is enqueued. Errors in the data
+ *     (a corrupt container, a non-finite input, a position past the cache)
+ *     never fault or hang a kernel: they are counted in the caller's dq_stats.
+ *   - No C++ exception crosses this boundary. There is no CPU fallback.
+ *
+ * Layouts (row-major, contiguous):
+ *   K/V new tokens   [B][Hkv][n_new][128]      fp32 or bf16
+ *   K cache          [B][Hkv][T_cap][C_k]      uint8 containers
+ *   V cache          [B][Hkv][T_cap][C_v]      uint8 containers
+ *   q                [B][Hq][128]              fp32 or bf16
+ *   out              [B][Hq][128]              fp32 or bf16
+ * Query head hq attends with KV head hq / (Hq / Hkv) (grouped-query
+ * attention). Container layout: bytes 0-1 the fp16 norm ||x||
+ * (little-endian), bytes 2-4 the final rANS state (little-endian), then the
+ * renormalisation bytes in decode order, then zero padding to C.
+ */
+#ifndef DQ_H
+#define DQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum dq_status {
+  DQ_OK = 0,
+  DQ_ERR_NULL = -1,      /* a required pointer is NULL                       */
+  DQ_ERR_CONFIG = -2,    /* head_dim != 128, prob_bits != 12, level counts    */
+  DQ_ERR_BUDGET = -3,    /* container too small for the level design          */
+  DQ_ERR_SHAPE = -4,     /* B, Hkv, Hq, n_new, T_cap, T_max out of range       */
+  DQ_ERR_WORKSPACE = -5, /* workspace smaller than dq_decode_workspace_bytes  */
+  DQ_ERR_ALIGN = -6,     /* pointer or T_cap alignment (see each call)        */
+  DQ_ERR_DTYPE = -7,     /* unknown dtype code                                */
+  DQ_ERR_CUDA = -8,      /* a CUDA runtime call or launch failed              */
+  DQ_ERR_DEVICE = -9     /* not an sm_100 device, or not the tables' device   */
+};
+
+enum dq_dtype { DQ_F32 = 0, DQ_BF16 = 1 };
+enum dq_stream_kind { DQ_STREAM_K = 0, DQ_STREAM_V = 1 };
+
+/* Table configuration. Container size C = round-half-up(bits * 128 / 8)
+ * when *_container_bytes is 0 (2.26 -> 36 B, 1.96 -> 31 B, 3.0 -> 48 B). */
+typedef struct {
+  int32_t head_dim;          /* must be 128                                  */
+  int32_t k_levels;          /* even, 2..8 (default 8)                       */
+  int32_t v_levels;          /* even, 2..8 (default 6)                       */
+  int32_t prob_bits;         /* must be 12 (M = 4096)                        */
+  int32_t k_container_bytes; /* 0: derive from k_bits_per_value              */
+  int32_t v_container_bytes; /* 0: derive from v_bits_per_value              */
+  float k_bits_per_value;    /* default 2.26                                 */
+  float v_bits_per_value;    /* default 2.26                                 */
+  int32_t n_kv_heads;        /* >= 1; one rotation-sign vector per KV head   */
+  int32_t reserved;          /* must be 0                                    */
+  uint64_t sign_seed;        /* rotation signs: splitmix64 from this seed    */
+  float k_rate_offset;       /* added to the target rate, bits/value (0)     */
+  float v_rate_offset;       /* added to the target rate, bits/value (0)     */
+} dq_config;
+
+/* Device counters, caller-owned (cudaMemset to 0 before use; may be NULL in
+ * every call that takes one). Updated with atomics. */
+typedef struct {
+  unsigned long long k_syms_drifted;     /* K symbols moved by drift         */
+  unsigned long long v_syms_drifted;     /* V symbols moved by drift         */
+  unsigned long long k_cont_drifted;     /* K containers with >= 1 move      */
+  unsigned long long v_cont_drifted;     /* V containers with >= 1 move      */
+  unsigned long long overflow_fallbacks; /* containers that took the fallback */
+  unsigned long long integrity_errors;   /* corrupt containers decoded       */
+  unsigned long long nonfinite_inputs;   /* input vectors treated as zero    */
+  unsigned long long dropped_writes;     /* append positions >= T_cap        */
+  unsigned long long clamped_lengths;    /* seq_len > T_max or > T_cap       */
+} dq_stats;
+
+typedef struct dq_tables dq_tables; /* opaque, library-owned */
+
+/* Fills *cfg with the defaults: head_dim 128, K 8 levels, V 6 levels,
+ * prob_bits 12, 2.26 bits/value for both streams (36-byte containers),
+ * n_kv_heads 8, sign_seed 0, no rate offsets. */
+void dq_config_default(dq_config *cfg);
+
+/* Designs the K and V tables ([news] "Drift..." 3rd paragraph: the
+ * probability model comes analytically from the normal distribution, no
+ * calibration data) and uploads them to the CURRENT device.
+ *   Level design: Lloyd-Max for N(0,1) when its entropy fits the target rate
+ *   r = (8(C-2) - 24)/128 + rate_offset, else the entropy-constrained scalar
+ *   quantiser whose entropy equals r. Integer frequencies sum to 4096.
+ * Returns DQ_ERR_CONFIG / DQ_ERR_BUDGET / DQ_ERR_DEVICE / DQ_ERR_CUDA on
+ * failure (and *out is left NULL). Ownership of *out passes to the caller,
+ * who releases it with dq_free_tables. Not asynchronous (one-time set-up). */
+int dq_build_tables(const dq_config *cfg, dq_tables **out);
+
+/* Releases the tables (host and device memory). NULL is allowed. Must not be
+ * called while work that uses the tables is still running on the device. */
+void dq_free_tables(dq_tables *t);
+
+/* Host copies of one stream's table (for inspection and tests). Arrays must
+ * hold 8 entries (levels, freq, cost), 9 (cum), 7 (thresholds). Any output
+ * pointer may be NULL. */
+int dq_get_stream_table(const dq_tables *t, int stream_kind, int32_t *n_levels,
+                        int32_t *container_bytes, float *levels,
+                        float *thresholds, uint32_t *freq, uint32_t *cum,
+                        float *cost);
+
+/* Design summary of one stream: ECSQ multiplier (0 for Lloyd-Max), entropy
+ * and target rate in bits/value, design MSE for N(0,1). */
+int dq_get_stream_design(const dq_tables *t, int stream_kind, double *lambda,
+                         double *entropy, double *rate, double *mse,
+                         int32_t *is_lloyd_max);
+
+/* Host-only design of one stream's table (no device is touched): the same
+ * design dq_build_tables uploads. Arrays: levels, freq, cost 8 entries;
+ * thresholds 7; cum 9 (entries past n_levels are 0, or 4096 for cum). Any
+ * output pointer may be NULL. Returns DQ_ERR_CONFIG / DQ_ERR_BUDGET like
+ * dq_build_tables. */
+int dq_design_stream(int32_t n_levels, int32_t container_bytes, double rate_offset,
+                     float *levels, float *thresholds, uint32_t *freq, uint32_t *cum,
+                     float *cost, double *lambda, double *entropy, double *mse);
+
+/* Host copy of the rotation signs, int8 [n_kv_heads][128], values +-1. */
+int dq_get_signs(const dq_tables *t, int8_t *signs);
+
+/* Appends n_new tokens per sequence ([news] "Drift: Bending Variable Back to
+ * Fixed": each token's K or V goes into a fixed-size container; when the
+ * entropy-coded stream is too long, a few symbols drift one level to a
+ * cheaper neighbour until it fits).
+ *   k, v        device, [B][Hkv][n_new][128], dtype DQ_F32 or DQ_BF16,
+ *               16-byte aligned
+ *   d_start_pos device int32 [B]: token j of sequence b is written at
+ *               position d_start_pos[b] + j; positions outside [0, T_cap)
+ *               are skipped and counted in dropped_writes
+ *   d_kcache    device [B][Hkv][T_cap][C_k]; d_vcache [B][Hkv][T_cap][C_v]
+ *   d_stats     device dq_stats or NULL
+ *   stream      cudaStream_t
+ * Hkv must equal the tables' n_kv_heads. Containers are bit-identical to the
+ * reference definition (fp32 rotation/normalisation in a fixed order, greedy
+ * drift, zero padding). */
+int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype,
+                 int B, int Hkv, int n_new, const int32_t *d_start_pos,
+                 uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
+                 dq_stats *d_stats, void *stream);
+
+/* Bytes of device workspace dq_decode_attention needs for these shapes
+ * (split-K partial results). Depends only on its arguments and the tables'
+ * device. Returns 0 on invalid shapes. */
+size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv,
+                                 int64_t T_max);
+
+/* Decode attention over the compressed cache ([abstract]: regular memory
+ * access and parallel dequantisation within attention kernels). For every
+ * (b, hq): out = softmax(sm_scale * q K^T) V over the first d_seq_lens[b]
+ * tokens of the cache, with K and V dequantised from their containers
+ * inside the kernel. Runs as a split-K kernel (rANS decode of K and V,
+ * q.K^T, online softmax, P.V per token chunk) plus a combine kernel
+ * (log-sum-exp merge of the chunks and the inverse rotation).
+ *   q           device [B][Hq][128], q_dtype DQ_F32 or DQ_BF16
+ *   d_kcache, d_vcache  device caches, 16-byte aligned, T_cap % 16 == 0
+ *   d_seq_lens  device int32 [B]; a length above T_max or T_cap is clamped
+ *               and counted in clamped_lengths; length 0 gives out = 0
+ *   T_max       host bound on max(d_seq_lens), 0 <= T_max <= T_cap
+ *   sm_scale    softmax scale (1/sqrt(128) is the usual choice)
+ *   out         device [B][Hq][128], out_dtype DQ_F32 or DQ_BF16
+ *   d_workspace device, >= dq_decode_workspace_bytes(...) bytes, 16-byte
+ *               aligned; contents need not be initialised
+ *   d_stats     device dq_stats or NULL (integrity_errors counts containers
+ *               whose decoder did not end in the initial state)
+ * Hq must be a multiple of Hkv with Hq/Hkv in {1, 2, 4, 8}; Hkv must equal
+ * the tables' n_kv_heads. */
+int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype,
+                        const uint8_t *d_kcache, const uint8_t *d_vcache,
+                        const int32_t *d_seq_lens, int B, int Hq, int Hkv,
+                        int64_t T_cap, int64_t T_max, float sm_scale,
+                        void *out, int out_dtype, void *d_workspace,
+                        size_t ws_bytes, dq_stats *d_stats, void *stream);
+
+/* Test hook: decodes n flat containers of one stream.
+ *   d_cache   device [n][C]; d_syms device uint8 [n][128]; d_norm16 device
+ *             uint16 [n]; d_status device int32 [n] (may be NULL)
+ * Status per container: 0 ok, 1 initial state below 2^16, 2 the decoder ran
+ * past the container, 3 final state != 2^16, 4 non-zero padding. Symbols
+ * after the point of failure are 0. Corrupt containers are also counted in
+ * d_stats->integrity_errors. */
+int dq_decode_symbols(const dq_tables *t, const uint8_t *d_cache,
+                      int stream_kind, int64_t n_containers, uint8_t *d_syms,
+                      uint16_t *d_norm16, int32_t *d_status, dq_stats *d_stats,
+                      void *stream);
+
+/* Static description of a status code. Never NULL. */
+const char *dq_error_string(int status);
+
+/* The last CUDA error code seen by the library on this thread (0 if none). */
+int dq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DQ_H */

@@ -1,0 +1,78 @@
+"""CPU checks of the C-ABI boundary (no GPU needed).
+
+libdq.so loads and exports every function include/dq.h declares; its
+host-side table design (dq_design_stream, the same code dq_build_tables
+uploads) is byte-identical to the oracle's independently written design.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from decode_attention_dq_b200 import _native as N
+from oracle import oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "dq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(dq_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = N.load()
+    declared = _declared_functions()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+    assert set(declared) == set(N.EXPORTED)
+
+
+def test_error_strings():
+    for code in range(-9, 1):
+        assert N.dq_error_string(code)
+    assert N.dq_error_string(-100) == "unknown status"
+
+
+BUDGETS = [(8, 36), (6, 36), (8, 31), (6, 31), (8, 48), (6, 48), (4, 36), (2, 36), (8, 64)]
+
+
+@pytest.mark.parametrize("n,cb", BUDGETS)
+def test_host_design_equals_oracle(n, cb):
+    lib = N.dq_design_stream(n, cb)
+    ref = o.Stream(n, cb)
+    assert lib["freq"] == [int(v) for v in ref.freq]
+    assert lib["cum"] == [int(v) for v in ref.cum]
+    np.testing.assert_array_equal(np.array(lib["levels"], np.float32), ref.yf)
+    np.testing.assert_array_equal(np.array(lib["thresholds"], np.float32), ref.tf)
+    np.testing.assert_array_equal(np.array(lib["cost"], np.float32), ref.cost)
+    assert lib["lam"] == pytest.approx(ref.lam, abs=1e-12)
+    assert lib["entropy"] == pytest.approx(ref.entropy, abs=1e-12)
+    assert lib["mse"] == pytest.approx(ref.mse, abs=1e-12)
+
+
+@pytest.mark.parametrize("off", [-0.1, 0.05, 0.2])
+def test_host_design_equals_oracle_with_rate_offsets(off):
+    for n in (8, 6):
+        lib = N.dq_design_stream(n, 36, off)
+        ref = o.Stream(n, 36, off)
+        assert lib["freq"] == [int(v) for v in ref.freq]
+        np.testing.assert_array_equal(np.array(lib["levels"], np.float32), ref.yf)
+        np.testing.assert_array_equal(np.array(lib["thresholds"], np.float32), ref.tf)
+
+
+def test_host_design_rejects_bad_configs():
+    with pytest.raises(N.DqError) as e:
+        N.dq_design_stream(8, 12)
+    assert e.value.code == -3
+    with pytest.raises(N.DqError) as e:
+        N.dq_design_stream(7, 36)
+    assert e.value.code == -2
+    with pytest.raises(N.DqError):
+        N.dq_design_stream(10, 36)  # the decoder supports at most 8 levels
