@@ -23,7 +23,7 @@ STATS_FIELDS = ("k_syms_drifted", "v_syms_drifted", "k_cont_drifted", "v_cont_dr
 EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_stream_table",
             "dq_get_stream_design", "dq_get_signs", "dq_append_kv", "dq_decode_workspace_bytes",
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",
-            "dq_design_stream")
+            "dq_design_stream", "dq_decode_attention_noalloc")
 
 
 class DqConfig(C.Structure):
@@ -74,6 +74,8 @@ def load():
     lib.dq_decode_attention.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int, C.c_int,
                                         i64, i64, C.c_float, vp, C.c_int, vp, C.c_size_t, vp, vp]
     lib.dq_decode_symbols.argtypes = [vp, vp, C.c_int, i64, vp, vp, vp, vp, vp]
+    lib.dq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int,
+                                                C.c_int, i64, i64, C.c_float, vp, C.c_int, vp, vp]
     lib.dq_error_string.argtypes = [C.c_int]
     lib.dq_error_string.restype = C.c_char_p
     lib.dq_last_cuda_error.argtypes = []
@@ -224,6 +226,24 @@ def dq_decode_attention(tab: Tables, q: torch.Tensor, kcache: torch.Tensor, vcac
         tab.handle, _ptr(q), _dtype_code(q), _ptr(kcache), _ptr(vcache), _ptr(seq_lens), B, Hq,
         Hkv, T_cap, T_max, float(sm_scale), _ptr(out), _dtype_code(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(stats), _stream(stream)))
+
+
+def dq_decode_attention_noalloc(tab: Tables, q: torch.Tensor, kcache: torch.Tensor,
+                                vcache: torch.Tensor, seq_lens: torch.Tensor, T_max: int,
+                                out: torch.Tensor, sm_scale: float | None = None,
+                                stats: torch.Tensor | None = None, stream=None) -> None:
+    """dq_decode_attention for callers that cannot allocate: no workspace
+    argument; the library's fixed 8 MiB device scratch array is used instead
+    (shared by all calls on a device, so overlapping calls must be ordered)."""
+    B, Hq, d = q.shape
+    Hkv, T_cap = kcache.shape[1], kcache.shape[2]
+    assert d == 128 and q.is_contiguous() and out.is_contiguous() and seq_lens.dtype == torch.int32
+    if sm_scale is None:
+        sm_scale = 128 ** -0.5
+    _check("dq_decode_attention_noalloc", load().dq_decode_attention_noalloc(
+        tab.handle, _ptr(q), _dtype_code(q), _ptr(kcache), _ptr(vcache), _ptr(seq_lens), B, Hq,
+        Hkv, T_cap, T_max, float(sm_scale), _ptr(out), _dtype_code(out), _ptr(stats),
+        _stream(stream)))
 
 
 def dq_decode_symbols(tab: Tables, cache: torch.Tensor, kind: int, syms: torch.Tensor,

@@ -199,6 +199,34 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype,
                         void *out, int out_dtype, void *d_workspace,
                         size_t ws_bytes, dq_stats *d_stats, void *stream);
 
+/* Decode attention without a caller-provided workspace. The D-Quant pages
+ * have no counterpart to this call: it exists for callers that cannot
+ * allocate device memory -- a host application or plugin that is handed only
+ * input and output device pointers, or a serving loop that must not call
+ * cudaMalloc once it is running (an allocation can synchronise the device and
+ * compete with a caching allocator that owns the memory). It computes exactly
+ * what dq_decode_attention computes, with the same arguments minus the
+ * workspace, and allocates nothing.
+ *   Scratch: the split-K partial results go to a fixed 8 MiB array in the
+ *   library's own device memory (held by every GPU that loads the library
+ *   until the process exits). Shapes whose partial results need more than
+ *   8 MiB (see dq_decode_workspace_bytes; about 16000 rows of
+ *   B x Hq x splits) are rejected with DQ_ERR_WORKSPACE before anything is
+ *   enqueued.
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, no allocation) with that device current; make that
+ *   first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents; nothing in it needs to start at zero. Calls whose work
+ *   overlaps on the GPU (for example on two streams) race on the array and
+ *   must be ordered by the caller. */
+int dq_decode_attention_noalloc(const dq_tables *t, const void *q, int q_dtype,
+                                const uint8_t *d_kcache, const uint8_t *d_vcache,
+                                const int32_t *d_seq_lens, int B, int Hq, int Hkv,
+                                int64_t T_cap, int64_t T_max, float sm_scale,
+                                void *out, int out_dtype, dq_stats *d_stats,
+                                void *stream);
+
 /* Test hook: decodes n flat containers of one stream.
  *   d_cache   device [n][C]; d_syms device uint8 [n][128]; d_norm16 device
  *             uint16 [n]; d_status device int32 [n] (may be NULL)
