@@ -46,7 +46,7 @@ void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
   std::memset(s, 0, sizeof(*s));
   for (int sym = 0; sym < d.n_levels; ++sym)
     for (uint32_t slot = d.cum[sym]; slot < d.cum[sym + 1]; ++slot)
-      s->lut[slot] = (slot - d.cum[sym]) | (d.freq[sym] << 12) | (static_cast<uint32_t>(sym) << 24);
+      s->lut[slot] = (slot - d.cum[sym]) | (static_cast<uint32_t>(sym) << 11) | (d.freq[sym] << 20);
   for (int i = 0; i < dqi::kMaxLevels; ++i) {
     s->levels[i] = i < d.n_levels ? d.levels[i] : 0.0f;
     s->thresholds[i] = d.thresholds[i];
@@ -74,7 +74,7 @@ struct Plan {
 };
 
 Plan plan_splits(int sm_count, int B, int Hkv, int64_t T_max) {
-  const int ctas_per_sm = 2;  // residency of the split kernel
+  const int ctas_per_sm = 1;  // the split kernel runs one persistent CTA per SM
   const int64_t slots = static_cast<int64_t>(sm_count) * ctas_per_sm;
   const int64_t bh = static_cast<int64_t>(B) * Hkv;
   const int64_t min_chunk = 256;
@@ -358,6 +358,13 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const ui
     a.chunk = p.chunk;
     a.ck = t->k.container_bytes;
     a.cv = t->v.container_bytes;
+    auto has_small_freq = [](const dqi::StreamDesign &d) {
+      for (int s = 0; s < d.n_levels; ++s)
+        if (d.freq[s] < 16) return true;
+      return false;
+    };
+    a.two_k = has_small_freq(t->k);
+    a.two_v = has_small_freq(t->v);
     a.stats = d_stats;
     int e = dqi::launch_decode_attention(a, stream);
     return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));

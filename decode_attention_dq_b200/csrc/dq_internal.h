@@ -40,7 +40,8 @@ void rotation_signs(uint64_t seed, int n_heads, int8_t *out /*[n][128]*/);
 
 // Device-resident table of one stream.
 struct DevStream {
-  // Decode look-up: slot -> (slot - cum[s]) | f_s << 12 | s << 24.
+  // Decode look-up: slot -> (slot - cum[s]) | s << 11 | f_s << 20
+  // (slot - cum[s] < f_s <= 2048 fits 11 bits; f_s fits 12 bits).
   uint32_t lut[kM];
   float levels[kMaxLevels];
   float thresholds[kMaxLevels];  // n-1 used, the rest +inf
@@ -86,6 +87,7 @@ struct DecodeArgs {
   int splits;
   int64_t chunk;  // tokens per split (multiple of 32)
   int ck, cv;
+  bool two_k, two_v;  // the stream's table has a symbol with f < 16
   dq_stats *stats;
 };
 int launch_decode_attention(const DecodeArgs &a, void *stream);

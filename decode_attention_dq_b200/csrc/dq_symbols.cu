@@ -59,8 +59,8 @@ decode_symbols_kernel(const DevStream *__restrict__ tab, const uint8_t *__restri
       int i = 0;
       for (; i < kD && st == 0; ++i) {
         const uint32_t e = lut[x & (kM - 1)];
-        const uint32_t s = e >> 24;
-        x = ((e >> 12) & 0xFFFu) * (x >> kProbBits) + (e & 0xFFFu);
+        const uint32_t s = (e >> 11) & 7u;
+        x = (e >> 20) * (x >> kProbBits) + (e & 0x7FFu);
         pack |= s << (8 * (i & 3));
         for (int r = 0; r < 2 && x < kL; ++r) {
           if (pos >= C) { st = 2; break; }

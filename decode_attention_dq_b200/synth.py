@@ -48,6 +48,9 @@ WORKLOADS = {
     "tiny_b1_t256": Workload("tiny_b1_t256", 1, 1, 1, 256, "f32", "tiny", 0),
     "qwen3_8b_b16_t8k": Workload("qwen3_8b_b16_t8k", 16, 8, 32, 8192, "bf16", "llm", 1),
     "serve_b128_t8k": Workload("serve_b128_t8k", 128, 8, 32, 8192, "bf16", "llm", 2),
+    # a quarter of the serving batch: same kernel and per-sequence work, a
+    # cache (151 MB) still larger than L2, small enough for profiler captures
+    "serve_b32_t8k": Workload("serve_b32_t8k", 32, 8, 32, 8192, "bf16", "llm", 2),
     "long_b4_t64k": Workload("long_b4_t64k", 4, 8, 32, 65536, "bf16", "llm", 3),
     "long_b4_t128k": Workload("long_b4_t128k", 4, 8, 32, 131072, "bf16", "llm", 3),
     "llama_b32_t32k_1p96": Workload("llama_b32_t32k_1p96", 32, 8, 32, 32768, "bf16", "llm", 4,
