@@ -266,7 +266,6 @@ def run_dq(args):
         achieved = ops / (dec_ms * 1e-3) / 1e12
         comp_bytes = token_heads * (ck + cv)
         hbm_gbs = comp_bytes / (dec_ms * 1e-3) / 1e9
-        splits = (nbytes // (w.B * w.Hq * 4 * 130)) if nbytes else 1
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,

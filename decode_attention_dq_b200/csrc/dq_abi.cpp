@@ -4,6 +4,7 @@
 // dq_build_tables.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -42,6 +43,58 @@ int check_device(const dq_tables *t) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// IEEE binary32 -> binary16, round to nearest even (overflow to infinity).
+uint16_t f32_to_f16_rn(float f) {
+  uint32_t x;
+  std::memcpy(&x, &f, 4);
+  const uint32_t sign = (x >> 16) & 0x8000u;
+  x &= 0x7FFFFFFFu;
+  if (x >= 0x7F800000u) return static_cast<uint16_t>(sign | (x > 0x7F800000u ? 0x7E00u : 0x7C00u));
+  if (x >= 0x477FF000u) return static_cast<uint16_t>(sign | 0x7C00u);  // rounds to >= 65520
+  if (x < 0x38800000u) {  // below 2^-14: subnormal half, units of 2^-24
+    float a;
+    std::memcpy(&a, &x, 4);
+    return static_cast<uint16_t>(sign | static_cast<uint32_t>(std::nearbyint(static_cast<double>(a) * 16777216.0)));
+  }
+  uint32_t h = ((((x >> 23) - 127u + 15u) << 10) | ((x & 0x7FFFFFu) >> 13));
+  const uint32_t rem = x & 0x1FFFu;
+  if (rem > 0x1000u || (rem == 0x1000u && (h & 1u))) ++h;
+  return static_cast<uint16_t>(sign | h);
+}
+
+double f16_to_double(uint16_t h) {
+  const int e = (h >> 10) & 0x1F;
+  const int m = h & 0x3FF;
+  double v = e == 0 ? std::ldexp(static_cast<double>(m), -24) : std::ldexp(1024.0 + m, e - 25);
+  return (h & 0x8000u) ? -v : v;
+}
+
+// Scale kappa in [1, 2) (steps of 2^-16) that minimises the largest relative
+// error of fp16(kappa * level) over the non-zero levels; the smallest such
+// kappa on ties.
+void choose_tile_scale(const dqi::StreamDesign &d, dqi::DevStream *s) {
+  double best_err = INFINITY;
+  double best_k = 1.0;
+  for (int j = 0; j < 65536; ++j) {
+    const double kappa = 1.0 + j / 65536.0;
+    double err = 0.0;
+    for (int i = 0; i < d.n_levels; ++i) {
+      const double y = static_cast<double>(d.levels[i]);
+      if (y == 0.0) continue;
+      const double h = f16_to_double(f32_to_f16_rn(static_cast<float>(kappa * y)));
+      err = std::max(err, std::fabs(h - kappa * y) / std::fabs(kappa * y));
+    }
+    if (err < best_err) {
+      best_err = err;
+      best_k = kappa;
+    }
+  }
+  s->tile_scale = static_cast<float>(best_k);
+  s->tile_rel_err = static_cast<float>(best_err);
+  for (int i = 0; i < dqi::kMaxLevels; ++i)
+    s->level16[i] = i < d.n_levels ? f32_to_f16_rn(static_cast<float>(best_k * static_cast<double>(d.levels[i]))) : 0u;
+}
+
 void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
   std::memset(s, 0, sizeof(*s));
   for (int sym = 0; sym < d.n_levels; ++sym)
@@ -54,6 +107,7 @@ void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
     s->freq[i] = i < d.n_levels ? d.freq[i] : 0u;
     s->cum[i] = i < d.n_levels ? d.cum[i] : dqi::kM;
   }
+  choose_tile_scale(d, s);
   s->n_levels = d.n_levels;
   s->container_bytes = d.container_bytes;
   s->payload_bytes = d.payload_bytes;
@@ -66,46 +120,29 @@ const dqi::StreamDesign *stream_of(const dq_tables *t, int kind) {
   return nullptr;
 }
 
-// Split-K plan: chunk of tokens per CTA (a multiple of 32) and number of
-// splits, chosen so the grid fills whole waves of the SMs.
-struct Plan {
-  int splits;
-  int64_t chunk;
+// Workspace of dq_decode_attention: the token-group prefix sums, then one
+// partial-state slot per (b, h) segment of a warp's range. Slot (b Hkv + h) +
+// warp is unique, so B Hkv + (total warps) slots cover every case.
+struct WsLayout {
+  int grid = 0;
+  int64_t total_warps = 0;
+  size_t prefix_off = 0, o_off = 0, ml_off = 0, total = 0;
 };
 
-Plan plan_splits(int sm_count, int B, int Hkv, int64_t T_max) {
-  const int ctas_per_sm = 1;  // the split kernel runs one persistent CTA per SM
-  const int64_t slots = static_cast<int64_t>(sm_count) * ctas_per_sm;
-  const int64_t bh = static_cast<int64_t>(B) * Hkv;
-  const int64_t min_chunk = 256;
-  int64_t max_splits = std::max<int64_t>(1, (T_max + min_chunk - 1) / min_chunk);
-  max_splits = std::min<int64_t>(max_splits, 256);
-  Plan best{1, std::max<int64_t>(32, ((T_max + 31) / 32) * 32)};
-  double best_score = -1.0;
-  for (int64_t s = 1; s <= max_splits; ++s) {
-    int64_t chunk = ((T_max + s - 1) / s + 31) / 32 * 32;
-    if (chunk < 32) chunk = 32;
-    int64_t eff_splits = (T_max + chunk - 1) / chunk;
-    if (eff_splits != s) continue;
-    const int64_t ctas = bh * s;
-    const double waves = static_cast<double>(ctas) / slots;
-    const double fill = waves / std::ceil(waves);
-    // prefer fuller waves; among near-equal fills prefer fewer splits
-    const double score = fill - 0.002 * s;
-    if (score > best_score) {
-      best_score = score;
-      best = Plan{static_cast<int>(s), chunk};
-    }
-  }
-  if (T_max == 0) best = Plan{1, 32};
-  return best;
-}
+size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 
-size_t workspace_bytes(const Plan &p, int B, int Hq) {
-  const size_t rows = static_cast<size_t>(B) * Hq * p.splits;
-  size_t o = rows * dqi::kD * sizeof(float);
-  o = (o + 255) / 256 * 256;
-  return o + rows * 2 * sizeof(float);
+WsLayout ws_layout(const dq_tables *t, int B, int Hkv, int G) {
+  WsLayout w;
+  const int nw = dqi::decode_warps_per_cta(G, t->k.container_bytes, t->v.container_bytes);
+  if (nw <= 0) return w;
+  w.grid = t->sm_count;
+  w.total_warps = static_cast<int64_t>(w.grid) * nw;
+  const size_t slots = static_cast<size_t>(B) * Hkv + static_cast<size_t>(w.total_warps);
+  w.prefix_off = 0;
+  w.o_off = round256((static_cast<size_t>(B) + 1) * sizeof(int64_t));
+  w.ml_off = w.o_off + round256(slots * G * dqi::kD * sizeof(float));
+  w.total = w.ml_off + slots * G * 2 * sizeof(float);
+  return w;
 }
 
 }  // namespace
@@ -308,8 +345,7 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, in
 
 size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv, int64_t T_max) {
   if (!t || B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || T_max < 0) return 0;
-  const Plan p = plan_splits(t->sm_count, B, Hkv, T_max);
-  return workspace_bytes(p, B, Hq);
+  return ws_layout(t, B, Hkv, Hq / Hkv).total;
 }
 
 int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
@@ -328,8 +364,9 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const ui
         !aligned(q, 4) || !aligned(out, 4))
       return DQ_ERR_ALIGN;
     if (!std::isfinite(sm_scale)) return DQ_ERR_SHAPE;
-    const Plan p = plan_splits(t->sm_count, B, Hkv, T_max);
-    if (ws_bytes < workspace_bytes(p, B, Hq)) return DQ_ERR_WORKSPACE;
+    const WsLayout wl = ws_layout(t, B, Hkv, G);
+    if (wl.total == 0) return DQ_ERR_SHAPE;
+    if (ws_bytes < wl.total) return DQ_ERR_WORKSPACE;
     int rc = check_device(t);
     if (rc != DQ_OK) return rc;
     if (B == 0) return DQ_OK;
@@ -350,12 +387,12 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const ui
     a.sm_scale = sm_scale;
     a.out = out;
     a.out_dtype = out_dtype;
-    size_t o_bytes = static_cast<size_t>(B) * Hq * p.splits * dqi::kD * sizeof(float);
-    o_bytes = (o_bytes + 255) / 256 * 256;
-    a.ws_o = static_cast<float *>(d_workspace);
-    a.ws_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(d_workspace) + o_bytes);
-    a.splits = p.splits;
-    a.chunk = p.chunk;
+    uint8_t *ws = static_cast<uint8_t *>(d_workspace);
+    a.prefix = reinterpret_cast<int64_t *>(ws + wl.prefix_off);
+    a.ws_o = reinterpret_cast<float *>(ws + wl.o_off);
+    a.ws_ml = reinterpret_cast<float *>(ws + wl.ml_off);
+    a.grid = wl.grid;
+    a.total_warps = wl.total_warps;
     a.ck = t->k.container_bytes;
     a.cv = t->v.container_bytes;
     auto has_small_freq = [](const dqi::StreamDesign &d) {

@@ -6,24 +6,36 @@
 // Meets KV Cache at 2.26 Bits", intro: rANS decoding runs inside the attention
 // kernel; "The Numbers" 2nd paragraph: entropy decoding adds computation.
 //
-// Split kernel: one persistent CTA per SM (as many warps as shared memory
-// allows) walks over work items (sequence b, KV head h, token chunk); all
-// warps of the CTA share the decode tables and q~ of the current item.
+// Work split. The cache of sequence b, KV head h is cut into groups of 32
+// tokens (one token per lane). All groups of all (b, h) are numbered in one
+// flat order (b, then h, then token group) and every warp of the grid takes
+// an equal contiguous range of that order, so the work is balanced to one
+// group whatever the batch's lengths are. Where a warp's range crosses from
+// one (b, h) to the next it writes the partial softmax state of the first
+// and starts the next; partial states go to slot (b Hkv + h) + warp, which is
+// unique because the warps' ranges are ordered. Warps never wait on each
+// other: one persistent CTA per SM only shares the decode tables.
+//
+// Prefix kernel (one CTA): token groups per sequence and their prefix sums.
+// Split kernel, per warp and per (b, h) segment of its range:
 //   D1  q~ = H D q / 128 for the G query heads of h (times sm_scale log2 e)
-//   D2  each warp stages 32 K and 32 V containers at a time into shared
+//   D2  the warp stages 32 K and 32 V containers at a time into shared
 //       memory with 16-byte cp.async, one group ahead
 //   D3  one lane per token: rANS-decode K (table look-up, multiply-add, byte
 //       renormalisation) and accumulate q~ . y_hat for the G heads
 //   D5  in the same loop the lane decodes V of the PREVIOUS group (whose
-//       softmax weights are known) into a half-width tile of levels, so every
-//       lane runs two independent rANS chains
+//       softmax weights are known) into a half-width (64-coordinate) fp16
+//       tile of scaled levels, so every lane runs two independent rANS chains
 //   D4  online softmax per head across the warp (score * ||k||)
-//   D5' P.V from the tile: each lane accumulates 4 coordinates x G heads
-//       over 16 tokens with packed fp32 multiply-adds
-//   D6  at the end of an item the warps' (m, l, o_rot) are merged and written
-//       to the workspace
+//   D5' P.V on the tensor cores: o_rot^T[128 x G] += Y^T[128 x 32] w[32 x G]
+//       per group with warp-level m16n8k16 fp16 MMAs, fp32 accumulation.
+//       Y^T comes from the tile with ldmatrix.trans; w = p ||v|| is split
+//       into two fp16 halves (hi + lo) so it keeps fp32 precision; the
+//       levels are stored as fp16(kappa y) with a per-table kappa that makes
+//       them exact to a few 1e-5 (relative), undone in the combine
+//   D6  at the end of a segment the warp writes (m, l, o_rot) to its slot
 // Combine kernel, one warp per (b, query head):
-//   D7  log-sum-exp merge of the splits, o = D H o_rot / (128 l)
+//   D7  log-sum-exp merge of the slots of (b, h), o = D H o_rot / (128 l)
 #include <type_traits>
 
 #include "dq_device.cuh"
@@ -33,20 +45,20 @@ namespace {
 
 constexpr int kMaxWarps = 16;      // warps per CTA (one persistent CTA per SM)
 constexpr int kTile = 32;          // tokens per warp group (one per lane)
-constexpr int kHalf = 64;          // coordinates per V tile half
-constexpr int kTStride = kHalf + 4;  // V tile row stride (floats): conflict-free 128-bit access
+constexpr int kHalf = 64;          // coordinates per V tile pass
+constexpr int kTileRow = kHalf * 2;  // bytes per token row of the fp16 V tile
+constexpr int kWhStride = 40;      // halves per head row of the weight buffer
 constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ inline size_t align16(size_t v) { return (v + 15) & ~size_t(15); }
 
-// Shared-memory layout of the split kernel. Everything a CTA shares (decode
-// tables, q~) comes first; each warp then owns its staging slots, V tile and
-// softmax-weight buffer.
+// Shared-memory layout of the split kernel: the decode tables shared by the
+// CTA, then one area per warp with its staging slots, V tile, softmax-weight
+// buffer (fp16 hi and lo, [2][8 heads][kWhStride]) and q~.
 struct SplitSmem {
-  size_t lut_k, lut_v, lev, qt, warp0, warp_bytes;
-  size_t kst, vst, tile, wbuf;  // offsets inside a warp's area
+  size_t lut_k, lut_v, lev, warp0, warp_bytes;
+  size_t kst, vst, tile, wbuf, qt;  // offsets inside a warp's area
   size_t total;
-  int nwarps;
 };
 
 __host__ __device__ inline SplitSmem split_smem_layout(int G, int ck, int cv, int nwarps) {
@@ -54,14 +66,13 @@ __host__ __device__ inline SplitSmem split_smem_layout(int G, int ck, int cv, in
   s.lut_k = 0;
   s.lut_v = s.lut_k + kM * 4;
   s.lev = s.lut_v + kM * 4;
-  s.qt = s.lev + 2 * kMaxLevels * 4;
-  s.warp0 = align16(s.qt + static_cast<size_t>(kD) * G * 4);
+  s.warp0 = align16(s.lev + 2 * kMaxLevels * 4);
   s.kst = 0;                                                        // 2 slots of 32 K containers
   s.vst = align16(2 * static_cast<size_t>(kTile) * ck);             // 2 slots of 32 V containers
-  s.tile = s.vst + align16(2 * static_cast<size_t>(kTile) * cv);    // [32][kTStride] floats
-  s.wbuf = s.tile + static_cast<size_t>(kTile) * kTStride * 4;      // [32][G] floats
-  s.warp_bytes = align16(s.wbuf + static_cast<size_t>(kTile) * G * 4);
-  s.nwarps = nwarps;
+  s.tile = s.vst + align16(2 * static_cast<size_t>(kTile) * cv);    // [32 tokens][64] fp16, swizzled
+  s.wbuf = s.tile + static_cast<size_t>(kTile) * kTileRow;          // [2][8][kWhStride] fp16
+  s.qt = s.wbuf + 2 * 8 * kWhStride * 2;                            // [128][G] floats
+  s.warp_bytes = align16(s.qt + static_cast<size_t>(kD) * G * 4);
   // 256 bytes of slack: a corrupt container can make its decoder read up to
   // 2 bytes per symbol past its start; those reads stay inside the CTA's
   // shared memory and only produce garbage (flagged by the final-state check).
@@ -151,39 +162,54 @@ __device__ __forceinline__ void score_fma(float (&sc)[G], const float *qi, float
   }
 }
 
-// Per-warp state of one work item's online softmax and P.V accumulators.
-// Lane l accumulates coordinates 4 (l & 15) .. +3 of each 64-coordinate half
-// over the tokens of its half-group (l >> 4); the two half-groups are summed
-// at the end of the item.
+// Byte offset in the V tile of token t's 16-byte chunk c (8 coordinates):
+// chunks are XOR-swizzled by t & 7, so a lane's 128-bit store of its own row
+// and an 8-row ldmatrix both touch 8 different 16-byte bank groups.
+__device__ __forceinline__ uint32_t tile_off(int t, int c) {
+  return static_cast<uint32_t>(t * kTileRow + ((c ^ (t & 7)) << 4));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t saddr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(saddr)
+               : "memory");
+}
+
+// d += a b for one m16n8k16 tile: fp16 operands, fp32 accumulators.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Per-warp state of one segment's online softmax and P.V accumulators. The
+// accumulators are the m16n8 C fragments of o_rot^T: c[mt] covers
+// coordinates 16 mt .. 16 mt + 15; lane l holds coordinates 16 mt + l / 4
+// (+ 8) of heads 2 (l % 4) and 2 (l % 4) + 1 (heads >= G stay zero).
 template <int G>
 struct WarpAcc {
   float m[G], l[G];
-  float2 o[2][G][2];  // [half][head][coordinate pair]: coordinates 4q + {0,1} and 4q + {2,3}
+  float c[kD / 16][4];
 };
 
-template <int G, int half>
-__device__ __forceinline__ void pv_half(WarpAcc<G> &acc, const float *tile, const float *wbuf, int lane) {
-  const int th = lane >> 4, q = lane & 15;
-#pragma unroll 4
-  for (int kk = 0; kk < 16; ++kk) {
-    const int t = th * 16 + kk;
-    const float4 y = *reinterpret_cast<const float4 *>(tile + t * kTStride + 4 * q);
-    float w[G];
-    if constexpr (G % 4 == 0) {
+// P.V for one 64-coordinate half of the current group: A = Y^T (16
+// coordinates x 16 tokens) by ldmatrix.trans from the tile, B = the group's
+// weights (16 tokens x 8 heads) as fp16 hi and lo fragments.
+template <int half>
+__device__ __forceinline__ void pv_mma_half(float (&c)[kD / 16][4], uint32_t tile_s, const uint32_t (&bh)[2][2],
+                                            const uint32_t (&bl)[2][2], int lane) {
+  const int r = (lane & 7) + ((lane >> 4) & 1) * 8;  // token row within a 16-token step
+  const int cadd = (lane >> 3) & 1;                   // second 8 coordinates of the m-tile
 #pragma unroll
-      for (int g4 = 0; g4 < G; g4 += 4) {
-        const float4 ww = *reinterpret_cast<const float4 *>(wbuf + t * G + g4);
-        w[g4] = ww.x; w[g4 + 1] = ww.y; w[g4 + 2] = ww.z; w[g4 + 3] = ww.w;
-      }
-    } else {
+  for (int ks = 0; ks < 2; ++ks) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) w[g] = wbuf[t * G + g];
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float2 wg = make_float2(w[g], w[g]);
-      acc.o[half][g][0] = __ffma2_rn(make_float2(y.x, y.y), wg, acc.o[half][g][0]);
-      acc.o[half][g][1] = __ffma2_rn(make_float2(y.z, y.w), wg, acc.o[half][g][1]);
+    for (int mt = 0; mt < 4; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_trans(a, tile_s + tile_off(ks * 16 + r, 2 * mt + cadd));
+      mma_16816(c[half * 4 + mt], a, bh[ks][0], bh[ks][1]);
+      mma_16816(c[half * 4 + mt], a, bl[ks][0], bl[ks][1]);
     }
   }
 }
@@ -192,25 +218,92 @@ __device__ __forceinline__ void pv_half(WarpAcc<G> &acc, const float *tile, cons
 // probabilities p (without the V norm) in `p` for the caller.
 template <int G>
 __device__ __forceinline__ void softmax_update(WarpAcc<G> &acc, const float (&sc)[G], float nk, bool valid,
-                                               float (&p)[G]) {
+                                               float (&p)[G], int lane) {
+  float alpha[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const float s = valid ? sc[g] * nk : -INFINITY;
     const float m_new = fmaxf(acc.m[g], warp_max(s));
-    float alpha = 1.0f;
+    alpha[g] = 1.0f;
     p[g] = 0.0f;
     if (m_new != -INFINITY) {
       p[g] = exp2f(s - m_new);
-      alpha = exp2f(acc.m[g] - m_new);
+      alpha[g] = exp2f(acc.m[g] - m_new);
     }
-    acc.l[g] = acc.l[g] * alpha + warp_sum(p[g]);
+    acc.l[g] = acc.l[g] * alpha[g] + warp_sum(p[g]);
     acc.m[g] = m_new;
-    const float2 a2 = make_float2(alpha, alpha);
+  }
+  // This lane's accumulators belong to heads 2 (lane % 4) and 2 (lane % 4) + 1.
+  float aa = 1.0f, ab = 1.0f;
+  const int cq = lane & 3;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      acc.o[h][g][0] = __fmul2_rn(acc.o[h][g][0], a2);
-      acc.o[h][g][1] = __fmul2_rn(acc.o[h][g][1], a2);
+  for (int g2 = 0; 2 * g2 < G; ++g2)
+    if (cq == g2) {
+      aa = alpha[2 * g2];
+      ab = (2 * g2 + 1 < G) ? alpha[2 * g2 + 1] : 1.0f;
     }
+  const float2 a2 = make_float2(aa, ab);
+#pragma unroll
+  for (int mt = 0; mt < kD / 16; ++mt) {
+    const float2 lo = __fmul2_rn(make_float2(acc.c[mt][0], acc.c[mt][1]), a2);
+    const float2 hi = __fmul2_rn(make_float2(acc.c[mt][2], acc.c[mt][3]), a2);
+    acc.c[mt][0] = lo.x; acc.c[mt][1] = lo.y; acc.c[mt][2] = hi.x; acc.c[mt][3] = hi.y;
+  }
+}
+
+__device__ __forceinline__ int64_t clamp_len(int32_t len, int64_t cap) {
+  int64_t v = len;
+  if (v < 0) v = 0;
+  if (v > cap) v = cap;
+  return v;
+}
+
+// First flat group index of warp w out of W over N groups (warp w owns
+// [first(w), first(w + 1))).
+__host__ __device__ __forceinline__ int64_t warp_first(int64_t w, int64_t W, int64_t N) { return (w * N) / W; }
+
+// Token groups per sequence and their prefix sums: prefix[b] = groups of
+// sequences 0..b-1, prefix[B] = total. One CTA of kPrefixThreads threads;
+// also counts the sequence lengths that had to be clamped.
+constexpr int kPrefixThreads = 1024;
+
+__global__ void __launch_bounds__(kPrefixThreads) prefix_kernel(const DecodeArgs a) {
+  __shared__ int64_t warp_tot[kPrefixThreads / 32];
+  __shared__ int64_t carry_s;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t cap = a.T_max < a.T_cap ? a.T_max : a.T_cap;
+  if (threadIdx.x == 0) {
+    carry_s = 0;
+    a.prefix[0] = 0;
+  }
+  unsigned clamped = 0;
+  __syncthreads();
+  for (int base = 0; base < a.B; base += kPrefixThreads) {
+    const int i = base + static_cast<int>(threadIdx.x);
+    int64_t v = 0;
+    if (i < a.B) {
+      const int32_t len = a.seq_lens[i];
+      if (len < 0 || len > cap) ++clamped;
+      v = (clamp_len(len, cap) + kTile - 1) / kTile;
+    }
+    int64_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t nb = __shfl_up_sync(kFull, inc, o);
+      if (lane >= o) inc += nb;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int64_t before = carry_s;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    if (i < a.B) a.prefix[i + 1] = before + inc;
+    __syncthreads();  // everyone has read carry_s and warp_tot
+    if (threadIdx.x == kPrefixThreads - 1) carry_s = before + inc;
+    __syncthreads();
+  }
+  if (a.stats) {
+    const unsigned c = static_cast<unsigned>(warp_sum(static_cast<float>(clamped)));
+    if (lane == 0 && c) atomicAdd(&a.stats->clamped_lengths, static_cast<unsigned long long>(c));
   }
 }
 
@@ -225,14 +318,15 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
   const SplitSmem L = split_smem_layout(G, a.ck, a.cv, nwarps);
   uint32_t *lut_k = reinterpret_cast<uint32_t *>(smem + L.lut_k);
   uint32_t *lut_v = reinterpret_cast<uint32_t *>(smem + L.lut_v);
-  float *lev = reinterpret_cast<float *>(smem + L.lev);  // [0..7] K, [8..15] V
-  float *qt = reinterpret_cast<float *>(smem + L.qt);    // [128][G]
+  float *lev = reinterpret_cast<float *>(smem + L.lev);  // [0..7] K levels, [8..15] V fp16 bits
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint8_t *wsm = smem + L.warp0 + warp * L.warp_bytes;
   uint8_t *kst = wsm + L.kst;
   uint8_t *vst = wsm + L.vst;
-  float *tile = reinterpret_cast<float *>(wsm + L.tile);
-  float *wbuf = reinterpret_cast<float *>(wsm + L.wbuf);
+  const uint32_t tile_s = static_cast<uint32_t>(__cvta_generic_to_shared(wsm + L.tile));
+  uint16_t *wh = reinterpret_cast<uint16_t *>(wsm + L.wbuf);  // [hi, lo][8 heads][kWhStride]
+  const uint32_t *whw = reinterpret_cast<const uint32_t *>(wh);
+  float *qt = reinterpret_cast<float *>(wsm + L.qt);  // [128][G]
   const int ck = a.ck, cv = a.cv;
 
   // Decode tables into shared memory (once per CTA).
@@ -247,224 +341,235 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
     }
     if (threadIdx.x < kMaxLevels) {
       lev[threadIdx.x] = a.tabs->k.levels[threadIdx.x];
-      lev[kMaxLevels + threadIdx.x] = a.tabs->v.levels[threadIdx.x];
+      reinterpret_cast<uint32_t *>(lev)[kMaxLevels + threadIdx.x] = a.tabs->v.level16[threadIdx.x];
     }
   }
-  const int S = a.splits;
-  const int64_t n_items = static_cast<int64_t>(a.B) * a.Hkv * S;
+  __syncthreads();
+
   const int64_t cap = a.T_max < a.T_cap ? a.T_max : a.T_cap;
+  const int64_t Hkv = a.Hkv;
+  const int64_t N = a.prefix[a.B] * Hkv;  // total token groups
+  const int64_t W = static_cast<int64_t>(gridDim.x) * nwarps;
+  const int64_t wid = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
+  int64_t g = warp_first(wid, W, N);
+  const int64_t g_end = warp_first(wid + 1, W, N);
+  if (g >= g_end) return;
   unsigned bad_count = 0;
 
-  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int bh = static_cast<int>(item / S);
-    const int split = static_cast<int>(item % S);
-    const int b = bh / a.Hkv, h = bh % a.Hkv;
-    int64_t len = a.seq_lens[b];
-    if (len < 0) len = 0;
-    if (len > cap) len = cap;
-    const int64_t c0 = static_cast<int64_t>(split) * a.chunk;
-    const int64_t c1 = (c0 + a.chunk) < len ? (c0 + a.chunk) : len;
-    const int64_t ngroups = (c1 > c0) ? (c1 - c0 + kTile - 1) / kTile : 0;
+  // Sequence holding flat group g: the largest b with prefix[b] * Hkv <= g
+  // (it has tokens, since g < prefix[b + 1] * Hkv).
+  int b = 0;
+  {
+    int lo = 0, hi = a.B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.prefix[mid] * Hkv <= g) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+  }
+  int64_t gb = a.prefix[b + 1] - a.prefix[b];  // token groups per head of sequence b
+  int h = static_cast<int>((g - a.prefix[b] * Hkv) / gb);
+  int64_t j0 = (g - a.prefix[b] * Hkv) % gb;
 
-    __syncthreads();  // previous item's merge area and q~ are no longer in use
+  while (true) {
+    const int64_t n = (g_end - g) < (gb - j0) ? (g_end - g) : (gb - j0);  // groups in this segment
+    const int64_t len = clamp_len(a.seq_lens[b], cap);
+    const int64_t bh = static_cast<int64_t>(b) * Hkv + h;
+
     // D1: q~ = H D q / 128 for the G query heads of KV head h, times sm_scale log2 e.
     {
       uint32_t sw[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
       const float qscale = a.sm_scale * kLog2e / static_cast<float>(kD);
-      for (int g = warp; g < G; g += nwarps) {
-        const int64_t qbase = (static_cast<int64_t>(b) * a.Hq + h * G + g) * kD;
+#pragma unroll 1
+      for (int gg = 0; gg < G; ++gg) {
+        const int64_t qbase = (static_cast<int64_t>(b) * a.Hq + h * G + gg) * kD;
         float v[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) v[k] = apply_sign(load_elem(a.q, qbase + lane + 32 * k, a.q_dtype), sw[k], lane);
         wht128_warp(v, lane);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) qt[(lane + 32 * k) * G + g] = v[k] * qscale;
+        for (int k = 0; k < 4; ++k) qt[(lane + 32 * k) * G + gg] = v[k] * qscale;
       }
     }
-    __syncthreads();
 
-    const uint8_t *krow = a.kcache + static_cast<int64_t>(bh) * a.T_cap * ck;
-    const uint8_t *vrow = a.vcache + static_cast<int64_t>(bh) * a.T_cap * cv;
-    auto group_t0 = [&](int64_t j) { return c0 + (warp + j * nwarps) * kTile; };
-    const int64_t nmine = (ngroups > warp) ? (ngroups - warp + nwarps - 1) / nwarps : 0;
+    const uint8_t *krow = a.kcache + bh * a.T_cap * ck;
+    const uint8_t *vrow = a.vcache + bh * a.T_cap * cv;
+    const int64_t tseg = j0 * kTile;
+    auto group_t0 = [&](int64_t j) { return tseg + j * kTile; };
     auto ncopy = [&](int64_t t0) { return (a.T_cap - t0) < kTile ? static_cast<int>(a.T_cap - t0) : kTile; };
 
     WarpAcc<G> acc;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      acc.m[g] = -INFINITY;
-      acc.l[g] = 0.0f;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        acc.o[hh][g][0] = make_float2(0.0f, 0.0f);
-        acc.o[hh][g][1] = make_float2(0.0f, 0.0f);
-      }
+    for (int gg = 0; gg < G; ++gg) {
+      acc.m[gg] = -INFINITY;
+      acc.l[gg] = 0.0f;
     }
+#pragma unroll
+    for (int mt = 0; mt < kD / 16; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc.c[mt][e] = 0.0f;
 
-    if (nmine > 0) {
-      // Prologue: K(0), V(0) into slot 0 and K(1) into K slot 1. Invariant at
-      // the top of iteration j: V(j) sits in V slot j%2 and K(j+1) in K slot
-      // (j+1)%2, both complete; iteration j prefetches K(j+2) and V(j+1).
+    // Prologue: K(0), V(0) into slot 0 and K(1) into K slot 1. Invariant at
+    // the top of iteration j: V(j) sits in V slot j%2 and K(j+1) in K slot
+    // (j+1)%2, both complete; iteration j prefetches K(j+2) and V(j+1).
+    {
+      const int64_t t0 = group_t0(0);
+      stage_group(kst, krow, t0, ncopy(t0), ck, lane);
+      stage_group(vst, vrow, t0, ncopy(t0), cv, lane);
+      if (n > 1) {
+        const int64_t t1 = group_t0(1);
+        stage_group(kst + kTile * ck, krow, t1, ncopy(t1), ck, lane);
+      }
+      cp_async_commit();
+      cp_async_wait_0();
+      __syncwarp();  // staged bytes and q~ visible to the whole warp
+    }
+    // K pass of group 0 on its own.
+    float sc[G], p[G];
+    {
+      const uint8_t *kb = kst + lane * ck;
+      RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) sc[gg] = 0.0f;
+#pragma unroll 4
+      for (int i = 0; i < kD; ++i) {
+        const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
+        const float yk = *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(lev) + ek);
+        score_fma<G>(sc, qt + i * G, yk);
+      }
+      const bool valid = group_t0(0) + lane < len;
+      bad_count += __popc(__ballot_sync(kFull, valid && rk.x != kL));
+      softmax_update(acc, sc, norm_of(kb), valid, p, lane);
+    }
+    for (int64_t j = 0; j < n; ++j) {
+      const int cur = static_cast<int>(j & 1), nxt = cur ^ 1;
+      const bool has_next = j + 1 < n;
+      // V(j) is in slot cur, K(j+1) in slot nxt (both staged). Weights of
+      // group j, w = p ||v||, as fp16 hi + lo, then this lane's B fragments:
+      // b[ks][0] holds tokens 16 ks + 2 (lane % 4) + {0, 1} of head lane / 4,
+      // b[ks][1] the same tokens + 8 (zero for heads >= G).
+      uint32_t fb_hi[2][2], fb_lo[2][2];
       {
-        const int64_t t0 = group_t0(0);
-        stage_group(kst, krow, t0, ncopy(t0), ck, lane);
-        stage_group(vst, vrow, t0, ncopy(t0), cv, lane);
-        if (nmine > 1) {
-          const int64_t t1 = group_t0(1);
-          stage_group(kst + kTile * ck, krow, t1, ncopy(t1), ck, lane);
+        const uint8_t *vb = vst + cur * kTile * cv + lane * cv;
+        const bool valid = group_t0(j) + lane < len;
+        const float nv = norm_of(vb);
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) {
+          const float w = valid ? p[gg] * nv : 0.0f;
+          const __half hi = __float2half_rn(w);
+          const __half lo = __float2half_rn(w - __half2float(hi));
+          wh[gg * kWhStride + lane] = __half_as_ushort(hi);
+          wh[(8 + gg) * kWhStride + lane] = __half_as_ushort(lo);
         }
-        cp_async_commit();
+        __syncwarp();
+        const int n_head = lane >> 2, cq = lane & 3;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int word = n_head * (kWhStride / 2) + ks * 8 + r * 4 + cq;
+            fb_hi[ks][r] = n_head < G ? whw[word] : 0u;
+            fb_lo[ks][r] = n_head < G ? whw[8 * (kWhStride / 2) + word] : 0u;
+          }
+      }
+      // Prefetch K(j+2) into slot cur and V(j+1) into slot nxt.
+      if (j + 2 < n) {
+        const int64_t t2 = group_t0(j + 2);
+        stage_group(kst + cur * kTile * ck, krow, t2, ncopy(t2), ck, lane);
+      }
+      if (has_next) {
+        const int64_t t1 = group_t0(j + 1);
+        stage_group(vst + nxt * kTile * cv, vrow, t1, ncopy(t1), cv, lane);
+      }
+      cp_async_commit();
+
+      const uint8_t *kb = kst + nxt * kTile * ck + lane * ck;
+      const uint8_t *vb = vst + cur * kTile * cv + lane * cv;
+      RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
+      RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
+#pragma unroll
+      for (int gg = 0; gg < G; ++gg) sc[gg] = 0.0f;
+      const uint32_t *lev16 = reinterpret_cast<const uint32_t *>(lev + kMaxLevels);
+      auto run_half = [&](auto half_c) {
+        constexpr int half = decltype(half_c)::value;
+#pragma unroll 1
+        for (int i8 = 0; i8 < kHalf; i8 += 8) {
+          uint32_t hv[8];
+          if (has_next) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = half * kHalf + i8 + u;
+              const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
+              const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
+              const float yk = *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(lev) + ek);
+              hv[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev16) + ev);
+              score_fma<G>(sc, qt + i * G, yk);
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
+              hv[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev16) + ev);
+            }
+          }
+          const uint4 pk = make_uint4(__byte_perm(hv[0], hv[1], 0x5410), __byte_perm(hv[2], hv[3], 0x5410),
+                                      __byte_perm(hv[4], hv[5], 0x5410), __byte_perm(hv[6], hv[7], 0x5410));
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(tile_s + tile_off(lane, i8 >> 3)),
+                       "r"(pk.x), "r"(pk.y), "r"(pk.z), "r"(pk.w)
+                       : "memory");
+        }
+        __syncwarp();
+        pv_mma_half<half>(acc.c, tile_s, fb_hi, fb_lo, lane);
+        __syncwarp();
+      };
+      run_half(std::integral_constant<int, 0>{});
+      run_half(std::integral_constant<int, 1>{});
+      {
+        const bool vvalid = group_t0(j) + lane < len;
+        bad_count += __popc(__ballot_sync(kFull, vvalid && rv.x != kL));
+      }
+      if (has_next) {
+        const bool valid = group_t0(j + 1) + lane < len;
+        bad_count += __popc(__ballot_sync(kFull, valid && rk.x != kL));
+        softmax_update(acc, sc, norm_of(kb), valid, p, lane);
+        // The next iteration needs V(j+1) (slot nxt) and K(j+2) (slot cur).
         cp_async_wait_0();
         __syncwarp();
       }
-      // K pass of group 0 on its own.
-      float sc[G], p[G];
-      {
-        const uint8_t *kb = kst + lane * ck;
-        RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
-#pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] = 0.0f;
-#pragma unroll 4
-        for (int i = 0; i < kD; ++i) {
-          const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
-          const float yk = *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(lev) + ek);
-          score_fma<G>(sc, qt + i * G, yk);
-        }
-        const bool valid = group_t0(0) + lane < c1;
-        bad_count += __popc(__ballot_sync(kFull, valid && rk.x != kL));
-        softmax_update(acc, sc, norm_of(kb), valid, p);
-      }
-      for (int64_t j = 0; j < nmine; ++j) {
-        const int cur = static_cast<int>(j & 1), nxt = cur ^ 1;
-        const bool has_next = j + 1 < nmine;
-        // V(j) is in slot cur, K(j+1) in slot nxt (both staged). Weights of group j:
-        {
-          const uint8_t *vb = vst + cur * kTile * cv + lane * cv;
-          const bool valid = group_t0(j) + lane < c1;
-          const float nv = norm_of(vb);
-#pragma unroll
-          for (int g = 0; g < G; ++g) wbuf[lane * G + g] = valid ? p[g] * nv : 0.0f;
-        }
-        __syncwarp();
-        // Prefetch K(j+2) into slot cur and V(j+1) into slot nxt.
-        if (j + 2 < nmine) {
-          const int64_t t2 = group_t0(j + 2);
-          stage_group(kst + cur * kTile * ck, krow, t2, ncopy(t2), ck, lane);
-        }
-        if (has_next) {
-          const int64_t t1 = group_t0(j + 1);
-          stage_group(vst + nxt * kTile * cv, vrow, t1, ncopy(t1), cv, lane);
-        }
-        cp_async_commit();
-
-        const uint8_t *kb = kst + nxt * kTile * ck + lane * ck;
-        const uint8_t *vb = vst + cur * kTile * cv + lane * cv;
-        RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
-        RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
-#pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] = 0.0f;
-        float *trow = tile + lane * kTStride;
-        auto run_half = [&](auto half_c) {
-          constexpr int half = decltype(half_c)::value;
-          if (has_next) {
-#pragma unroll 2
-            for (int i4 = 0; i4 < kHalf; i4 += 4) {
-              float yv[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int i = half * kHalf + i4 + u;
-                const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
-                const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
-                const float yk = *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(lev) + ek);
-                yv[u] = *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(lev + kMaxLevels) + ev);
-                score_fma<G>(sc, qt + i * G, yk);
-              }
-              *reinterpret_cast<float4 *>(trow + i4) = make_float4(yv[0], yv[1], yv[2], yv[3]);
-            }
-          } else {
-#pragma unroll 2
-            for (int i4 = 0; i4 < kHalf; i4 += 4) {
-              float yv[4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
-                yv[u] = *reinterpret_cast<const float *>(reinterpret_cast<const uint8_t *>(lev + kMaxLevels) + ev);
-              }
-              *reinterpret_cast<float4 *>(trow + i4) = make_float4(yv[0], yv[1], yv[2], yv[3]);
-            }
-          }
-          __syncwarp();
-          pv_half<G, half>(acc, tile, wbuf, lane);
-          __syncwarp();
-        };
-        run_half(std::integral_constant<int, 0>{});
-        run_half(std::integral_constant<int, 1>{});
-        {
-          const bool vvalid = group_t0(j) + lane < c1;
-          bad_count += __popc(__ballot_sync(kFull, vvalid && rv.x != kL));
-        }
-        if (has_next) {
-          const bool valid = group_t0(j + 1) + lane < c1;
-          bad_count += __popc(__ballot_sync(kFull, valid && rk.x != kL));
-          softmax_update(acc, sc, norm_of(kb), valid, p);
-          // The next iteration needs V(j+1) (slot nxt) and K(j+2) (slot cur).
-          cp_async_wait_0();
-          __syncwarp();
-        }
-      }
-      cp_async_wait_0();
     }
-    // Sum the two half-groups of tokens.
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          acc.o[hh][g][c2].x += __shfl_xor_sync(kFull, acc.o[hh][g][c2].x, 16);
-          acc.o[hh][g][c2].y += __shfl_xor_sync(kFull, acc.o[hh][g][c2].y, 16);
-        }
+    cp_async_wait_0();
+    __syncwarp();  // staging and q~ areas are free for the next segment
 
-    // D6: merge the warps' partial softmax states.
-    __syncthreads();
-    float *mrg_m = reinterpret_cast<float *>(smem + L.warp0);  // [nwarps][G]
-    float *mrg_l = mrg_m + nwarps * G;                          // [nwarps][G]
-    float *mrg_o = mrg_l + nwarps * G;                          // [nwarps][G][128]
+    // D6: write this segment's state (o_rot in units of the V tile scale).
+    const int64_t slot = bh + wid;
     if (lane == 0)
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        mrg_m[warp * G + g] = acc.m[g];
-        mrg_l[warp * G + g] = acc.l[g];
-      }
-    if (lane < 16)
+      for (int gg = 0; gg < G; ++gg)
+        *reinterpret_cast<float2 *>(a.ws_ml + (slot * G + gg) * 2) = make_float2(acc.m[gg], acc.l[gg]);
+    {
+      const int row = lane >> 2, head0 = 2 * (lane & 3);
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
+      for (int mt = 0; mt < kD / 16; ++mt)
 #pragma unroll
-        for (int g = 0; g < G; ++g)
-          *reinterpret_cast<float4 *>(mrg_o + (warp * G + g) * kD + hh * kHalf + 4 * lane) =
-              make_float4(acc.o[hh][g][0].x, acc.o[hh][g][0].y, acc.o[hh][g][1].x, acc.o[hh][g][1].y);
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < G * kD; idx += blockDim.x) {
-      const int g = idx / kD, c = idx % kD;
-      float M = -INFINITY;
-      for (int w = 0; w < nwarps; ++w) M = fmaxf(M, mrg_m[w * G + g]);
-      float o = 0.0f, l = 0.0f;
-      if (M != -INFINITY)
-        for (int w = 0; w < nwarps; ++w) {
-          const float mw = mrg_m[w * G + g];
-          if (mw == -INFINITY) continue;
-          const float sc = exp2f(mw - M);
-          o = fmaf(sc, mrg_o[(w * G + g) * kD + c], o);
-          l = fmaf(sc, mrg_l[w * G + g], l);
+        for (int e = 0; e < 4; ++e) {
+          const int head = head0 + (e & 1);
+          if (head < G) a.ws_o[(slot * G + head) * kD + 16 * mt + row + 8 * (e >> 1)] = acc.c[mt][e];
         }
-      const int64_t row = (static_cast<int64_t>(b) * a.Hq + h * G + g) * S + split;
-      a.ws_o[row * kD + c] = o;
-      if (c == 0) {
-        a.ws_ml[row * 2] = M;
-        a.ws_ml[row * 2 + 1] = l;
-      }
+    }
+
+    g += n;
+    if (g >= g_end) break;
+    // Next segment: the following head of b, else the next sequence with tokens.
+    j0 = 0;
+    if (++h == a.Hkv) {
+      h = 0;
+      do {
+        ++b;
+      } while (a.prefix[b + 1] == a.prefix[b]);
+      gb = a.prefix[b + 1] - a.prefix[b];
     }
   }
   if (a.stats && lane == 0 && bad_count) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(bad_count));
@@ -475,27 +580,42 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a) {
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);  // b * Hq + hq
   if (row >= static_cast<int64_t>(a.B) * a.Hq) return;
   const int b = static_cast<int>(row / a.Hq), hq = static_cast<int>(row % a.Hq);
-  const int h = hq / a.G;
-  const int S = a.splits;
-  if (hq == 0 && lane == 0 && a.stats) {
-    const int64_t len = a.seq_lens[b];
-    const int64_t cap = a.T_max < a.T_cap ? a.T_max : a.T_cap;
-    if (len < 0 || len > cap) atomicAdd(&a.stats->clamped_lengths, 1ull);
-  }
+  const int G = a.G;
+  const int h = hq / G, gg = hq % G;
+  const int64_t Hkv = a.Hkv;
+  const int64_t N = a.prefix[a.B] * Hkv;
+  const int64_t W = a.total_warps;
+  const int64_t gb = a.prefix[b + 1] - a.prefix[b];
+  const int64_t bh = static_cast<int64_t>(b) * Hkv + h;
   float M = -INFINITY;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, a.ws_ml[(row * S + s) * 2]);
   float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   float Ls = 0.0f;
-  if (M != -INFINITY)
-    for (int s = 0; s < S; ++s) {
-      const float ms = a.ws_ml[(row * S + s) * 2];
-      if (ms == -INFINITY) continue;
-      const float sc = exp2f(ms - M);
-      Ls = fmaf(sc, a.ws_ml[(row * S + s) * 2 + 1], Ls);
+  if (gb > 0) {
+    // Warps whose ranges cover groups [g0, g1) of (b, h): from the warp
+    // holding g0 to the warp holding g1 - 1 (the warp holding g is the
+    // largest w with first(w) <= g), skipping warps with empty ranges.
+    const int64_t g0 = a.prefix[b] * Hkv + h * gb, g1 = g0 + gb;
+    const int64_t w_lo = ((g0 + 1) * W - 1) / N;
+    const int64_t w_hi = (g1 * W - 1) / N;
+    auto covers = [&](int64_t w) {
+      const int64_t s = warp_first(w, W, N), e = warp_first(w + 1, W, N);
+      return s < e && s < g1 && e > g0;
+    };
+    for (int64_t w = w_lo; w <= w_hi; ++w)
+      if (covers(w)) M = fmaxf(M, a.ws_ml[((bh + w) * G + gg) * 2]);
+    if (M != -INFINITY)
+      for (int64_t w = w_lo; w <= w_hi; ++w) {
+        if (!covers(w)) continue;
+        const int64_t slot = bh + w;
+        const float ms = a.ws_ml[(slot * G + gg) * 2];
+        if (ms == -INFINITY) continue;
+        const float sc = exp2f(ms - M);
+        Ls = fmaf(sc, a.ws_ml[(slot * G + gg) * 2 + 1], Ls);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) v[k] = fmaf(sc, a.ws_o[(row * S + s) * kD + lane + 32 * k], v[k]);
-    }
-  const float inv = (Ls > 0.0f) ? 1.0f / (Ls * static_cast<float>(kD)) : 0.0f;
+        for (int k = 0; k < 4; ++k) v[k] = fmaf(sc, a.ws_o[(slot * G + gg) * kD + lane + 32 * k], v[k]);
+      }
+  }
+  const float inv = (Ls > 0.0f) ? 1.0f / (Ls * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
   wht128_warp(v, lane);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -514,18 +634,12 @@ int warps_for(int G, int ck, int cv) {
 template <int G, bool kTwoK, bool kTwoV>
 int launch_split(const DecodeArgs &a, cudaStream_t st) {
   const int nw = warps_for(G, a.ck, a.cv);
+  if (static_cast<int64_t>(a.grid) * nw != a.total_warps) return static_cast<int>(cudaErrorInvalidValue);
   const SplitSmem L = split_smem_layout(G, a.ck, a.cv, nw);
   auto kern = decode_split_kernel<G, kTwoK, kTwoV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
   if (e != cudaSuccess) return static_cast<int>(e);
-  int dev = 0, sms = 0;
-  e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return static_cast<int>(e);
-  const int64_t items = static_cast<int64_t>(a.B) * a.Hkv * a.splits;
-  const int grid = static_cast<int>(items < sms ? items : sms);
-  if (grid <= 0) return 0;
-  kern<<<grid, nw * 32, L.total, st>>>(a);
+  kern<<<a.grid, nw * 32, L.total, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -539,9 +653,18 @@ int launch_split_g(const DecodeArgs &a, cudaStream_t st) {
 
 }  // namespace
 
+int decode_warps_per_cta(int G, int ck, int cv) {
+  if (G != 1 && G != 2 && G != 4 && G != 8) return 0;
+  if (ck < 1 || cv < 1 || ck > kMaxContainer || cv > kMaxContainer) return 0;
+  return warps_for(G, ck, cv);
+}
+
 int launch_decode_attention(const DecodeArgs &a, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (a.ck > kMaxContainer || a.cv > kMaxContainer) return static_cast<int>(cudaErrorInvalidValue);
+  if (a.ck > kMaxContainer || a.cv > kMaxContainer || a.grid < 1) return static_cast<int>(cudaErrorInvalidValue);
+  prefix_kernel<<<1, kPrefixThreads, 0, st>>>(a);
+  const cudaError_t ce = cudaGetLastError();
+  if (ce != cudaSuccess) return static_cast<int>(ce);
   int e = 0;
   switch (a.G) {
     case 1: e = launch_split_g<1>(a, st); break;

@@ -38,8 +38,9 @@ int design_stream(int n_levels, int container_bytes, double rate_offset,
 int container_bytes_for(double bits_per_value);
 void rotation_signs(uint64_t seed, int n_heads, int8_t *out /*[n][128]*/);
 
-// Device-resident table of one stream.
-struct DevStream {
+// Device-resident table of one stream. Kernels copy `lut` with 16-byte
+// loads, so the struct keeps a 16-byte multiple size inside DevTables.
+struct alignas(16) DevStream {
   // Decode look-up: slot -> (slot - cum[s]) | s << 11 | f_s << 20
   // (slot - cum[s] < f_s <= 2048 fits 11 bits; f_s fits 12 bits).
   uint32_t lut[kM];
@@ -48,12 +49,19 @@ struct DevStream {
   float cost[kMaxLevels];
   uint32_t freq[kMaxLevels];
   uint32_t cum[kMaxLevels];
+  // Levels for fp16 tensor-core operands: level16[s] holds the fp16 bits of
+  // tile_scale * levels[s]; tile_scale in [1, 2) is chosen on the host so that
+  // these fp16 values are as close as possible (relatively) to the scaled
+  // fp32 levels; tile_rel_err is the largest relative error left.
+  uint32_t level16[kMaxLevels];
+  float tile_scale, tile_rel_err;
   int32_t n_levels, container_bytes, payload_bytes, pad;
 };
 
 struct DevTables {
   DevStream k, v;
 };
+static_assert(sizeof(DevStream) % 16 == 0, "DevStream must keep 16-byte alignment of the v table");
 
 // Kernel launchers (defined in the .cu files). All return cudaError_t as int.
 struct AppendArgs {
@@ -82,15 +90,18 @@ struct DecodeArgs {
   float sm_scale;
   void *out;
   int out_dtype;
-  float *ws_o;   // [B*Hq][S][128]
-  float *ws_ml;  // [B*Hq][S][2]
-  int splits;
-  int64_t chunk;  // tokens per split (multiple of 32)
+  int64_t *prefix;     // [B + 1] token-group prefix sums (written by the prefix kernel)
+  float *ws_o;         // [slots][G][128] partial o_rot per (b, h) segment of a warp
+  float *ws_ml;        // [slots][G][2]   partial (max, sum)
+  int grid;            // CTAs of the split kernel (one per SM)
+  int64_t total_warps;  // grid * decode_warps_per_cta(G, ck, cv); slots = B * Hkv + total_warps
   int ck, cv;
   bool two_k, two_v;  // the stream's table has a symbol with f < 16
   dq_stats *stats;
 };
 int launch_decode_attention(const DecodeArgs &a, void *stream);
+// Warps per CTA of the split kernel for these shapes (0 if unsupported).
+int decode_warps_per_cta(int G, int ck, int cv);
 
 struct SymbolsArgs {
   const DevStream *tab;

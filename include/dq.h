@@ -167,8 +167,10 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype,
                  dq_stats *d_stats, void *stream);
 
 /* Bytes of device workspace dq_decode_attention needs for these shapes
- * (split-K partial results). Depends only on its arguments and the tables'
- * device. Returns 0 on invalid shapes. */
+ * (token-group prefix sums and the warps' partial softmax states: about
+ * (B*Hkv + SMs*warps_per_SM) * G * 520 bytes, G = Hq/Hkv). Depends only on
+ * its arguments, the tables' container sizes and the tables' device; T_max
+ * does not change it. Returns 0 on invalid shapes. */
 size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv,
                                  int64_t T_max);
 
@@ -176,9 +178,11 @@ size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv,
  * access and parallel dequantisation within attention kernels). For every
  * (b, hq): out = softmax(sm_scale * q K^T) V over the first d_seq_lens[b]
  * tokens of the cache, with K and V dequantised from their containers
- * inside the kernel. Runs as a split-K kernel (rANS decode of K and V,
- * q.K^T, online softmax, P.V per token chunk) plus a combine kernel
- * (log-sum-exp merge of the chunks and the inverse rotation).
+ * inside the kernel. Runs as a prefix kernel (token groups per sequence), a
+ * split kernel (every warp takes an equal share of all 32-token groups of
+ * all (b, h): rANS decode of K and V, q.K^T, online softmax, P.V) and a
+ * combine kernel (log-sum-exp merge of the partial states and the inverse
+ * rotation).
  *   q           device [B][Hq][128], q_dtype DQ_F32 or DQ_BF16
  *   d_kcache, d_vcache  device caches, 16-byte aligned, T_cap % 16 == 0
  *   d_seq_lens  device int32 [B]; a length above T_max or T_cap is clamped
@@ -207,12 +211,12 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype,
  * compete with a caching allocator that owns the memory). It computes exactly
  * what dq_decode_attention computes, with the same arguments minus the
  * workspace, and allocates nothing.
- *   Scratch: the split-K partial results go to a fixed 8 MiB array in the
+ *   Scratch: the partial results go to a fixed 8 MiB array in the
  *   library's own device memory (held by every GPU that loads the library
- *   until the process exits). Shapes whose partial results need more than
- *   8 MiB (see dq_decode_workspace_bytes; about 16000 rows of
- *   B x Hq x splits) are rejected with DQ_ERR_WORKSPACE before anything is
- *   enqueued.
+ *   until the process exits). Shapes whose workspace is above 8 MiB (see
+ *   dq_decode_workspace_bytes; on a 148-SM B200 with 36-byte containers
+ *   that is B*Hkv above about 1650 for G = 4, above about 250 for G = 8)
+ *   are rejected with DQ_ERR_WORKSPACE before anything is enqueued.
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, no allocation) with that device current; make that
  *   first call before any stream capture.

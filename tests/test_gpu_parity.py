@@ -2,8 +2,9 @@
 
 Containers, symbols, norms and drift counters must be bit-identical; attention
 must be within max-abs 2e-3 x RMS of the oracle's fp64 attention over the same
-containers. Sizes span several 32-token tiles with ragged tails, several
-splits, every supported GQA group size and both input dtypes.
+containers. Sizes span several 32-token tiles with ragged tails, warp ranges
+that start and end inside a (sequence, head), every supported GQA group size
+and both input dtypes.
 """
 import numpy as np
 import pytest
@@ -168,6 +169,9 @@ ATTN_CASES = [
     ("qwen3_8b_b16_t8k", 2, 2, 2, 130, [33, 130]),
     ("qwen3_8b_b16_t8k", 2, 1, 8, 96, [64, 95]),
     ("qwen3_8b_b16_t8k", 1, 2, 4, 3000, [2999]),
+    # more token groups than warps in the grid: warp ranges cross (b, h) edges
+    ("qwen3_8b_b16_t8k", 8, 8, 4, 3001, [3000, 33, 2900, 0, 2600, 2500, 40, 3001]),
+    ("long_b4_t64k", 2, 8, 4, 20000, [20000, 12345]),
 ]
 
 
