@@ -147,7 +147,7 @@ def run_dq(args):
     tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
     ck, cv = tab.k.container_bytes, tab.v.container_bytes
     T = w.T
-    T_cap = (T + 15) // 16 * 16
+    T_cap = (T + 31) // 32 * 32
     G = w.Hq // w.Hkv
     kc = torch.zeros((w.B, w.Hkv, T_cap, ck), dtype=torch.uint8, device=dev)
     vc = torch.zeros((w.B, w.Hkv, T_cap, cv), dtype=torch.uint8, device=dev)

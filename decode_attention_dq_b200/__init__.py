@@ -2,12 +2,14 @@
 
 The compute runs in libdq (include/dq.h): an append/encode kernel that
 rotates, normalises, quantises, rANS-codes and drifts each K/V head vector
-into a fixed-size container, and a split-K decode-attention kernel plus a
-combine kernel that decode the containers inside attention. This package is a
+into a fixed-size container, and a decode-attention kernel (every warp takes
+an equal share of all token groups) plus a combine kernel that decode the
+containers inside attention. This package is a
 thin ctypes binding (argument marshalling only) plus seeded synthetic inputs.
 """
 from ._native import (DQ_BF16, DQ_F32, DQ_STREAM_K, DQ_STREAM_V, DqConfig, DqError,  # noqa: F401
-                      Tables, dq_append_kv, dq_build_tables, dq_config_default,
+                      Tables, containers_of, dq_append_kv, dq_build_tables, dq_config_default,
                       dq_decode_attention, dq_decode_attention_noalloc,
                       dq_decode_symbols, dq_decode_workspace_bytes,
-                      dq_design_stream, dq_error_string, load, new_stats, stats_dict)
+                      dq_design_stream, dq_error_string, load, new_cache, new_stats,
+                      stats_dict)

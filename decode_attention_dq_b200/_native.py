@@ -192,11 +192,26 @@ def stats_dict(stats: torch.Tensor) -> dict:
     return dict(zip(STATS_FIELDS, vals))
 
 
+def new_cache(B: int, Hkv: int, T_cap: int, C: int, device=None) -> torch.Tensor:
+    """Zeroed uint8 cache of shape [B, Hkv, T_cap, C] (T_cap a multiple of 32).
+    The bytes are in the library's interleaved layout; use containers_of()
+    to read flat containers."""
+    assert T_cap % 32 == 0, "T_cap must be a multiple of 32"
+    return torch.zeros((B, Hkv, T_cap, C), dtype=torch.uint8, device=device or "cuda")
+
+
+def containers_of(cache: torch.Tensor) -> torch.Tensor:
+    """Flat containers [B, Hkv, T_cap, C] (a copy) of a cache whose bytes are in
+    the interleaved layout [B][Hkv][T_cap/32][C][32]."""
+    B, H, T_cap, C = cache.shape
+    return cache.reshape(B, H, T_cap // 32, C, 32).transpose(-1, -2).reshape(B, H, T_cap, C).contiguous()
+
+
 def dq_append_kv(tab: Tables, k: torch.Tensor, v: torch.Tensor, start_pos: torch.Tensor,
                  kcache: torch.Tensor, vcache: torch.Tensor, stats: torch.Tensor | None = None,
                  stream=None) -> None:
     """k, v: [B, Hkv, n_new, 128] (f32/bf16, contiguous, CUDA); start_pos int32 [B];
-    caches uint8 [B, Hkv, T_cap, C]."""
+    caches uint8 [B, Hkv, T_cap, C] holding the interleaved layout (see new_cache)."""
     B, Hkv, n_new, d = k.shape
     assert d == 128 and v.shape == k.shape and k.dtype == v.dtype
     assert k.is_contiguous() and v.is_contiguous() and kcache.is_contiguous() and vcache.is_contiguous()

@@ -314,7 +314,7 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, in
     if (!t || !k || !v || !d_start_pos || !d_kcache || !d_vcache) return DQ_ERR_NULL;
     if (dtype != DQ_F32 && dtype != DQ_BF16) return DQ_ERR_DTYPE;
     if (B < 0 || n_new < 0 || T_cap < 0 || Hkv != t->cfg.n_kv_heads) return DQ_ERR_SHAPE;
-    if (!aligned(k, 16) || !aligned(v, 16)) return DQ_ERR_ALIGN;
+    if (!aligned(k, 16) || !aligned(v, 16) || T_cap % 32) return DQ_ERR_ALIGN;
     int rc = check_device(t);
     if (rc != DQ_OK) return rc;
     if (B == 0 || n_new == 0) return DQ_OK;
@@ -360,7 +360,7 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const ui
     const int G = Hq / Hkv;
     if (G != 1 && G != 2 && G != 4 && G != 8) return DQ_ERR_SHAPE;
     if (T_cap < 0 || T_max < 0 || T_max > T_cap) return DQ_ERR_SHAPE;
-    if (T_cap % 16 || !aligned(d_kcache, 16) || !aligned(d_vcache, 16) || !aligned(d_workspace, 16) ||
+    if (T_cap % 32 || !aligned(d_kcache, 16) || !aligned(d_vcache, 16) || !aligned(d_workspace, 16) ||
         !aligned(q, 4) || !aligned(out, 4))
       return DQ_ERR_ALIGN;
     if (!std::isfinite(sm_scale)) return DQ_ERR_SHAPE;

@@ -113,6 +113,8 @@ __device__ __forceinline__ int rans_encode(SymFn sym, const AppendTables &T, uin
   return 3 + np;
 }
 
+// Writes one container; byte k goes to dst[32 k] (the cache interleaves the
+// bytes of the 32 tokens of a block).
 __device__ __forceinline__ void store_container(uint8_t *dst, int C, uint16_t n16, uint32_t x, const uint8_t *stack,
                                                 int len) {
   const int np = len - 3;
@@ -123,7 +125,7 @@ __device__ __forceinline__ void store_container(uint8_t *dst, int C, uint16_t n1
     else if (k < 5) byte = static_cast<uint8_t>((x >> (8 * (k - 2))) & 0xFFu);
     else if (k - 5 < np) byte = stack[np - 1 - (k - 5)];
     else byte = 0;
-    dst[k] = byte;
+    dst[32 * k] = byte;
   }
 }
 
@@ -236,7 +238,9 @@ __global__ void __launch_bounds__(kAW * 32) append_kernel(const AppendArgs a, in
     const int j = static_cast<int>(v % a.n_new);
     const int64_t pos = static_cast<int64_t>(a.start_pos[b]) + j;
     *dropped = pos < 0 || pos >= a.T_cap;
-    return *dropped ? nullptr : cache + ((static_cast<int64_t>(b) * a.Hkv + h) * a.T_cap + pos) * C;
+    if (*dropped) return nullptr;
+    // Byte 0 of the container: block pos / 32 of row (b, h), lane pos % 32.
+    return cache + ((static_cast<int64_t>(b) * a.Hkv + h) * a.T_cap + (pos & ~int64_t(31))) * C + (pos & 31);
   };
 
   // ---- phase 2: lane per vector, first encode ----

@@ -19,8 +19,11 @@
 // Prefix kernel (one CTA): token groups per sequence and their prefix sums.
 // Split kernel, per warp and per (b, h) segment of its range:
 //   D1  q~ = H D q / 128 for the G query heads of h (times sm_scale log2 e)
-//   D2  the warp stages 32 K and 32 V containers at a time into shared
-//       memory with 16-byte cp.async, one group ahead
+//   D2  the warp stages 32 K and 32 V containers at a time (one 32-token
+//       block of the cache, whose containers are byte-interleaved) into
+//       shared memory with 16-byte cp.async, one group ahead; lane l reads
+//       byte j of its container at offset 32 j + l, so the 32 lanes' byte
+//       reads fall into different banks even after their cursors drift apart
 //   D3  one lane per token: rANS-decode K (table look-up, multiply-add, byte
 //       renormalisation) and accumulate q~ . y_hat for the G heads
 //   D5  in the same loop the lane decodes V of the PREVIOUS group (whose
@@ -73,10 +76,14 @@ __host__ __device__ inline SplitSmem split_smem_layout(int G, int ck, int cv, in
   s.wbuf = s.tile + static_cast<size_t>(kTile) * kTileRow;          // [2][8][kWhStride] fp16
   s.qt = s.wbuf + 2 * 8 * kWhStride * 2;                            // [128][G] floats
   s.warp_bytes = align16(s.qt + static_cast<size_t>(kD) * G * 4);
-  // 256 bytes of slack: a corrupt container can make its decoder read up to
-  // 2 bytes per symbol past its start; those reads stay inside the CTA's
-  // shared memory and only produce garbage (flagged by the final-state check).
-  s.total = s.warp0 + static_cast<size_t>(nwarps) * s.warp_bytes + 256;
+  // A corrupt container can make its decoder's cursor run past the
+  // container, by at most 2 bytes per symbol (byte 5 + 2 * 128 at most),
+  // i.e. 32 * 261 bytes from the staged block in the interleaved layout.
+  // Those reads only produce garbage (flagged by the final-state check); the
+  // slack keeps the last warp's reads inside the CTA's shared memory.
+  const size_t reach = s.vst + static_cast<size_t>(kTile) * cv + static_cast<size_t>(kTile) * (kHeaderBytes + 2 * kD + 1);
+  const size_t slack = reach > s.warp_bytes ? align16(reach - s.warp_bytes) + 256 : 256;
+  s.total = s.warp0 + static_cast<size_t>(nwarps) * s.warp_bytes + slack;
   return s;
 }
 
@@ -87,17 +94,17 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
-// Copies the containers of tokens [t0, t0 + n) of one cache row (n is 16 or
-// 32, so n * C is a multiple of 16) into shared memory, 16 bytes per copy.
-__device__ __forceinline__ void stage_group(uint8_t *dst, const uint8_t *row, int64_t t0, int n, int C,
-                                            int lane) {
-  const int chunks = (n * C) >> 4;
+// Copies the 32-token block starting at token t0 (a multiple of 32) of one
+// cache row into shared memory, 16 bytes per copy (32 C is a multiple of 16).
+__device__ __forceinline__ void stage_group(uint8_t *dst, const uint8_t *row, int64_t t0, int C, int lane) {
+  const int chunks = (kTile * C) >> 4;
   const uint8_t *src = row + t0 * C;
   for (int c = lane; c < chunks; c += 32) cp_async16(dst + c * 16, src + c * 16);
 }
 
 // rANS decoder state of one lane: the 32-bit state and the shared-memory
-// offset (from the kernel's shared base) of the next container byte.
+// offset (from the kernel's shared base) of the next container byte; byte j
+// of the lane's container is 32 j past byte 0.
 struct RansLane {
   uint32_t x;
   uint32_t p;
@@ -105,9 +112,9 @@ struct RansLane {
 
 __device__ __forceinline__ RansLane rans_open(const uint8_t *smem, uint32_t off) {
   RansLane r;
-  r.x = static_cast<uint32_t>(smem[off + 2]) | (static_cast<uint32_t>(smem[off + 3]) << 8) |
-        (static_cast<uint32_t>(smem[off + 4]) << 16);
-  r.p = off + kHeaderBytes;
+  r.x = static_cast<uint32_t>(smem[off + 2 * kTile]) | (static_cast<uint32_t>(smem[off + 3 * kTile]) << 8) |
+        (static_cast<uint32_t>(smem[off + 4 * kTile]) << 16);
+  r.p = off + kHeaderBytes * kTile;
   return r;
 }
 
@@ -118,15 +125,15 @@ __device__ __forceinline__ RansLane rans_open(const uint8_t *smem, uint32_t off)
 // shifts in the next byte b and the cursor moves by n. A second byte can only
 // be needed after a symbol with f < 16 (x >= 16 f after the step); kTwo
 // enables that step for tables that have such a symbol. The byte reads never
-// leave the staged shared memory (the cursor moves at most 2 bytes per
-// symbol; 256 bytes of slack follow the last staged container). Returns the
-// byte offset 4 s of the symbol's level.
+// leave the kernel's shared memory (the cursor moves at most 2 bytes per
+// symbol and the layout leaves room for that). Returns the byte offset 4 s
+// of the symbol's level.
 template <bool kTwo>
 __device__ __forceinline__ uint32_t rans_step(RansLane &r, const uint32_t *lut, const uint8_t *smem) {
   const uint32_t e = lut[r.x & (kM - 1)];
   uint32_t x = (e >> 20) * (r.x >> kProbBits) + (e & 0x7FFu);
   const uint32_t b0 = smem[r.p];
-  const uint32_t b1 = kTwo ? static_cast<uint32_t>(smem[r.p + 1]) : 0u;
+  const uint32_t b1 = kTwo ? static_cast<uint32_t>(smem[r.p + kTile]) : 0u;
   const uint32_t n0 = __umulhi(x - kL, 2u);
   x += n0 * (x * 255u + b0);
   uint32_t adv = n0;
@@ -135,13 +142,14 @@ __device__ __forceinline__ uint32_t rans_step(RansLane &r, const uint32_t *lut, 
     x += n1 * (x * 255u + b1);
     adv += n1;
   }
-  r.p += adv;
+  r.p += adv * kTile;
   r.x = x;
   return (e >> 9) & 0x1Cu;
 }
 
+// fp16 norm in bytes 0 and 1 of a staged (interleaved) container.
 __device__ __forceinline__ float norm_of(const uint8_t *cb) {
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(cb[0] | (cb[1] << 8))));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(cb[0] | (cb[kTile] << 8))));
 }
 
 // sc[g] += q~[i][g] * y for the G heads, two heads per packed fp32 FMA.
@@ -399,7 +407,6 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
     const uint8_t *vrow = a.vcache + bh * a.T_cap * cv;
     const int64_t tseg = j0 * kTile;
     auto group_t0 = [&](int64_t j) { return tseg + j * kTile; };
-    auto ncopy = [&](int64_t t0) { return (a.T_cap - t0) < kTile ? static_cast<int>(a.T_cap - t0) : kTile; };
 
     WarpAcc<G> acc;
 #pragma unroll
@@ -417,11 +424,11 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
     // (j+1)%2, both complete; iteration j prefetches K(j+2) and V(j+1).
     {
       const int64_t t0 = group_t0(0);
-      stage_group(kst, krow, t0, ncopy(t0), ck, lane);
-      stage_group(vst, vrow, t0, ncopy(t0), cv, lane);
+      stage_group(kst, krow, t0, ck, lane);
+      stage_group(vst, vrow, t0, cv, lane);
       if (n > 1) {
         const int64_t t1 = group_t0(1);
-        stage_group(kst + kTile * ck, krow, t1, ncopy(t1), ck, lane);
+        stage_group(kst + kTile * ck, krow, t1, ck, lane);
       }
       cp_async_commit();
       cp_async_wait_0();
@@ -430,7 +437,7 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
     // K pass of group 0 on its own.
     float sc[G], p[G];
     {
-      const uint8_t *kb = kst + lane * ck;
+      const uint8_t *kb = kst + lane;
       RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
 #pragma unroll
       for (int gg = 0; gg < G; ++gg) sc[gg] = 0.0f;
@@ -453,7 +460,7 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
       // b[ks][1] the same tokens + 8 (zero for heads >= G).
       uint32_t fb_hi[2][2], fb_lo[2][2];
       {
-        const uint8_t *vb = vst + cur * kTile * cv + lane * cv;
+        const uint8_t *vb = vst + cur * kTile * cv + lane;
         const bool valid = group_t0(j) + lane < len;
         const float nv = norm_of(vb);
 #pragma unroll
@@ -478,16 +485,16 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
       // Prefetch K(j+2) into slot cur and V(j+1) into slot nxt.
       if (j + 2 < n) {
         const int64_t t2 = group_t0(j + 2);
-        stage_group(kst + cur * kTile * ck, krow, t2, ncopy(t2), ck, lane);
+        stage_group(kst + cur * kTile * ck, krow, t2, ck, lane);
       }
       if (has_next) {
         const int64_t t1 = group_t0(j + 1);
-        stage_group(vst + nxt * kTile * cv, vrow, t1, ncopy(t1), cv, lane);
+        stage_group(vst + nxt * kTile * cv, vrow, t1, cv, lane);
       }
       cp_async_commit();
 
-      const uint8_t *kb = kst + nxt * kTile * ck + lane * ck;
-      const uint8_t *vb = vst + cur * kTile * cv + lane * cv;
+      const uint8_t *kb = kst + nxt * kTile * ck + lane;
+      const uint8_t *vb = vst + cur * kTile * cv + lane;
       RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
       RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
 #pragma unroll

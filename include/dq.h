@@ -30,15 +30,20 @@
  *   - No C++ exception crosses this boundary. There is no CPU fallback.
  *
  * Layouts (row-major, contiguous):
- *   K/V new tokens   [B][Hkv][n_new][128]      fp32 or bf16
- *   K cache          [B][Hkv][T_cap][C_k]      uint8 containers
- *   V cache          [B][Hkv][T_cap][C_v]      uint8 containers
- *   q                [B][Hq][128]              fp32 or bf16
- *   out              [B][Hq][128]              fp32 or bf16
+ *   K/V new tokens   [B][Hkv][n_new][128]           fp32 or bf16
+ *   K cache          [B][Hkv][T_cap/32][C_k][32]    uint8, T_cap % 32 == 0
+ *   V cache          [B][Hkv][T_cap/32][C_v][32]    uint8, T_cap % 32 == 0
+ *   q                [B][Hq][128]                   fp32 or bf16
+ *   out              [B][Hq][128]                   fp32 or bf16
  * Query head hq attends with KV head hq / (Hq / Hkv) (grouped-query
  * attention). Container layout: bytes 0-1 the fp16 norm ||x||
  * (little-endian), bytes 2-4 the final rANS state (little-endian), then the
  * renormalisation bytes in decode order, then zero padding to C.
+ * Cache layout: the containers of each block of 32 consecutive tokens are
+ * byte-interleaved, byte j of token t at index [t / 32][j][t % 32]; a cache
+ * is the same number of bytes (T_cap * C per (b, h)) as flat containers. The
+ * decoder's 32 lanes (one per token) then read their next bytes from 32
+ * different shared-memory banks. dq_decode_symbols takes flat containers.
  */
 #ifndef DQ_H
 #define DQ_H
@@ -155,7 +160,9 @@ int dq_get_signs(const dq_tables *t, int8_t *signs);
  *   d_start_pos device int32 [B]: token j of sequence b is written at
  *               position d_start_pos[b] + j; positions outside [0, T_cap)
  *               are skipped and counted in dropped_writes
- *   d_kcache    device [B][Hkv][T_cap][C_k]; d_vcache [B][Hkv][T_cap][C_v]
+ *   d_kcache    device cache of C_k-byte containers, d_vcache of C_v-byte
+ *               ones, both in the interleaved cache layout above;
+ *               T_cap % 32 == 0 (else DQ_ERR_ALIGN)
  *   d_stats     device dq_stats or NULL
  *   stream      cudaStream_t
  * Hkv must equal the tables' n_kv_heads. Containers are bit-identical to the
@@ -184,7 +191,8 @@ size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv,
  * combine kernel (log-sum-exp merge of the partial states and the inverse
  * rotation).
  *   q           device [B][Hq][128], q_dtype DQ_F32 or DQ_BF16
- *   d_kcache, d_vcache  device caches, 16-byte aligned, T_cap % 16 == 0
+ *   d_kcache, d_vcache  device caches (interleaved layout), 16-byte
+ *               aligned, T_cap % 32 == 0
  *   d_seq_lens  device int32 [B]; a length above T_max or T_cap is clamped
  *               and counted in clamped_lengths; length 0 gives out = 0
  *   T_max       host bound on max(d_seq_lens), 0 <= T_max <= T_cap

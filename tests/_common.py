@@ -37,7 +37,12 @@ def inputs(w: synth.Workload, T: int | None = None):
 
 
 def t_cap_for(T):
-    return max(16, (T + 15) // 16 * 16)
+    return max(32, (T + 31) // 32 * 32)
+
+
+def flat(cache):
+    """Flat containers (numpy [B, Hkv, T_cap, C]) of a GPU cache."""
+    return dq.containers_of(cache).cpu().numpy()
 
 
 def gpu_append_all(tab, K, V, dtype, T_cap=None, stats=None):

@@ -105,9 +105,10 @@ def test_append_bit_exact(wname, T, kb, vb):
     stats = dq.new_stats()
     kc, vc = cm.gpu_append_all(lib, K, V, w.torch_dtype, stats=stats)
     torch.cuda.synchronize()
-    np.testing.assert_array_equal(kc[:, :, :T].cpu().numpy(), rk)
-    np.testing.assert_array_equal(vc[:, :, :T].cpu().numpy(), rv)
-    assert not kc[:, :, T:].any() and not vc[:, :, T:].any()
+    kf, vf = cm.flat(kc), cm.flat(vc)
+    np.testing.assert_array_equal(kf[:, :, :T], rk)
+    np.testing.assert_array_equal(vf[:, :, :T], rv)
+    assert not kf[:, :, T:].any() and not vf[:, :, T:].any()
     s = dq.stats_dict(stats)
     assert s["k_syms_drifted"] == kst.syms_drifted and s["v_syms_drifted"] == vst.syms_drifted
     assert s["k_cont_drifted"] == kst.cont_drifted and s["v_cont_drifted"] == vst.cont_drifted
@@ -121,13 +122,13 @@ def test_append_incremental_positions_and_drops():
     ref = cm.oracle_tables(2)
     lib = cm.lib_tables(2)
     rk, rv, _, _, _, _ = o.encode_cache(ref, K, V)
-    T_cap = 80
-    kc = torch.zeros((3, 2, T_cap, 36), dtype=torch.uint8, device="cuda")
-    vc = torch.zeros_like(kc)
+    T_cap = 96
+    kc = dq.new_cache(3, 2, T_cap, 36)
+    vc = dq.new_cache(3, 2, T_cap, 36)
     stats = dq.new_stats()
-    # three appends of 40, 1 and 39 tokens; sequence 2 starts 5 positions late
-    # so its last 5 tokens fall past T_cap and are dropped.
-    shift = np.array([0, 0, 5])
+    # three appends of 40, 1 and 39 tokens; sequence 2 starts 21 positions
+    # late so its last 5 tokens fall past T_cap and are dropped.
+    shift = np.array([0, 0, 21])
     done = 0
     for n in (40, 1, 39):
         kt = torch.from_numpy(K[:, :, done:done + n]).to("cuda", torch.bfloat16).contiguous()
@@ -136,11 +137,13 @@ def test_append_incremental_positions_and_drops():
         dq.dq_append_kv(lib, kt, vt, start, kc, vc, stats=stats)
         done += n
     torch.cuda.synchronize()
-    kn, vn = kc.cpu().numpy(), vc.cpu().numpy()
-    np.testing.assert_array_equal(kn[:2], rk[:2])
-    np.testing.assert_array_equal(vn[:2], rv[:2])
-    np.testing.assert_array_equal(kn[2, :, 5:], rk[2, :, :75])
-    np.testing.assert_array_equal(vn[2, :, 5:], rv[2, :, :75])
+    kn, vn = cm.flat(kc), cm.flat(vc)
+    np.testing.assert_array_equal(kn[:2, :, :80], rk[:2])
+    np.testing.assert_array_equal(vn[:2, :, :80], rv[:2])
+    assert not kn[:2, :, 80:].any() and not vn[:2, :, 80:].any()
+    np.testing.assert_array_equal(kn[2, :, 21:], rk[2, :, :75])
+    np.testing.assert_array_equal(vn[2, :, 21:], rv[2, :, :75])
+    assert not kn[2, :, :21].any() and not vn[2, :, :21].any()
     assert dq.stats_dict(stats)["dropped_writes"] == 2 * 2 * 5  # K and V, 2 heads, 5 tokens
 
 
@@ -157,8 +160,8 @@ def test_append_nonfinite_and_zero_vectors():
     stats = dq.new_stats()
     kc, vc = cm.gpu_append_all(lib, K, V, torch.float32, stats=stats)
     torch.cuda.synchronize()
-    np.testing.assert_array_equal(kc[:, :, :64].cpu().numpy(), rk)
-    np.testing.assert_array_equal(vc[:, :, :64].cpu().numpy(), rv)
+    np.testing.assert_array_equal(cm.flat(kc)[:, :, :64], rk)
+    np.testing.assert_array_equal(cm.flat(vc)[:, :, :64], rv)
     assert dq.stats_dict(stats)["nonfinite_inputs"] == kst.nonfinite_inputs + vst.nonfinite_inputs == 3
 
 
@@ -244,5 +247,7 @@ def test_argument_errors():
         dq.dq_decode_attention(lib, q.half(), kc, kc, seq, 1, out, ws)
     k = torch.zeros((1, 3, 1, 128), device="cuda")
     assert code(lambda: dq.dq_append_kv(lib, k, k, seq, kc, kc)) == -4  # Hkv mismatch
+    k2 = torch.zeros((1, 2, 1, 128), device="cuda")
+    assert code(lambda: dq.dq_append_kv(lib, k2, k2, seq, bad_cap, bad_cap)) == -6  # T_cap % 32
     with pytest.raises(dq.DqError):
         dq.dq_build_tables(n_kv_heads=2, head_dim=64)

@@ -51,7 +51,7 @@ def test_noalloc_matches_workspace_entry_on_two_calls():
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     tab = cm.lib_tables(8)
-    B, Hq, Hkv, T_cap = 256, 64, 8, 16  # 16384 partial rows > the 8 MiB scratch
+    B, Hq, Hkv, T_cap = 256, 64, 8, 32  # 2048 (b, h) slots of 8 heads > the 8 MiB scratch
     assert dq.dq_decode_workspace_bytes(tab, B, Hq, Hkv, T_cap) > (8 << 20)
     kc = torch.zeros((B, Hkv, T_cap, 36), dtype=torch.uint8, device="cuda")
     q = torch.zeros((B, Hq, 128), dtype=torch.float32, device="cuda")
