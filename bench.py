@@ -39,6 +39,34 @@ WORKLOAD = "serve_b128_t8k"
 # + 8 G softmax ops, counted in lane-ops (issue slots x 32).
 RANS_OPS_PER_SYMBOL = 5.5
 SOFTMAX_OPS_PER_HEAD = 8
+# Encode (append) work per vector, same convention: 896 WHT + 256 norm/scale
+# + 384 quantise + 128 x 8 rANS encode lane-ops.
+ENCODE_OPS_PER_VECTOR = 2560
+# Kernel launches of one step: dq_append_kv (1) + dq_decode_attention
+# (prefix, split, combine).
+LAUNCHES_PER_STEP = 4
+# DRAM traffic of decode_split_kernel from one ncu capture (dram__bytes_read
+# + dram__bytes_write) of the 32-sequence, 8192-token workload with 36-byte
+# containers: 151.37 MB + 3.74 MB per launch over 32*8*8192 token-heads. It
+# scales with the token-heads a launch processes (reads are the containers,
+# writes the partial states). It belongs to one version of the kernel source:
+# for any other, or other container sizes, traffic is reported as null.
+DECODE_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_decode.cu",
+                  "sha256_16": "2badf4fff5fba524", "ck": 36, "cv": 36,
+                  "bytes_per_token_head": (151.367168e6 + 3.742464e6) / (32 * 8 * 8192)}
+
+
+def decode_traffic(token_heads, ck, cv):
+    import hashlib
+    t = DECODE_TRAFFIC
+    try:
+        with open(os.path.join(ROOT, t["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if sha != t["sha256_16"] or (ck, cv) != (t["ck"], t["cv"]):
+        return None
+    return token_heads * t["bytes_per_token_head"]
 
 
 def ops_per_token_head(G: int) -> float:
@@ -153,10 +181,14 @@ def run_dq(args):
     vc = torch.zeros((w.B, w.Hkv, T_cap, cv), dtype=torch.uint8, device=dev)
     prefill_stats = dq.new_stats(dev)
     t0 = time.time()
-    synth.prefill_cache(tab, w, kc, vc, T - 1, stats=prefill_stats, threads=args.threads)
+    enc_timings = []
+    synth.prefill_cache(tab, w, kc, vc, T - 1, stats=prefill_stats, threads=args.threads,
+                        timings=enc_timings)
     torch.cuda.synchronize()
     prefill_s = time.time() - t0
     pstats = dq.stats_dict(prefill_stats)
+    enc_ms = sum(a.elapsed_time(b) for a, b, _ in enc_timings)
+    enc_vectors = sum(n for _, _, n in enc_timings)  # per stream (K and V each)
 
     # Per-step inputs: a distinct new token and q for each step (host, pinned).
     nsteps_inputs = 4
@@ -278,13 +310,16 @@ def run_dq(args):
                        "parallelism": "replicas x%d" % ws},
             "hbm_gbs": hbm_gbs,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tlaneop/s",
-                         "frac": achieved / alu_peak, "traffic": None,
+                         "frac": achieved / alu_peak, "traffic": decode_traffic(token_heads, ck, cv),
+                         "traffic_note": "decode_split_kernel DRAM bytes per launch, scaled from an ncu "
+                                         "capture of the 32-sequence case by token-heads",
+                         "algorithmic_bytes": comp_bytes,
                          "kernel": "decode_split_kernel + combine_kernel (dq_decode_attention)",
                          "kernel_ms": dec_ms, "peak_source": "%s clock, %d SMs x 128 lanes" % (src, sm_count),
                          "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": peaks.get("hbm_gbs"),
                                  "frac": hbm_gbs / float(peaks.get("hbm_gbs", 6650.0))}},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk,
             "drift": {"prefill_k_syms_pct": 100.0 * pstats["k_syms_drifted"] / (token_heads * 128),
                       "prefill_v_syms_pct": 100.0 * pstats["v_syms_drifted"] / (token_heads * 128),
@@ -293,6 +328,7 @@ def run_dq(args):
                       "fallbacks": pstats["overflow_fallbacks"]},
             "integrity_errors": st["integrity_errors"],
             "prefill_s": prefill_s,
+            "encode": encode_report(enc_ms, enc_vectors, w, ck, cv, alu_peak, peaks),
         }
         if ws == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(w, tab_seed=0, seconds=args.cpu_seconds)
@@ -300,6 +336,25 @@ def run_dq(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def encode_report(enc_ms, enc_vectors, w, ck, cv, alu_peak, peaks):
+    """Throughput of dq_append_kv over the prefill (device time of the append
+    calls only; host generation of the inputs is outside the events)."""
+    if enc_ms <= 0:
+        return None
+    containers = 2 * enc_vectors
+    s = enc_ms * 1e-3
+    in_bytes = containers * 128 * (2 if w.dtype == "bf16" else 4)
+    out_bytes = enc_vectors * (ck + cv)
+    achieved = containers * ENCODE_OPS_PER_VECTOR / s / 1e12
+    return {"what": "prefill append of %d tokens x %d sequences x %d KV heads (K and V)"
+                    % (w.T - 1, w.B, w.Hkv),
+            "ms": enc_ms, "containers_per_s": containers / s,
+            "hbm_gbs": (in_bytes + out_bytes) / s / 1e9,
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tlaneop/s",
+                         "frac": achieved / alu_peak,
+                         "hbm_frac": (in_bytes + out_bytes) / s / 1e9 / float(peaks.get("hbm_gbs", 6650.0))}}
 
 
 def oracle_sample_step(w, tabs, rows, cache_rows):
@@ -327,7 +382,7 @@ def oracle_sample_step(w, tabs, rows, cache_rows):
         o.attention_fp64(tabs, qb, kfull, vfull, [kc.shape[0]], rows=[(0, h)])
 
 
-def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=64):
+def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512):
     """The oracle, as it stands, on the host: bounded sample of the step."""
     import numpy as np
     from decode_attention_dq_b200 import synth

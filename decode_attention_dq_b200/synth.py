@@ -140,10 +140,13 @@ def scaled(w: Workload, **changes) -> Workload:
 
 
 def prefill_cache(tab, w: Workload, kcache, vcache, n_tokens: int, seqs_per_call: int = 8,
-                  threads: int = 16, stats=None):
+                  threads: int = 16, stats=None, timings: list | None = None):
     """Fill positions [0, n_tokens) of every sequence's cache with the
     workload's seeded K/V, appended through dq_append_kv in batches of
-    sequences (the inputs are drawn on the host, then copied to the device)."""
+    sequences (the inputs are drawn on the host, then copied to the device).
+    With `timings`, each dq_append_kv call is bracketed by CUDA events on the
+    current stream and (start event, end event, vectors per stream) is
+    appended to the list."""
     from ._native import dq_append_kv  # local import: synth itself needs no GPU
 
     for b0 in range(0, w.B, seqs_per_call):
@@ -156,4 +159,10 @@ def prefill_cache(tab, w: Workload, kcache, vcache, n_tokens: int, seqs_per_call
         vt = torch.from_numpy(V).to(device=kcache.device, dtype=w.torch_dtype).view(
             b1 - b0, w.Hkv, n_tokens, 128)
         start = torch.zeros(b1 - b0, dtype=torch.int32, device=kcache.device)
+        if timings is not None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
         dq_append_kv(tab, kt, vt, start, kcache[b0:b1], vcache[b0:b1], stats=stats)
+        if timings is not None:
+            e1.record()
+            timings.append((e0, e1, (b1 - b0) * w.Hkv * n_tokens))
