@@ -113,6 +113,13 @@ void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
   s->payload_bytes = d.payload_bytes;
 }
 
+// A symbol with f < 16 can make one coding step move two bytes.
+bool has_small_freq(const dqi::StreamDesign &d) {
+  for (int s = 0; s < d.n_levels; ++s)
+    if (d.freq[s] < 16) return true;
+  return false;
+}
+
 const dqi::StreamDesign *stream_of(const dq_tables *t, int kind) {
   if (!t) return nullptr;
   if (kind == DQ_STREAM_K) return &t->k;
@@ -335,6 +342,8 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, in
     a.cv = t->v.container_bytes;
     a.nk = t->k.n_levels;
     a.nv = t->v.n_levels;
+    a.two_k = has_small_freq(t->k);
+    a.two_v = has_small_freq(t->v);
     a.stats = d_stats;
     int e = dqi::launch_append(a, stream);
     return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
@@ -395,11 +404,6 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const ui
     a.total_warps = wl.total_warps;
     a.ck = t->k.container_bytes;
     a.cv = t->v.container_bytes;
-    auto has_small_freq = [](const dqi::StreamDesign &d) {
-      for (int s = 0; s < d.n_levels; ++s)
-        if (d.freq[s] < 16) return true;
-      return false;
-    };
     a.two_k = has_small_freq(t->k);
     a.two_v = has_small_freq(t->v);
     a.stats = d_stats;

@@ -14,108 +14,59 @@
 // __fmul_rn, __fdiv_rn, __fsqrt_rn) so no multiply-add is contracted: the
 // containers are bit-identical to the format's definition.
 //
-// Work split: one warp takes `vpw` (1..32) vectors of one stream.
-//   phase 1 (warp per vector): E1 sign flip, E2 Walsh-Hadamard transform
-//     (shuffles for stages 1..16, registers for 32 and 64), E3 norm in a fixed
-//     tree, scale, fp16 norm, E4 quantisation; u and symbols to shared memory.
-//   phase 2 (lane per vector): E5 rANS encode last-to-first; containers that
+// Work split: one warp takes 32 consecutive vectors of one stream, one per lane.
+//   phase 1 (lane per vector, all in registers): E1 sign flip, E2 Walsh-
+//     Hadamard transform (the seven butterfly stages in order), E3 norm in
+//     the fixed tree (the 32 partial sums of four squares, then pairwise
+//     over offsets 16, 8, 4, 2, 1), scale, fp16 norm, E4 quantisation by a
+//     three-step search over the sorted thresholds; symbols packed 4 per
+//     register.
+//   phase 2 (lane per vector): E5 rANS encode last-to-first without branches
+//     (a renormalisation push is written every step and kept only when
+//     needed; the division by f is an exact multiply-shift); containers that
 //     fit are stored at once.
-//   phase 3 (warp per over-long container): E6 drift. The greedy rule (least
-//     key first, ties to the lower index) applies moves in a fixed order, so
-//     the warp ranks the candidate moves by repeated arg-min and lane m
-//     encodes the string with the first m+1 moves applied; the smallest m that
-//     fits is the greedy result. 32 move counts are tried per pass.
+//   phase 3 (warp per over-long container, a few percent): E6 drift. The warp
+//     recomputes the vector's rotated coordinates (4 per lane, the same
+//     arithmetic), ranks the candidate moves by repeated arg-min (least key
+//     first, ties to the lower index), and lane m encodes the string with the
+//     first m+1 moves applied; the smallest m that fits is the greedy result.
+//     32 move counts are tried per pass.
 #include "dq_device.cuh"
 
 namespace dqi {
 namespace {
 
-constexpr int kAW = 4;  // warps per CTA
-constexpr int kUStride = kD + 1;
-constexpr int kQStride = kD + 4;
-constexpr int kStack = kMaxContainer;
+constexpr int kAW = 4;                  // warps per CTA
+constexpr int kStackSlots = 64;         // bytes of push stack per lane
 constexpr float kSqrtD = 11.3137084989847604f;  // fl32(sqrt(128))
 constexpr uint8_t kNoRank = 255;
 
+// Division by f for the encoder: q = floor(x / f) = (x * m) >> k for every
+// x < 4096 f, with k = 12 + ceil(log2 f^2) and m = ceil(2^k / f). (x m / 2^k
+// = x / f + x e / (f 2^k) with e = m f - 2^k < f, and x e < 4096 f^2 <= 2^k,
+// so the excess stays below 1 / f and the floor is exact.)
+struct EncSym {
+  uint32_t m, k, xmax, cum;  // xmax = 4096 f: push while x >= xmax
+  uint32_t g, f, pad0, pad1; // g = 4096 - f: x' = x + q g + cum
+};
+
 struct AppendTables {
-  float lev[kMaxLevels], thr[kMaxLevels], cost[kMaxLevels];
+  EncSym es[kMaxLevels];
+  float thr[kMaxLevels];  // thresholds, padded with +inf
+  float lev[kMaxLevels], cost[kMaxLevels];
   uint32_t freq[kMaxLevels], cum[kMaxLevels];
-  unsigned long long rcp[kMaxLevels];  // ceil(2^40 / f)
 };
 
-// Per-warp shared-memory area; vpw vectors per warp.
+// Per-warp shared memory: push stacks (byte j of lane l at [j][l]) and the
+// symbols, move ranks and targets of the container being drifted.
 struct WarpArea {
-  float *u;           // [vpw][kUStride]
-  uint8_t *q;         // [vpw][kQStride]
-  uint8_t *stack;     // [32][kStack]
-  uint8_t *rank;      // [128] move rank of each symbol, kNoRank if none yet
-  uint8_t *tgt;       // [128] level a drifted symbol moves to
-  uint16_t *norm16;   // [vpw]
-  uint8_t *nonfinite; // [vpw]
+  uint8_t stack[kStackSlots * 32];
+  uint8_t q[kD], rank[kD], tgt[kD];
 };
-
-__host__ __device__ inline size_t warp_area_bytes(int vpw) {
-  size_t b = static_cast<size_t>(vpw) * kUStride * 4;
-  b += static_cast<size_t>(vpw) * kQStride;
-  b += 32 * kStack + 128 + 128;
-  b += static_cast<size_t>(vpw) * 2 + vpw;
-  return (b + 15) & ~size_t(15);
-}
-
-__device__ inline WarpArea warp_area(uint8_t *base, int vpw) {
-  WarpArea w;
-  uint8_t *p = base;
-  w.u = reinterpret_cast<float *>(p);
-  p += static_cast<size_t>(vpw) * kUStride * 4;
-  w.q = p;
-  p += static_cast<size_t>(vpw) * kQStride;
-  w.stack = p;
-  p += 32 * kStack;
-  w.rank = p;
-  p += 128;
-  w.tgt = p;
-  p += 128;
-  w.norm16 = reinterpret_cast<uint16_t *>(p);
-  p += static_cast<size_t>(vpw) * 2;
-  w.nonfinite = p;
-  return w;
-}
-
-// Exact x / f and x mod f for x < 2^24 and 1 <= f <= 4096 with M = ceil(2^40 / f):
-// x M / 2^40 = x / f + d with 0 <= d < x / 2^40 < 2^-16 < 1 / f, so the floor
-// is x / f.
-__device__ __forceinline__ uint32_t div_rcp(uint32_t x, unsigned long long M) {
-  return static_cast<uint32_t>((static_cast<unsigned long long>(x) * M) >> 40);
-}
-
-// E5: rANS-encode 128 symbols, coded 127 -> 0, starting from x = 2^16.
-// sym(i) gives symbol i. Pushed bytes go to `stack` in push order. Returns the
-// total length 3 + #pushed, or cap + 1 as soon as it exceeds `cap`.
-template <typename SymFn>
-__device__ __forceinline__ int rans_encode(SymFn sym, const AppendTables &T, uint8_t *stack, int cap,
-                                           uint32_t *x_out) {
-  uint32_t x = kL;
-  int np = 0;
-  const int max_push = cap - 3;
-  for (int i = kD - 1; i >= 0; --i) {
-    const uint32_t s = sym(i);
-    const uint32_t f = T.freq[s];
-    const uint32_t xmax = ((kL >> kProbBits) << 8) * f;
-    while (x >= xmax) {
-      if (np >= max_push) return cap + 1;
-      stack[np++] = static_cast<uint8_t>(x & 0xFFu);
-      x >>= 8;
-    }
-    const uint32_t qf = div_rcp(x, T.rcp[s]);
-    x = qf * kM + (x - qf * f) + T.cum[s];
-  }
-  *x_out = x;
-  return 3 + np;
-}
 
 // Writes one container; byte k goes to dst[32 k] (the cache interleaves the
-// bytes of the 32 tokens of a block).
-__device__ __forceinline__ void store_container(uint8_t *dst, int C, uint16_t n16, uint32_t x, const uint8_t *stack,
+// bytes of the 32 tokens of a block). stk[32 j] holds push j.
+__device__ __forceinline__ void store_container(uint8_t *dst, int C, uint16_t n16, uint32_t x, const uint8_t *stk,
                                                 int len) {
   const int np = len - 3;
   for (int k = 0; k < C; ++k) {
@@ -123,7 +74,7 @@ __device__ __forceinline__ void store_container(uint8_t *dst, int C, uint16_t n1
     if (k == 0) byte = static_cast<uint8_t>(n16 & 0xFFu);
     else if (k == 1) byte = static_cast<uint8_t>(n16 >> 8);
     else if (k < 5) byte = static_cast<uint8_t>((x >> (8 * (k - 2))) & 0xFFu);
-    else if (k - 5 < np) byte = stack[np - 1 - (k - 5)];
+    else if (k - 5 < np) byte = stk[32 * (np - 1 - (k - 5))];
     else byte = 0;
     dst[32 * k] = byte;
   }
@@ -152,222 +103,481 @@ __device__ __forceinline__ float best_move(const AppendTables &T, int nl, int s,
   return best;
 }
 
-__global__ void __launch_bounds__(kAW * 32) append_kernel(const AppendArgs a, int vpw) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  AppendTables &T = *reinterpret_cast<AppendTables *>(smem_raw);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  WarpArea W = warp_area(smem_raw + ((sizeof(AppendTables) + 15) & ~size_t(15)) + warp * warp_area_bytes(vpw), vpw);
-  const bool is_v = blockIdx.y == 1;
-  const DevStream &tab = is_v ? a.tabs->v : a.tabs->k;
-  const int nl = is_v ? a.nv : a.nk;
-  const int C = is_v ? a.cv : a.ck;
-  const int P = C - 2;
-  const void *src = is_v ? a.v : a.k;
-  uint8_t *cache = is_v ? a.vcache : a.kcache;
-  if (threadIdx.x < kMaxLevels) {
-    const int s = threadIdx.x;
-    T.lev[s] = tab.levels[s];
-    T.thr[s] = tab.thresholds[s];
-    T.cost[s] = tab.cost[s];
-    T.freq[s] = tab.freq[s];
-    T.cum[s] = tab.cum[s];
-    const unsigned long long f = tab.freq[s] ? tab.freq[s] : 1u;
-    T.rcp[s] = ((1ull << 40) + f - 1) / f;
-  }
-  __syncthreads();
+// E4: symbol = number of thresholds <= u (ties go up), by a three-step
+// search over the 7 sorted thresholds t0..t6 (padded with +inf).
+__device__ __forceinline__ uint32_t quantize7(float u, const float (&t)[7]) {
+  const bool p1 = t[3] <= u;
+  const float ta = p1 ? t[5] : t[1];
+  const bool p2 = ta <= u;
+  const float tb = p1 ? (p2 ? t[6] : t[4]) : (p2 ? t[2] : t[0]);
+  const bool p3 = tb <= u;
+  return (p1 ? 4u : 0u) + (p2 ? 2u : 0u) + (p3 ? 1u : 0u);
+}
 
-  const int64_t per_seq = static_cast<int64_t>(a.Hkv) * a.n_new;
-  const int64_t nvec = static_cast<int64_t>(a.B) * per_seq;
-  const int64_t v0 = (static_cast<int64_t>(blockIdx.x) * kAW + warp) * vpw;
-  if (v0 >= nvec) return;
-  const int nmine = static_cast<int>((nvec - v0) < vpw ? (nvec - v0) : vpw);
+// Sign word bit `b` moved to the float sign position.
+__device__ __forceinline__ uint32_t sign_bit(uint32_t word, int b) { return (word << (31 - b)) & 0x80000000u; }
 
-  // ---- phase 1: warp per vector ----
-  for (int vv = 0; vv < nmine; ++vv) {
-    const int64_t v = v0 + vv;
-    const int h = static_cast<int>((v % per_seq) / a.n_new);
-    float z[4];
-    bool nf = false;
+// Phase 1 for the vector of this lane: loads, signs, WHT, norm, scale and
+// quantisation, all in registers. Writes the packed symbols (byte i % 4 of
+// pk[i / 4] = symbol i), the fp16 norm and whether the vector was
+// non-finite (then it is encoded as the zero vector).
+template <bool kBF16>
+__device__ __forceinline__ void lane_prepare(const void *src, int64_t v, const uint32_t (&sw)[4],
+                                             const float (&t)[7], uint32_t (&pk)[32], uint16_t *n16_out,
+                                             bool *nf_out) {
+  float z[kD];
+  if constexpr (kBF16) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(src) + v * kD);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float xv = load_elem(src, v * kD + lane + 32 * k, a.dtype);
-      nf |= !isfinite(xv);
-      z[k] = apply_sign(xv, __ldg(a.sign_bits + h * 4 + k), lane);
-    }
-    nf = __any_sync(kFull, nf);
-    float u[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    uint16_t n16 = 0;
-    if (!nf) {
-      wht128_warp(z, lane);
-      float part = __fadd_rn(__fadd_rn(__fmul_rn(z[0], z[0]), __fmul_rn(z[1], z[1])),
-                             __fadd_rn(__fmul_rn(z[2], z[2]), __fmul_rn(z[3], z[3])));
+    for (int c = 0; c < 16; ++c) {
+      const uint4 w = __ldg(p + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) part = __fadd_rn(part, __shfl_xor_sync(kFull, part, off));
-      if (!isfinite(part)) {
-        nf = true;
-      } else {
-        const float r = __fsqrt_rn(part);
-        const float sigma = (r == 0.0f) ? 0.0f : __fdiv_rn(kSqrtD, r);
-        if (r != 0.0f && isfinite(sigma)) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) u[k] = __fmul_rn(z[k], sigma);
-        }
-        float nv = __fdiv_rn(r, kSqrtD);
-        if (nv > 65504.0f) nv = 65504.0f;
-        n16 = __half_as_ushort(__float2half_rn(nv));
+      for (int e = 0; e < 4; ++e) {
+        const int i = 8 * c + 2 * e;
+        z[i] = __uint_as_float((ww[e] << 16) ^ sign_bit(sw[i >> 5], i & 31));
+        z[i + 1] = __uint_as_float((ww[e] & 0xFFFF0000u) ^ sign_bit(sw[(i + 1) >> 5], (i + 1) & 31));
       }
     }
+  } else {
+    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const float *>(src) + v * kD);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      int c = 0;
-      for (int j = 0; j < nl - 1; ++j) c += (T.thr[j] <= u[k]) ? 1 : 0;
-      W.u[vv * kUStride + lane + 32 * k] = u[k];
-      W.q[vv * kQStride + lane + 32 * k] = static_cast<uint8_t>(c);
-    }
-    if (lane == 0) {
-      W.norm16[vv] = n16;
-      W.nonfinite[vv] = nf ? 1 : 0;
+    for (int c = 0; c < 32; ++c) {
+      const uint4 w = __ldg(p + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * c + e;
+        z[i] = __uint_as_float(ww[e] ^ sign_bit(sw[i >> 5], i & 31));
+      }
     }
   }
-  __syncwarp();
+  // E2: stages h = 1, 2, ..., 64; (a, b) -> (a + b, a - b) on the pairs
+  // (j, j + h) with bit h of j clear.
+#pragma unroll
+  for (int st = 0; st < 7; ++st) {
+    const int h = 1 << st;
+#pragma unroll
+    for (int pr = 0; pr < kD / 2; ++pr) {
+      const int j = ((pr >> st) << (st + 1)) | (pr & (h - 1));
+      const float a0 = z[j], b0 = z[j + h];
+      z[j] = __fadd_rn(a0, b0);
+      z[j + h] = __fsub_rn(a0, b0);
+    }
+  }
+  // E3: p_l = (z_l^2 + z_{l+32}^2) + (z_{l+64}^2 + z_{l+96}^2), then the
+  // pairwise tree over offsets 16, 8, 4, 2, 1.
+  float p[32];
+#pragma unroll
+  for (int l = 0; l < 32; ++l)
+    p[l] = __fadd_rn(__fadd_rn(__fmul_rn(z[l], z[l]), __fmul_rn(z[l + 32], z[l + 32])),
+                     __fadd_rn(__fmul_rn(z[l + 64], z[l + 64]), __fmul_rn(z[l + 96], z[l + 96])));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+    for (int l = 0; l < o; ++l) p[l] = __fadd_rn(p[l], p[l + o]);
+  const float ss = p[0];
+  bool nf = !isfinite(ss);
+  uint16_t n16 = 0;
+  float sigma = 0.0f;
+  if (!nf) {
+    const float r = __fsqrt_rn(ss);
+    sigma = (r == 0.0f) ? 0.0f : __fdiv_rn(kSqrtD, r);
+    if (!(r != 0.0f && isfinite(sigma))) sigma = 0.0f;
+    float nv = __fdiv_rn(r, kSqrtD);
+    if (nv > 65504.0f) nv = 65504.0f;
+    n16 = __half_as_ushort(__float2half_rn(nv));
+  }
+  // E4 (u = 0 for the zero and the non-finite vector).
+#pragma unroll
+  for (int w = 0; w < 32; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float u = nf ? 0.0f : __fmul_rn(z[4 * w + e], sigma);
+      word |= quantize7(u, t) << (8 * e);
+    }
+    pk[w] = word;
+  }
+  *n16_out = n16;
+  *nf_out = nf;
+}
 
-  auto dst_of = [&](int vv, bool *dropped) -> uint8_t * {
-    const int64_t v = v0 + vv;
+// E5 without branches: rANS-encode 128 symbols (sym(i) gives symbol i),
+// coded 127 -> 0 from x = 2^16. A renormalisation push writes the low byte of
+// x to the lane's stack every step and keeps it only when x >= 4096 f; pushes
+// go to stk[32 j]. Returns the total length 3 + #pushed; above `cap` the
+// container is too long (pushes past the stack wrap around and are never
+// stored). No lane branches, so all 32 lanes of a warp stay converged. kTwo:
+// the table has a symbol with f < 16, so a step can push two bytes.
+// One encode step of encode_bf.
+template <bool kTwo>
+__device__ __forceinline__ void encode_step(uint32_t s, const uint8_t *esb, uint8_t *stk, uint32_t &x, uint32_t &np) {
+  const uint4 e0 = *reinterpret_cast<const uint4 *>(esb + s * sizeof(EncSym));  // {m, k, xmax, cum}
+  const uint32_t g = *reinterpret_cast<const uint32_t *>(esb + s * sizeof(EncSym) + 16);
+  bool push = x >= e0.z;
+  stk[32 * (np & (kStackSlots - 1))] = static_cast<uint8_t>(x);
+  np += push ? 1u : 0u;
+  x = push ? (x >> 8) : x;
+  if constexpr (kTwo) {
+    push = x >= e0.z;
+    stk[32 * (np & (kStackSlots - 1))] = static_cast<uint8_t>(x);
+    np += push ? 1u : 0u;
+    x = push ? (x >> 8) : x;
+  }
+  const uint32_t q = static_cast<uint32_t>((static_cast<unsigned long long>(x) * e0.x) >> e0.y);
+  x = (x + e0.w) + q * g;
+}
+
+// kRegs: symbols come from registers (the loop is unrolled completely so
+// that sym(i) indexes them statically); otherwise from shared memory.
+template <bool kTwo, bool kRegs, typename SymFn>
+__device__ __forceinline__ int encode_bf(SymFn sym, const EncSym *es, uint8_t *stk, uint32_t *x_out) {
+  uint32_t x = kL;
+  uint32_t np = 0;
+  const uint8_t *esb = reinterpret_cast<const uint8_t *>(es);
+  if constexpr (kRegs) {
+#pragma unroll
+    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo>(sym(i), esb, stk, x, np);
+  } else {
+#pragma unroll 4
+    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo>(sym(i), esb, stk, x, np);
+  }
+  *x_out = x;
+  return 3 + static_cast<int>(np);
+}
+
+// Phase-1 arithmetic for one vector spread over the warp (coordinate
+// lane + 32 k in u[k]): same operations, same order, so the same u, symbols
+// and norm as lane_prepare. Writes the symbols to q[]; returns the fp16 norm
+// and whether the vector was non-finite.
+__device__ __forceinline__ void warp_prepare(const AppendArgs &a, const void *src, int64_t v, int h,
+                                             const float (&t)[7], int lane, float (&u)[4], uint8_t *q,
+                                             uint16_t *n16_out, bool *nf_out) {
+  float z[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    z[k] = apply_sign(load_elem(src, v * kD + lane + 32 * k, a.dtype), __ldg(a.sign_bits + h * 4 + k), lane);
+  wht128_warp(z, lane);
+  float part = __fadd_rn(__fadd_rn(__fmul_rn(z[0], z[0]), __fmul_rn(z[1], z[1])),
+                         __fadd_rn(__fmul_rn(z[2], z[2]), __fmul_rn(z[3], z[3])));
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) part = __fadd_rn(part, __shfl_xor_sync(kFull, part, off));
+  const bool nf = !isfinite(part);
+  float sigma = 0.0f;
+  uint16_t n16 = 0;
+  if (!nf) {
+    const float r = __fsqrt_rn(part);
+    sigma = (r == 0.0f) ? 0.0f : __fdiv_rn(kSqrtD, r);
+    if (!(r != 0.0f && isfinite(sigma))) sigma = 0.0f;
+    float nv = __fdiv_rn(r, kSqrtD);
+    if (nv > 65504.0f) nv = 65504.0f;
+    n16 = __half_as_ushort(__float2half_rn(nv));
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    u[k] = nf ? 0.0f : __fmul_rn(z[k], sigma);
+    q[lane + 32 * k] = static_cast<uint8_t>(quantize7(u[k], t));
+  }
+  *n16_out = n16;
+  *nf_out = nf;
+}
+
+// Where the vectors of one append call come from and go to (one stream).
+struct StreamCtx {
+  const void *src;
+  uint8_t *cache;
+  int nl, C, P;
+  int64_t per_seq, nvec;
+  float t[7];
+
+  __device__ int head_of(const AppendArgs &a, int64_t v) const {
+    return static_cast<int>((v % per_seq) / a.n_new);
+  }
+  // Byte 0 of vector v's container (block pos / 32 of row (b, h), lane
+  // pos % 32), or null when the position is outside the cache.
+  __device__ uint8_t *dst_of(const AppendArgs &a, int64_t v, bool *dropped) const {
     const int b = static_cast<int>(v / per_seq);
-    const int h = static_cast<int>((v % per_seq) / a.n_new);
+    const int h = head_of(a, v);
     const int j = static_cast<int>(v % a.n_new);
     const int64_t pos = static_cast<int64_t>(a.start_pos[b]) + j;
     *dropped = pos < 0 || pos >= a.T_cap;
     if (*dropped) return nullptr;
-    // Byte 0 of the container: block pos / 32 of row (b, h), lane pos % 32.
     return cache + ((static_cast<int64_t>(b) * a.Hkv + h) * a.T_cap + (pos & ~int64_t(31))) * C + (pos & 31);
-  };
+  }
+};
 
-  // ---- phase 2: lane per vector, first encode ----
-  bool dropped = false, too_long = false;
-  if (lane < nmine) {
-    const uint8_t *q = W.q + lane * kQStride;
-    uint8_t *stack = W.stack + lane * kStack;
+// Copies one stream's tables into shared memory (threads 0..7) and fills the
+// stream context. Callers synchronise before using T.
+__device__ __forceinline__ StreamCtx stream_setup(const AppendArgs &a, AppendTables &T, bool is_v) {
+  const DevStream &tab = is_v ? a.tabs->v : a.tabs->k;
+  StreamCtx c;
+  c.nl = is_v ? a.nv : a.nk;
+  c.C = is_v ? a.cv : a.ck;
+  c.P = c.C - 2;
+  c.src = is_v ? a.v : a.k;
+  c.cache = is_v ? a.vcache : a.kcache;
+  c.per_seq = static_cast<int64_t>(a.Hkv) * a.n_new;
+  c.nvec = static_cast<int64_t>(a.B) * c.per_seq;
+  if (threadIdx.x < kMaxLevels) {
+    const int s = threadIdx.x;
+    T.lev[s] = tab.levels[s];
+    T.thr[s] = (s < c.nl - 1) ? tab.thresholds[s] : INFINITY;
+    T.cost[s] = tab.cost[s];
+    const uint32_t f = tab.freq[s] ? tab.freq[s] : 1u;
+    T.freq[s] = tab.freq[s];
+    T.cum[s] = tab.cum[s];
+    EncSym e;
+    const uint32_t lg = 32 - __clz(f * f - 1u);  // ceil(log2 f^2); 0 for f = 1
+    e.k = 12 + (f == 1 ? 0u : lg);
+    e.m = static_cast<uint32_t>(((1ull << e.k) + f - 1) / f);
+    e.xmax = f << 12;
+    e.cum = tab.cum[s];
+    e.g = 4096u - f;
+    e.f = f;
+    e.pad0 = e.pad1 = 0;
+    T.es[s] = e;
+  }
+#pragma unroll
+  for (int j = 0; j < 7; ++j) c.t[j] = (j < c.nl - 1) ? tab.thresholds[j] : INFINITY;
+  return c;
+}
+
+// Drift counters of one warp.
+struct DriftCount {
+  unsigned moves = 0, containers = 0, fallbacks = 0;
+};
+
+// E6 for one over-long container, by the whole warp. On entry W.q holds the
+// symbols and u[k] this lane's coordinates lane + 32 k.
+template <bool kTwo>
+__device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T, WarpArea &W,
+                                          int64_t vd, uint16_t n16v, const float (&u)[4], int lane, DriftCount &dc) {
+  uint8_t *stk = W.stack + lane;
+  // Best move and key of the 4 symbols this lane owns (i = lane + 32 k).
+  float key[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = lane + 32 * k;
+    int tj;
+    key[k] = best_move(T, c.nl, W.q[i], u[k], &tj);
+    W.rank[i] = kNoRank;
+    W.tgt[i] = static_cast<uint8_t>(tj);
+  }
+  __syncwarp();
+  int ranked = 0;    // moves ranked so far
+  int applied = -1;  // number of moves in the result
+  bool exhausted = false;
+  while (applied < 0 && !exhausted) {
+    // Rank the next (up to) 32 moves: repeated arg-min over (key, index).
+    int added = 0;
+    for (; added < 32; ++added) {
+      float bk = key[0];
+      int bi = lane;
+#pragma unroll
+      for (int k = 1; k < 4; ++k)
+        if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const float ok = __shfl_xor_sync(kFull, bk, off);
+        const int oi = __shfl_xor_sync(kFull, bi, off);
+        if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
+      }
+      if (bk == INFINITY) break;  // no candidate left
+      if ((bi & 31) == lane) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (bi == lane + 32 * k) key[k] = INFINITY;
+        W.rank[bi] = static_cast<uint8_t>(ranked + added);
+      }
+    }
+    __syncwarp();
+    // Lane m encodes the string with moves 0 .. ranked + m applied (lanes
+    // m >= added too, with all ranked moves; their result is not used).
+    const int m_moves = ranked + lane;  // highest rank applied by this lane
     uint32_t x = 0;
-    const int len = rans_encode([&](int i) { return static_cast<uint32_t>(q[i]); }, T, stack, P, &x);
-    too_long = len > P;
-    uint8_t *dst = dst_of(lane, &dropped);
-    if (!too_long && dst) store_container(dst, C, W.norm16[lane], x, stack, len);
+    const int len = encode_bf<kTwo, false>(
+        [&](int i) {
+          const uint32_t r = W.rank[i];
+          return (r != kNoRank && static_cast<int>(r) <= m_moves) ? static_cast<uint32_t>(W.tgt[i])
+                                                                  : static_cast<uint32_t>(W.q[i]);
+        },
+        T.es, stk, &x);
+    const unsigned fit = __ballot_sync(kFull, lane < added && len <= c.P);
+    if (fit) {
+      const int win = __ffs(fit) - 1;
+      applied = ranked + win + 1;
+      if (lane == win) {
+        bool dr = false;
+        uint8_t *dst = c.dst_of(a, vd, &dr);
+        if (dst) store_container(dst, c.C, n16v, x, stk, len);
+      }
+    } else {
+      ranked += added;
+      exhausted = added < 32;
+    }
+    __syncwarp();
+  }
+  if (applied < 0) {
+    // Fallback (candidates exhausted): every symbol to the innermost level
+    // of its side, with the moves made so far counted.
+    const int hlf = c.nl / 2;
+    uint32_t x = 0;
+    const int len = encode_bf<kTwo, false>(
+        [&](int i) {
+          const uint32_t r = W.rank[i];
+          const uint32_t s = (r != kNoRank) ? W.tgt[i] : W.q[i];
+          return static_cast<uint32_t>(s >= static_cast<uint32_t>(hlf) ? hlf : hlf - 1);
+        },
+        T.es, stk, &x);
+    if (lane == 0) {
+      bool dr = false;
+      uint8_t *dst = c.dst_of(a, vd, &dr);
+      if (dst && len <= c.P) store_container(dst, c.C, n16v, x, stk, len);
+    }
+    applied = ranked;
+    ++dc.fallbacks;
+  }
+  dc.moves += static_cast<unsigned>(applied);
+  dc.containers += applied > 0 ? 1u : 0u;
+  __syncwarp();
+}
+
+__device__ __forceinline__ void add_stats(const AppendArgs &a, bool is_v, const DriftCount &dc, unsigned nf,
+                                          unsigned drops) {
+  if (!a.stats) return;
+  if (dc.moves) atomicAdd(is_v ? &a.stats->v_syms_drifted : &a.stats->k_syms_drifted, (unsigned long long)dc.moves);
+  if (dc.containers)
+    atomicAdd(is_v ? &a.stats->v_cont_drifted : &a.stats->k_cont_drifted, (unsigned long long)dc.containers);
+  if (dc.fallbacks) atomicAdd(&a.stats->overflow_fallbacks, (unsigned long long)dc.fallbacks);
+  if (nf) atomicAdd(&a.stats->nonfinite_inputs, (unsigned long long)nf);
+  if (drops) atomicAdd(&a.stats->dropped_writes, (unsigned long long)drops);
+}
+
+// Lane-per-vector body: 32 consecutive vectors per warp.
+template <bool kBF16, bool kTwo>
+__device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, WarpArea &W, bool is_v) {
+  const int lane = threadIdx.x & 31;
+  const StreamCtx c = stream_setup(a, T, is_v);
+  __syncthreads();
+  const int64_t v0 = (static_cast<int64_t>(blockIdx.x) * kAW + (threadIdx.x >> 5)) * 32;
+  if (v0 >= c.nvec) return;
+  const int64_t v = v0 + lane;
+  const bool valid = v < c.nvec;
+
+  // ---- phases 1 and 2: lane per vector ----
+  uint8_t *stk = W.stack + lane;
+  uint16_t n16 = 0;
+  bool nf = false, dropped = false, too_long = false;
+  if (valid) {
+    const int h = c.head_of(a, v);
+    uint32_t sw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
+    uint32_t pk[32];
+    lane_prepare<kBF16>(c.src, v, sw, c.t, pk, &n16, &nf);
+    uint32_t x = 0;
+    const int len = encode_bf<kTwo, true>([&](int i) { return __byte_perm(pk[i >> 2], 0u, 0x4440u + (i & 3)); },
+                                          T.es, stk, &x);
+    too_long = len > c.P;
+    uint8_t *dst = c.dst_of(a, v, &dropped);
+    if (!too_long && dst) store_container(dst, c.C, n16, x, stk, len);
   }
   unsigned drift_mask = __ballot_sync(kFull, too_long);
-  unsigned moves_total = 0, cont_drifted = 0, fallbacks = 0;
-  unsigned drops = __ballot_sync(kFull, dropped);
+  const unsigned nf_mask = __ballot_sync(kFull, valid && nf);
+  const unsigned drops = __ballot_sync(kFull, dropped);
 
   // ---- phase 3: warp per over-long container (E6 drift) ----
+  DriftCount dc;
   while (drift_mask) {
     const int vv = __ffs(drift_mask) - 1;
     drift_mask &= drift_mask - 1;
-    uint8_t *q = W.q + vv * kQStride;
-    const float *uu = W.u + vv * kUStride;
-    // Best move and key of the 4 symbols this lane owns (i = lane + 32 k).
-    float key[4];
-    int tj[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int i = lane + 32 * k;
-      key[k] = best_move(T, nl, q[i], uu[i], &tj[k]);
-      W.rank[i] = kNoRank;
-      W.tgt[i] = static_cast<uint8_t>(tj[k]);
-    }
+    const int64_t vd = v0 + vv;
+    float u[4];
+    uint16_t n16v;
+    bool nfv;
+    warp_prepare(a, c.src, vd, c.head_of(a, vd), c.t, lane, u, W.q, &n16v, &nfv);
     __syncwarp();
-    int ranked = 0;       // moves ranked so far
-    int applied = -1;     // number of moves in the result
-    bool exhausted = false;
-    while (applied < 0 && !exhausted) {
-      // Rank the next (up to) 32 moves: repeated arg-min over (key, index).
-      int added = 0;
-      for (; added < 32; ++added) {
-        float bk = key[0];
-        int bi = lane;
-#pragma unroll
-        for (int k = 1; k < 4; ++k)
-          if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          const float ok = __shfl_xor_sync(kFull, bk, off);
-          const int oi = __shfl_xor_sync(kFull, bi, off);
-          if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-        }
-        if (bk == INFINITY) break;  // no candidate left
-        if ((bi & 31) == lane) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            if (bi == lane + 32 * k) key[k] = INFINITY;
-          W.rank[bi] = static_cast<uint8_t>(ranked + added);
-        }
-      }
-      __syncwarp();
-      // Lane m (m < added) encodes the string with moves 0 .. ranked + m applied.
-      const int m_moves = ranked + lane;  // highest rank applied by this lane
-      int len = P + 1;
-      uint32_t x = 0;
-      uint8_t *stack = W.stack + lane * kStack;
-      if (lane < added)
-        len = rans_encode(
-            [&](int i) {
-              const uint32_t r = W.rank[i];
-              return (r != kNoRank && static_cast<int>(r) <= m_moves) ? static_cast<uint32_t>(W.tgt[i])
-                                                                      : static_cast<uint32_t>(q[i]);
-            },
-            T, stack, P, &x);
-      const unsigned fit = __ballot_sync(kFull, lane < added && len <= P);
-      if (fit) {
-        const int win = __ffs(fit) - 1;
-        applied = ranked + win + 1;
-        if (lane == win) {
-          bool dr = false;
-          uint8_t *dst = dst_of(vv, &dr);
-          if (dst) store_container(dst, C, W.norm16[vv], x, stack, len);
-        }
-      } else {
-        ranked += added;
-        exhausted = added < 32;
-      }
-      __syncwarp();
-    }
-    if (applied < 0) {
-      // Fallback (candidates exhausted): every symbol to the innermost level
-      // of its side, with the moves made so far counted.
-      const int hlf = nl / 2;
-      if (lane == 0) {
-        uint32_t x = 0;
-        uint8_t *stack = W.stack;
-        const int len = rans_encode(
-            [&](int i) {
-              const uint32_t r = W.rank[i];
-              const uint32_t s = (r != kNoRank) ? W.tgt[i] : q[i];
-              return static_cast<uint32_t>(s >= static_cast<uint32_t>(hlf) ? hlf : hlf - 1);
-            },
-            T, stack, P, &x);
-        bool dr = false;
-        uint8_t *dst = dst_of(vv, &dr);
-        if (dst && len <= P) store_container(dst, C, W.norm16[vv], x, stack, len);
-      }
-      applied = ranked;
-      ++fallbacks;
-    }
-    moves_total += static_cast<unsigned>(applied);
-    cont_drifted += applied > 0 ? 1u : 0u;
-    __syncwarp();
+    drift_one<kTwo>(a, c, T, W, vd, n16v, u, lane, dc);
   }
+  if (lane == 0) add_stats(a, is_v, dc, __popc(nf_mask), __popc(drops));
+}
 
-  if (a.stats && lane == 0) {
-    const unsigned nfs = [&]() {
-      unsigned c = 0;
-      for (int vv = 0; vv < nmine; ++vv) c += W.nonfinite[vv];
-      return c;
-    }();
-    if (moves_total) atomicAdd(is_v ? &a.stats->v_syms_drifted : &a.stats->k_syms_drifted, (unsigned long long)moves_total);
-    if (cont_drifted) atomicAdd(is_v ? &a.stats->v_cont_drifted : &a.stats->k_cont_drifted, (unsigned long long)cont_drifted);
-    if (fallbacks) atomicAdd(&a.stats->overflow_fallbacks, (unsigned long long)fallbacks);
-    if (nfs) atomicAdd(&a.stats->nonfinite_inputs, (unsigned long long)nfs);
-    if (drops) atomicAdd(&a.stats->dropped_writes, (unsigned long long)__popc(drops));
+// Warp-per-vector body for small appends (a decode step): many warps with
+// one vector each, so drift and latency spread over the whole GPU.
+template <bool kTwo>
+__device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, WarpArea &W, bool is_v) {
+  const int lane = threadIdx.x & 31;
+  const StreamCtx c = stream_setup(a, T, is_v);
+  __syncthreads();
+  const int64_t v = static_cast<int64_t>(blockIdx.x) * kAW + (threadIdx.x >> 5);
+  if (v >= c.nvec) return;
+  float u[4];
+  uint16_t n16;
+  bool nf;
+  warp_prepare(a, c.src, v, c.head_of(a, v), c.t, lane, u, W.q, &n16, &nf);
+  __syncwarp();
+  uint8_t *stk = W.stack + lane;
+  uint32_t x = 0;
+  const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(W.q[i]); }, T.es, stk, &x);
+  bool dropped = false;
+  uint8_t *dst = c.dst_of(a, v, &dropped);
+  DriftCount dc;
+  if (len <= c.P) {
+    if (lane == 0 && dst) store_container(dst, c.C, n16, x, stk, len);
+  } else {
+    __syncwarp();
+    drift_one<kTwo>(a, c, T, W, v, n16, u, lane, dc);
   }
+  if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u);
+}
+
+// One CTA = kAW warps of one stream (blockIdx.y: 0 = K, 1 = V).
+template <bool kBF16, bool kTwoK, bool kTwoV>
+__global__ void __launch_bounds__(kAW * 32, 3) append_lane_kernel(const AppendArgs a) {
+  __shared__ AppendTables T;
+  __shared__ WarpArea W[kAW];
+  const bool is_v = blockIdx.y == 1;
+  WarpArea &w = W[threadIdx.x >> 5];
+  if constexpr (kTwoK == kTwoV) {
+    lane_body<kBF16, kTwoK>(a, T, w, is_v);
+  } else {
+    if (is_v) lane_body<kBF16, kTwoV>(a, T, w, true);
+    else lane_body<kBF16, kTwoK>(a, T, w, false);
+  }
+}
+
+template <bool kTwoK, bool kTwoV>
+__global__ void __launch_bounds__(kAW * 32) append_warp_kernel(const AppendArgs a) {
+  __shared__ AppendTables T;
+  __shared__ WarpArea W[kAW];
+  const bool is_v = blockIdx.y == 1;
+  WarpArea &w = W[threadIdx.x >> 5];
+  if constexpr (kTwoK == kTwoV) {
+    warp_body<kTwoK>(a, T, w, is_v);
+  } else {
+    if (is_v) warp_body<kTwoV>(a, T, w, true);
+    else warp_body<kTwoK>(a, T, w, false);
+  }
+}
+
+template <bool kBF16, bool kTwoK, bool kTwoV>
+int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, cudaStream_t st) {
+  const int64_t per_cta = lanes ? static_cast<int64_t>(kAW) * 32 : kAW;
+  const int64_t gx = (nvec + per_cta - 1) / per_cta;
+  if (gx > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidConfiguration);
+  const dim3 grid(static_cast<unsigned>(gx), 2);
+  if (lanes) append_lane_kernel<kBF16, kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
+  else append_warp_kernel<kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
+  return static_cast<int>(cudaGetLastError());
+}
+
+template <bool kBF16>
+int launch_dtype(const AppendArgs &a, bool lanes, int64_t nvec, cudaStream_t st) {
+  if (a.two_k && a.two_v) return launch_two<kBF16, true, true>(a, lanes, nvec, st);
+  if (a.two_k) return launch_two<kBF16, true, false>(a, lanes, nvec, st);
+  if (a.two_v) return launch_two<kBF16, false, true>(a, lanes, nvec, st);
+  return launch_two<kBF16, false, false>(a, lanes, nvec, st);
 }
 
 }  // namespace
@@ -375,24 +585,14 @@ __global__ void __launch_bounds__(kAW * 32) append_kernel(const AppendArgs a, in
 int launch_append(const AppendArgs &a, void *stream) {
   if (a.ck > kMaxContainer || a.cv > kMaxContainer) return static_cast<int>(cudaErrorInvalidValue);
   const int64_t nvec = static_cast<int64_t>(a.B) * a.Hkv * a.n_new;
+  if (nvec == 0) return 0;
   int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Vectors per warp: 32 when there is enough work for every SM, fewer (down
-  // to 1) for small appends such as one decode step, so the work still
-  // spreads over all SMs.
-  int vpw = 32;
-  while (vpw > 1 && nvec < static_cast<int64_t>(vpw) * kAW * sms * 4) vpw >>= 1;
-  const int64_t per_cta = static_cast<int64_t>(kAW) * vpw;
-  const int64_t gx = (nvec + per_cta - 1) / per_cta;
-  if (gx > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidConfiguration);
-  const size_t smem = ((sizeof(AppendTables) + 15) & ~size_t(15)) + kAW * warp_area_bytes(vpw);
-  cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return static_cast<int>(e);
-  dim3 grid(static_cast<unsigned>(gx), 2);
-  append_kernel<<<grid, kAW * 32, smem, static_cast<cudaStream_t>(stream)>>>(a, vpw);
-  return static_cast<int>(cudaGetLastError());
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // Lane per vector once every SM gets a few full CTAs of 128 vectors per
+  // stream; below that, a warp per vector spreads the work wider.
+  const bool lanes = nvec >= static_cast<int64_t>(sms) * kAW * 32 * 2;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return a.dtype == DQ_BF16 ? launch_dtype<true>(a, lanes, nvec, st) : launch_dtype<false>(a, lanes, nvec, st);
 }
 
 }  // namespace dqi

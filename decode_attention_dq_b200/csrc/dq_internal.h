@@ -74,6 +74,7 @@ struct AppendArgs {
   int64_t T_cap;
   int ck, cv;       // container bytes
   int nk, nv;       // levels
+  bool two_k, two_v;  // the stream's table has a symbol with f < 16 (two pushes per step)
   dq_stats *stats;
 };
 int launch_append(const AppendArgs &a, void *stream);

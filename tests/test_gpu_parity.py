@@ -86,11 +86,18 @@ def test_decode_symbols_flags_corruption_like_oracle():
     assert set(np.unique(r_st)) >= {0, 1, 3}
 
 
+# Appends of up to ~38K vectors per stream run the warp-per-vector kernel on a
+# 148-SM B200, larger ones the lane-per-vector kernel: both are covered, for
+# fp32 (tiny) and bf16 inputs and every budget.
 APPEND_CASES = [
     ("tiny_b1_t256", 256, 2.26, 2.26),
     ("qwen3_8b_b16_t8k", 300, 2.26, 2.26),
     ("llama_b32_t32k_1p96", 160, 1.96, 1.96),
     ("llama_b32_t32k_3p0", 160, 3.0, 3.0),
+    ("tiny_b1_t256", 65536, 2.26, 2.26),
+    ("qwen3_8b_b16_t8k", 4096, 2.26, 2.26),
+    ("llama_b32_t32k_1p96", 4096, 1.96, 1.96),
+    ("llama_b32_t32k_3p0", 4096, 3.0, 3.0),
 ]
 
 
