@@ -30,7 +30,8 @@
 //     arithmetic), ranks the candidate moves by repeated arg-min (least key
 //     first, ties to the lower index), and lane m encodes the string with the
 //     first m+1 moves applied; the smallest m that fits is the greedy result.
-//     32 move counts are tried per pass.
+//     The first pass tries 8 move counts (32 in the warp-per-vector
+//     kernel), later ones 32.
 #include "dq_device.cuh"
 
 namespace dqi {
@@ -352,7 +353,8 @@ struct DriftCount {
 // symbols and u[k] this lane's coordinates lane + 32 k.
 template <bool kTwo>
 __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T, WarpArea &W,
-                                          int64_t vd, uint16_t n16v, const float (&u)[4], int lane, DriftCount &dc) {
+                                          int64_t vd, uint16_t n16v, const float (&u)[4], int lane, int first_batch,
+                                          DriftCount &dc) {
   uint8_t *stk = W.stack + lane;
   // Best move and key of the 4 symbols this lane owns (i = lane + 32 k).
   float key[4];
@@ -369,9 +371,11 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
   int applied = -1;  // number of moves in the result
   bool exhausted = false;
   while (applied < 0 && !exhausted) {
-    // Rank the next (up to) 32 moves: repeated arg-min over (key, index).
+    // Rank the next moves by repeated arg-min over (key, index):
+    // first_batch on the first pass, then up to 32 per pass.
+    const int batch = ranked == 0 ? first_batch : 32;
     int added = 0;
-    for (; added < 32; ++added) {
+    for (; added < batch; ++added) {
       float bk = key[0];
       int bi = lane;
 #pragma unroll
@@ -414,7 +418,7 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
       }
     } else {
       ranked += added;
-      exhausted = added < 32;
+      exhausted = added < batch;
     }
     __syncwarp();
   }
@@ -498,7 +502,8 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
     bool nfv;
     warp_prepare(a, c.src, vd, c.head_of(a, vd), c.t, lane, u, W.q, &n16v, &nfv);
     __syncwarp();
-    drift_one<kTwo>(a, c, T, W, vd, n16v, u, lane, dc);
+    // Most containers need a few moves: rank 8 first (throughput).
+    drift_one<kTwo>(a, c, T, W, vd, n16v, u, lane, 8, dc);
   }
   if (lane == 0) add_stats(a, is_v, dc, __popc(nf_mask), __popc(drops));
 }
@@ -527,7 +532,8 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
     if (lane == 0 && dst) store_container(dst, c.C, n16, x, stk, len);
   } else {
     __syncwarp();
-    drift_one<kTwo>(a, c, T, W, v, n16, u, lane, dc);
+    // One pass of 32 in most cases (latency of a small append).
+    drift_one<kTwo>(a, c, T, W, v, n16, u, lane, 32, dc);
   }
   if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u);
 }
