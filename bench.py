@@ -141,6 +141,30 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def replica_workload(w, rank):
+    """Each rank of a multi-GPU run is an independent replica with its own
+    sequences (same shapes, its own seed); rank 0 keeps the workload's seed."""
+    from decode_attention_dq_b200 import synth
+    return w if rank == 0 else synth.scaled(w, seed=w.seed + 1000 * rank, name=w.name)
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise maximum of a list of floats over all ranks (the slowest
+    rank's times); the values unchanged without a process group."""
+    if dist is None:
+        return list(values)
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(units_per_step_per_rank, world_size, ms_per_step):
+    """Throughput of the whole job: every rank's units over the slowest
+    rank's time per step."""
+    return units_per_step_per_rank * world_size / (ms_per_step * 1e-3)
+
+
 def dist_setup(args):
     import torch
     ws = int(os.environ.get("WORLD_SIZE", "1"))
@@ -168,9 +192,7 @@ def run_dq(args):
     dist = None
     if ws > 1:
         import torch.distributed as dist
-    w = synth.WORKLOADS[args.workload]
-    if rank:  # each replica its own sequences
-        w = synth.scaled(w, seed=w.seed + 1000 * rank, name=w.name)
+    w = replica_workload(synth.WORKLOADS[args.workload], rank)
     dev = torch.device("cuda", torch.cuda.current_device())
     tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
     ck, cv = tab.k.container_bytes, tab.v.container_bytes
@@ -247,13 +269,10 @@ def run_dq(args):
     clk = clocks.stop()
     elapsed_ms = e0.elapsed_time(e1)
     dec_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / args.steps
-    if dist is not None:
-        t = torch.tensor([elapsed_ms, dec_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, dec_ms = float(t[0]), float(t[1])
+    elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], dist, dev)
     ms_per_step = elapsed_ms / args.steps
     kv_tokens_step = w.B * T
-    value = kv_tokens_step * ws / (ms_per_step * 1e-3)
+    value = whole_job_rate(kv_tokens_step, ws, ms_per_step)
 
     # ---- e2e: host buffers, copies inside the timed region ----
     def step_e2e(s):
@@ -277,12 +296,8 @@ def run_dq(args):
     f1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = f0.elapsed_time(f1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = kv_tokens_step * ws / (e2e_ms / args.steps * 1e-3)
+    e2e_ms = max_over_ranks([f0.elapsed_time(f1)], dist, dev)[0]
+    e2e_value = whole_job_rate(kv_tokens_step, ws, e2e_ms / args.steps)
     h2d = (host_k[0].numel() + host_v[0].numel() + host_q[0].numel()) * host_k[0].element_size()
     d2h = out_host.numel() * out_host.element_size()
     st = dq.stats_dict(stats)
