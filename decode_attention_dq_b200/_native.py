@@ -23,7 +23,8 @@ STATS_FIELDS = ("k_syms_drifted", "v_syms_drifted", "k_cont_drifted", "v_cont_dr
 EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_stream_table",
             "dq_get_stream_design", "dq_get_signs", "dq_append_kv", "dq_decode_workspace_bytes",
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",
-            "dq_design_stream", "dq_decode_attention_noalloc")
+            "dq_design_stream", "dq_decode_attention_noalloc", "dq_append_workspace_bytes",
+            "dq_append_kv_ws")
 
 
 class DqConfig(C.Structure):
@@ -69,6 +70,10 @@ def load():
     lib.dq_get_signs.argtypes = [vp, vp]
     lib.dq_append_kv.argtypes = [vp, vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, vp, vp, vp,
                                  i64, vp, vp]
+    lib.dq_append_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int]
+    lib.dq_append_workspace_bytes.restype = C.c_size_t
+    lib.dq_append_kv_ws.argtypes = [vp, vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, vp, vp, vp,
+                                    i64, vp, C.c_size_t, vp, vp]
     lib.dq_decode_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int, i64]
     lib.dq_decode_workspace_bytes.restype = C.c_size_t
     lib.dq_decode_attention.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int, C.c_int,
@@ -207,19 +212,35 @@ def containers_of(cache: torch.Tensor) -> torch.Tensor:
     return cache.reshape(B, H, T_cap // 32, C, 32).transpose(-1, -2).reshape(B, H, T_cap, C).contiguous()
 
 
+def dq_append_workspace_bytes(tab: Tables, B: int, Hkv: int, n_new: int) -> int:
+    return int(load().dq_append_workspace_bytes(tab.handle, B, Hkv, n_new))
+
+
 def dq_append_kv(tab: Tables, k: torch.Tensor, v: torch.Tensor, start_pos: torch.Tensor,
                  kcache: torch.Tensor, vcache: torch.Tensor, stats: torch.Tensor | None = None,
-                 stream=None) -> None:
+                 stream=None, workspace: torch.Tensor | None = None) -> None:
     """k, v: [B, Hkv, n_new, 128] (f32/bf16, contiguous, CUDA); start_pos int32 [B];
-    caches uint8 [B, Hkv, T_cap, C] holding the interleaved layout (see new_cache)."""
+    caches uint8 [B, Hkv, T_cap, C] holding the interleaved layout (see new_cache).
+    Calls dq_append_kv_ws; without `workspace` one is taken from PyTorch's
+    allocator on the caches' device. workspace=False calls dq_append_kv (drift
+    inside the encode kernel)."""
     B, Hkv, n_new, d = k.shape
     assert d == 128 and v.shape == k.shape and k.dtype == v.dtype
     assert k.is_contiguous() and v.is_contiguous() and kcache.is_contiguous() and vcache.is_contiguous()
     assert start_pos.dtype == torch.int32 and kcache.dtype == torch.uint8
     T_cap = kcache.shape[2]
-    _check("dq_append_kv", load().dq_append_kv(
+    if workspace is False:
+        _check("dq_append_kv", load().dq_append_kv(
+            tab.handle, _ptr(k), _ptr(v), _dtype_code(k), B, Hkv, n_new, _ptr(start_pos),
+            _ptr(kcache), _ptr(vcache), T_cap, _ptr(stats), _stream(stream)))
+        return
+    if workspace is None:
+        nbytes = dq_append_workspace_bytes(tab, B, Hkv, n_new)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=kcache.device)
+    _check("dq_append_kv_ws", load().dq_append_kv_ws(
         tab.handle, _ptr(k), _ptr(v), _dtype_code(k), B, Hkv, n_new, _ptr(start_pos),
-        _ptr(kcache), _ptr(vcache), T_cap, _ptr(stats), _stream(stream)))
+        _ptr(kcache), _ptr(vcache), T_cap, _ptr(workspace), workspace.numel(), _ptr(stats),
+        _stream(stream)))
 
 
 def dq_decode_workspace_bytes(tab: Tables, B: int, Hq: int, Hkv: int, T_max: int) -> int:

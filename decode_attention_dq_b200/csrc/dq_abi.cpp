@@ -314,9 +314,21 @@ int dq_get_signs(const dq_tables *t, int8_t *signs) {
   return DQ_OK;
 }
 
+size_t dq_append_workspace_bytes(const dq_tables *t, int B, int Hkv, int n_new) {
+  if (!t || B < 0 || Hkv < 1 || n_new < 0) return 0;
+  return dqi::append_workspace_bytes(static_cast<int64_t>(B) * Hkv * n_new);
+}
+
 int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv,
                  int n_new, const int32_t *d_start_pos, uint8_t *d_kcache, uint8_t *d_vcache,
                  int64_t T_cap, dq_stats *d_stats, void *stream) {
+  return dq_append_kv_ws(t, k, v, dtype, B, Hkv, n_new, d_start_pos, d_kcache, d_vcache, T_cap, nullptr, 0,
+                         d_stats, stream);
+}
+
+int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv, int n_new,
+                    const int32_t *d_start_pos, uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
+                    void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream) {
   try {
     if (!t || !k || !v || !d_start_pos || !d_kcache || !d_vcache) return DQ_ERR_NULL;
     if (dtype != DQ_F32 && dtype != DQ_BF16) return DQ_ERR_DTYPE;
@@ -345,6 +357,14 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, in
     a.two_k = has_small_freq(t->k);
     a.two_v = has_small_freq(t->v);
     a.stats = d_stats;
+    const int64_t nvec = static_cast<int64_t>(B) * Hkv * n_new;
+    if (d_workspace) {
+      if (!aligned(d_workspace, 16)) return DQ_ERR_ALIGN;
+      if (ws_bytes < dqi::append_workspace_bytes(nvec)) return DQ_ERR_WORKSPACE;
+      a.drift_count = static_cast<uint32_t *>(d_workspace);
+      a.drift_list = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(d_workspace) + 256);
+      a.list_cap = nvec;
+    }
     int e = dqi::launch_append(a, stream);
     return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
   } catch (...) {

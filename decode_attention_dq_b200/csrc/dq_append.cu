@@ -490,9 +490,19 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
   unsigned drift_mask = __ballot_sync(kFull, too_long);
   const unsigned nf_mask = __ballot_sync(kFull, valid && nf);
   const unsigned drops = __ballot_sync(kFull, dropped);
+  DriftCount dc;
+
+  if (a.drift_list) {
+    // List the over-long containers for the drift kernel (one atomic per warp).
+    uint32_t base = 0;
+    if (lane == 0 && drift_mask) base = atomicAdd(&a.drift_count[is_v ? 1 : 0], static_cast<uint32_t>(__popc(drift_mask)));
+    base = __shfl_sync(kFull, base, 0);
+    if (too_long)
+      a.drift_list[(is_v ? a.list_cap : 0) + base + __popc(drift_mask & ((1u << lane) - 1u))] = static_cast<uint32_t>(v);
+    drift_mask = 0;
+  }
 
   // ---- phase 3: warp per over-long container (E6 drift) ----
-  DriftCount dc;
   while (drift_mask) {
     const int vv = __ffs(drift_mask) - 1;
     drift_mask &= drift_mask - 1;
@@ -538,6 +548,43 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u);
 }
 
+// E6 for the containers listed by the lane-per-vector kernel: each warp of
+// a persistent grid takes list entries gridDim.x * kAW apart.
+template <bool kTwo>
+__device__ __forceinline__ void drift_body(const AppendArgs &a, AppendTables &T, WarpArea &W, bool is_v) {
+  const int lane = threadIdx.x & 31;
+  const StreamCtx c = stream_setup(a, T, is_v);
+  __syncthreads();
+  const uint32_t n = a.drift_count[is_v ? 1 : 0];
+  const uint32_t *list = a.drift_list + (is_v ? a.list_cap : 0);
+  const uint32_t stride = gridDim.x * kAW;
+  DriftCount dc;
+  for (uint32_t i = blockIdx.x * kAW + (threadIdx.x >> 5); i < n; i += stride) {
+    const int64_t vd = list[i];
+    float u[4];
+    uint16_t n16;
+    bool nf;
+    warp_prepare(a, c.src, vd, c.head_of(a, vd), c.t, lane, u, W.q, &n16, &nf);
+    __syncwarp();
+    drift_one<kTwo>(a, c, T, W, vd, n16, u, lane, 8, dc);
+  }
+  if (lane == 0) add_stats(a, is_v, dc, 0u, 0u);
+}
+
+template <bool kTwoK, bool kTwoV>
+__global__ void __launch_bounds__(kAW * 32) append_drift_kernel(const AppendArgs a) {
+  __shared__ AppendTables T;
+  __shared__ WarpArea W[kAW];
+  const bool is_v = blockIdx.y == 1;
+  WarpArea &w = W[threadIdx.x >> 5];
+  if constexpr (kTwoK == kTwoV) {
+    drift_body<kTwoK>(a, T, w, is_v);
+  } else {
+    if (is_v) drift_body<kTwoV>(a, T, w, true);
+    else drift_body<kTwoK>(a, T, w, false);
+  }
+}
+
 // One CTA = kAW warps of one stream (blockIdx.y: 0 = K, 1 = V).
 template <bool kBF16, bool kTwoK, bool kTwoV>
 __global__ void __launch_bounds__(kAW * 32, 3) append_lane_kernel(const AppendArgs a) {
@@ -568,22 +615,33 @@ __global__ void __launch_bounds__(kAW * 32) append_warp_kernel(const AppendArgs 
 }
 
 template <bool kBF16, bool kTwoK, bool kTwoV>
-int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, cudaStream_t st) {
+int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, int sms, cudaStream_t st) {
   const int64_t per_cta = lanes ? static_cast<int64_t>(kAW) * 32 : kAW;
   const int64_t gx = (nvec + per_cta - 1) / per_cta;
   if (gx > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidConfiguration);
   const dim3 grid(static_cast<unsigned>(gx), 2);
-  if (lanes) append_lane_kernel<kBF16, kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
-  else append_warp_kernel<kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
+  if (!lanes) {
+    append_warp_kernel<kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
+    return static_cast<int>(cudaGetLastError());
+  }
+  if (a.drift_list) {
+    const cudaError_t e = cudaMemsetAsync(a.drift_count, 0, 2 * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return static_cast<int>(e);
+  }
+  append_lane_kernel<kBF16, kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || !a.drift_list) return static_cast<int>(e);
+  // Drift: a persistent grid of 4 CTAs per SM and stream walks the lists.
+  append_drift_kernel<kTwoK, kTwoV><<<dim3(static_cast<unsigned>(4 * sms), 2), kAW * 32, 0, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 
 template <bool kBF16>
-int launch_dtype(const AppendArgs &a, bool lanes, int64_t nvec, cudaStream_t st) {
-  if (a.two_k && a.two_v) return launch_two<kBF16, true, true>(a, lanes, nvec, st);
-  if (a.two_k) return launch_two<kBF16, true, false>(a, lanes, nvec, st);
-  if (a.two_v) return launch_two<kBF16, false, true>(a, lanes, nvec, st);
-  return launch_two<kBF16, false, false>(a, lanes, nvec, st);
+int launch_dtype(const AppendArgs &a, bool lanes, int64_t nvec, int sms, cudaStream_t st) {
+  if (a.two_k && a.two_v) return launch_two<kBF16, true, true>(a, lanes, nvec, sms, st);
+  if (a.two_k) return launch_two<kBF16, true, false>(a, lanes, nvec, sms, st);
+  if (a.two_v) return launch_two<kBF16, false, true>(a, lanes, nvec, sms, st);
+  return launch_two<kBF16, false, false>(a, lanes, nvec, sms, st);
 }
 
 }  // namespace
@@ -597,8 +655,15 @@ int launch_append(const AppendArgs &a, void *stream) {
   // Lane per vector once every SM gets a few full CTAs of 128 vectors per
   // stream; below that, a warp per vector spreads the work wider.
   const bool lanes = nvec >= static_cast<int64_t>(sms) * kAW * 32 * 2;
+  AppendArgs b = a;
+  // The drift list holds 32-bit vector indices, one slot per vector.
+  if (!lanes || b.list_cap < nvec || nvec > 0xFFFFFFFFll) b.drift_list = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return a.dtype == DQ_BF16 ? launch_dtype<true>(a, lanes, nvec, st) : launch_dtype<false>(a, lanes, nvec, st);
+  return b.dtype == DQ_BF16 ? launch_dtype<true>(b, lanes, nvec, sms, st) : launch_dtype<false>(b, lanes, nvec, sms, st);
+}
+
+size_t append_workspace_bytes(int64_t nvec) {
+  return 256 + 2 * static_cast<size_t>(nvec) * sizeof(uint32_t);
 }
 
 }  // namespace dqi

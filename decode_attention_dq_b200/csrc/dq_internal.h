@@ -76,7 +76,16 @@ struct AppendArgs {
   int nk, nv;       // levels
   bool two_k, two_v;  // the stream's table has a symbol with f < 16 (two pushes per step)
   dq_stats *stats;
+  // Optional drift list (workspace): over-long containers of the
+  // lane-per-vector kernel are listed here ([2][list_cap] vector indices, K
+  // then V; counts in drift_count[2]) and drifted by a separate kernel.
+  // nullptr: drift runs inside the encode kernel.
+  uint32_t *drift_list;
+  uint32_t *drift_count;
+  int64_t list_cap;
 };
+// Bytes of the optional append workspace for nvec vectors per stream.
+size_t append_workspace_bytes(int64_t nvec);
 int launch_append(const AppendArgs &a, void *stream);
 
 struct DecodeArgs {

@@ -146,7 +146,8 @@ def prefill_cache(tab, w: Workload, kcache, vcache, n_tokens: int, seqs_per_call
     sequences (the inputs are drawn on the host, then copied to the device).
     With `timings`, each dq_append_kv call is bracketed by CUDA events on the
     current stream and (start event, end event, vectors per stream) is
-    appended to the list."""
+    appended to the list; the first call is then made twice and only its
+    second run is timed (the first also loads the kernels)."""
     from ._native import dq_append_kv  # local import: synth itself needs no GPU
 
     for b0 in range(0, w.B, seqs_per_call):
@@ -160,6 +161,8 @@ def prefill_cache(tab, w: Workload, kcache, vcache, n_tokens: int, seqs_per_call
             b1 - b0, w.Hkv, n_tokens, 128)
         start = torch.zeros(b1 - b0, dtype=torch.int32, device=kcache.device)
         if timings is not None:
+            if b0 == 0:  # untimed first run (same inputs, same containers)
+                dq_append_kv(tab, kt, vt, start, kcache[b0:b1], vcache[b0:b1])
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
         dq_append_kv(tab, kt, vt, start, kcache[b0:b1], vcache[b0:b1], stats=stats)

@@ -173,6 +173,25 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype,
                  uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
                  dq_stats *d_stats, void *stream);
 
+/* Bytes of the optional workspace of dq_append_kv_ws for these shapes:
+ * 256 + 8 * B * Hkv * n_new (a list of the over-long containers of each
+ * stream). Returns 0 on invalid shapes. */
+size_t dq_append_workspace_bytes(const dq_tables *t, int B, int Hkv, int n_new);
+
+/* dq_append_kv with a caller-provided device workspace (16-byte aligned, at
+ * least dq_append_workspace_bytes; contents need not be initialised). Large
+ * appends then list their over-long containers there and drift them ([news]
+ * "Drift: Bending Variable Back to Fixed") in a separate kernel that runs
+ * at higher occupancy than the encode kernel; the containers are the same
+ * bytes as with dq_append_kv. d_workspace NULL gives dq_append_kv. Calls
+ * sharing a workspace must not overlap on the GPU. DQ_ERR_WORKSPACE if
+ * ws_bytes is too small, DQ_ERR_ALIGN if the workspace is misaligned. */
+int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype,
+                    int B, int Hkv, int n_new, const int32_t *d_start_pos,
+                    uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
+                    void *d_workspace, size_t ws_bytes, dq_stats *d_stats,
+                    void *stream);
+
 /* Bytes of device workspace dq_decode_attention needs for these shapes
  * (token-group prefix sums and the warps' partial softmax states: about
  * (B*Hkv + SMs*warps_per_SM) * G * 520 bytes, G = Hq/Hkv). Depends only on

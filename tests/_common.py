@@ -45,7 +45,7 @@ def flat(cache):
     return dq.containers_of(cache).cpu().numpy()
 
 
-def gpu_append_all(tab, K, V, dtype, T_cap=None, stats=None):
+def gpu_append_all(tab, K, V, dtype, T_cap=None, stats=None, workspace=None):
     """Append all T tokens of K, V (numpy float32) through dq_append_kv."""
     B, H, T, _ = K.shape
     T_cap = t_cap_for(T) if T_cap is None else T_cap
@@ -54,7 +54,7 @@ def gpu_append_all(tab, K, V, dtype, T_cap=None, stats=None):
     kc = torch.zeros((B, H, T_cap, tab.k.container_bytes), dtype=torch.uint8, device="cuda")
     vc = torch.zeros((B, H, T_cap, tab.v.container_bytes), dtype=torch.uint8, device="cuda")
     start = torch.zeros(B, dtype=torch.int32, device="cuda")
-    dq.dq_append_kv(tab, kt, vt, start, kc, vc, stats=stats)
+    dq.dq_append_kv(tab, kt, vt, start, kc, vc, stats=stats, workspace=workspace)
     return kc, vc
 
 

@@ -101,8 +101,9 @@ APPEND_CASES = [
 ]
 
 
+@pytest.mark.parametrize("inline_drift", [False, True])
 @pytest.mark.parametrize("wname,T,kb,vb", APPEND_CASES)
-def test_append_bit_exact(wname, T, kb, vb):
+def test_append_bit_exact(wname, T, kb, vb, inline_drift):
     w = synth.WORKLOADS[wname]
     w = synth.scaled(w, B=min(w.B, 2), T=T)
     K, V, _ = cm.inputs(w)
@@ -110,7 +111,11 @@ def test_append_bit_exact(wname, T, kb, vb):
     lib = cm.lib_tables(w.Hkv, kb, vb)
     rk, rv, _, _, kst, vst = o.encode_cache(ref, K, V)
     stats = dq.new_stats()
-    kc, vc = cm.gpu_append_all(lib, K, V, w.torch_dtype, stats=stats)
+    # inline_drift: dq_append_kv without a workspace (drift inside the encode
+    # kernel); otherwise large appends list their over-long containers for
+    # the separate drift kernel.
+    kc, vc = cm.gpu_append_all(lib, K, V, w.torch_dtype, stats=stats,
+                               workspace=False if inline_drift else None)
     torch.cuda.synchronize()
     kf, vf = cm.flat(kc), cm.flat(vc)
     np.testing.assert_array_equal(kf[:, :, :T], rk)
