@@ -12,6 +12,8 @@ per step); the HBM rate of the compressed bytes and the dominant kernel's
 roofline fraction are reported beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dq|reference]
+                  [--workload NAME] [--paged]
+--paged keeps the caches in page pools behind a shuffled page table.
 Under torchrun every rank runs an independent replica (no data-path
 collective): value = all ranks' KV tokens / the slowest rank's time.
 """
@@ -199,13 +201,23 @@ def run_dq(args):
     T = w.T
     T_cap = (T + 31) // 32 * 32
     G = w.Hq // w.Hkv
-    kc = torch.zeros((w.B, w.Hkv, T_cap, ck), dtype=torch.uint8, device=dev)
-    vc = torch.zeros((w.B, w.Hkv, T_cap, cv), dtype=torch.uint8, device=dev)
+    page_table = None
+    if args.paged:
+        # Pages of 32 tokens handed out in a shuffled order from one pool.
+        max_pages = T_cap // 32
+        num_pages = w.B * max_pages
+        perm = np.random.default_rng(w.seed).permutation(num_pages).astype(np.int32)
+        page_table = torch.from_numpy(perm.reshape(w.B, max_pages)).to(dev)
+        kc = dq.new_pool(num_pages, w.Hkv, ck, dev)
+        vc = dq.new_pool(num_pages, w.Hkv, cv, dev)
+    else:
+        kc = torch.zeros((w.B, w.Hkv, T_cap, ck), dtype=torch.uint8, device=dev)
+        vc = torch.zeros((w.B, w.Hkv, T_cap, cv), dtype=torch.uint8, device=dev)
     prefill_stats = dq.new_stats(dev)
     t0 = time.time()
     enc_timings = []
     synth.prefill_cache(tab, w, kc, vc, T - 1, stats=prefill_stats, threads=args.threads,
-                        timings=enc_timings)
+                        timings=enc_timings, page_table=page_table)
     torch.cuda.synchronize()
     prefill_s = time.time() - t0
     pstats = dq.stats_dict(prefill_stats)
@@ -234,12 +246,29 @@ def run_dq(args):
     stats = dq.new_stats(dev)
     stream = torch.cuda.current_stream()
 
+    app_ws = torch.empty(max(16, dq.dq_append_workspace_bytes(tab, w.B, w.Hkv, 1)), dtype=torch.uint8,
+                         device=dev)
+
+    def append(i):
+        if page_table is None:
+            dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kc, vc, stats=stats, stream=stream, workspace=app_ws)
+        else:
+            dq.dq_append_kv_paged(tab, dev_k[i], dev_v[i], start, kc, vc, page_table, stats=stats,
+                                  stream=stream, workspace=app_ws)
+
+    def decode(i):
+        if page_table is None:
+            dq.dq_decode_attention(tab, dev_q[i], kc, vc, seq, T, out, wsp, stats=stats, stream=stream)
+        else:
+            dq.dq_decode_attention_paged(tab, dev_q[i], kc, vc, page_table, seq, T, out, wsp, stats=stats,
+                                         stream=stream)
+
     def step(s, e_dec0=None, e_dec1=None):
         i = s % nsteps_inputs
-        dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kc, vc, stats=stats, stream=stream)
+        append(i)
         if e_dec0 is not None:
             e_dec0.record(stream)
-        dq.dq_decode_attention(tab, dev_q[i], kc, vc, seq, T, out, wsp, stats=stats, stream=stream)
+        decode(i)
         if e_dec1 is not None:
             e_dec1.record(stream)
 
@@ -280,8 +309,8 @@ def run_dq(args):
         dev_k[i].copy_(host_k[i], non_blocking=True)
         dev_v[i].copy_(host_v[i], non_blocking=True)
         dev_q[i].copy_(host_q[i], non_blocking=True)
-        dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kc, vc, stats=stats, stream=stream)
-        dq.dq_decode_attention(tab, dev_q[i], kc, vc, seq, T, out, wsp, stats=stats, stream=stream)
+        append(i)
+        decode(i)
         out_host.copy_(out, non_blocking=True)
 
     for s in range(2):
@@ -322,10 +351,12 @@ def run_dq(args):
                        "k_bits_per_value": w.k_bits, "v_bits_per_value": w.v_bits,
                        "k_container_bytes": ck, "v_container_bytes": cv,
                        "l2": "inputs larger than L2 (%.0f MB of containers read per step)" % (comp_bytes / 1e6),
+                       "cache": "paged: 32-token pages in a shuffled order" if args.paged else "contiguous",
                        "parallelism": "replicas x%d" % ws},
             "hbm_gbs": hbm_gbs,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tlaneop/s",
-                         "frac": achieved / alu_peak, "traffic": decode_traffic(token_heads, ck, cv),
+                         "frac": achieved / alu_peak,
+                         "traffic": None if args.paged else decode_traffic(token_heads, ck, cv),
                          "traffic_note": "decode_split_kernel DRAM bytes per launch, scaled from an ncu "
                                          "capture of the 32-sequence case by token-heads",
                          "algorithmic_bytes": comp_bytes,
@@ -481,6 +512,7 @@ def main():
     ap.add_argument("--threads", type=int, default=max(4, min(32, os.cpu_count() or 8)))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--paged", action="store_true", help="page pools and a shuffled page table")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -9,7 +9,8 @@ thin ctypes binding (argument marshalling only) plus seeded synthetic inputs.
 """
 from ._native import (DQ_BF16, DQ_F32, DQ_STREAM_K, DQ_STREAM_V, DqConfig, DqError,  # noqa: F401
                       Tables, containers_of, dq_append_kv, dq_append_workspace_bytes, dq_build_tables, dq_config_default,
-                      dq_decode_attention, dq_decode_attention_noalloc,
+                      dq_append_kv_paged, dq_decode_attention, dq_decode_attention_noalloc,
+                      dq_decode_attention_paged, new_pool,
                       dq_decode_symbols, dq_decode_workspace_bytes,
                       dq_design_stream, dq_error_string, load, new_cache, new_stats,
                       stats_dict)

@@ -19,12 +19,12 @@ DQ_F32, DQ_BF16 = 0, 1
 DQ_STREAM_K, DQ_STREAM_V = 0, 1
 STATS_FIELDS = ("k_syms_drifted", "v_syms_drifted", "k_cont_drifted", "v_cont_drifted",
                 "overflow_fallbacks", "integrity_errors", "nonfinite_inputs",
-                "dropped_writes", "clamped_lengths")
+                "dropped_writes", "clamped_lengths", "bad_pages")
 EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_stream_table",
             "dq_get_stream_design", "dq_get_signs", "dq_append_kv", "dq_decode_workspace_bytes",
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",
             "dq_design_stream", "dq_decode_attention_noalloc", "dq_append_workspace_bytes",
-            "dq_append_kv_ws")
+            "dq_append_kv_ws", "dq_append_kv_paged", "dq_decode_attention_paged")
 
 
 class DqConfig(C.Structure):
@@ -74,6 +74,11 @@ def load():
     lib.dq_append_workspace_bytes.restype = C.c_size_t
     lib.dq_append_kv_ws.argtypes = [vp, vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, vp, vp, vp,
                                     i64, vp, C.c_size_t, vp, vp]
+    lib.dq_append_kv_paged.argtypes = [vp, vp, vp, C.c_int, C.c_int, C.c_int, C.c_int, vp, vp, vp,
+                                       i64, vp, i64, vp, C.c_size_t, vp, vp]
+    lib.dq_decode_attention_paged.argtypes = [vp, vp, C.c_int, vp, vp, i64, vp, i64, vp, C.c_int,
+                                              C.c_int, C.c_int, i64, C.c_float, vp, C.c_int, vp,
+                                              C.c_size_t, vp, vp]
     lib.dq_decode_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, C.c_int, i64]
     lib.dq_decode_workspace_bytes.restype = C.c_size_t
     lib.dq_decode_attention.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int, C.c_int,
@@ -188,7 +193,7 @@ def dq_build_tables(cfg: DqConfig | None = None, **overrides) -> Tables:
 
 
 def new_stats(device=None) -> torch.Tensor:
-    """A zeroed device dq_stats (9 x uint64)."""
+    """A zeroed device dq_stats (one uint64 per field of STATS_FIELDS)."""
     return torch.zeros(len(STATS_FIELDS), dtype=torch.int64, device=device or "cuda")
 
 
@@ -308,3 +313,45 @@ def dq_design_stream(n_levels: int, container_bytes: int, rate_offset: float = 0
     return dict(levels=list(lev)[:n], thresholds=list(thr)[:n - 1], freq=list(f)[:n],
                 cum=list(cum)[:n + 1], cost=list(cost)[:n], lam=lam.value, entropy=ent.value,
                 mse=mse.value)
+
+
+def new_pool(num_pages: int, Hkv: int, C: int, device=None) -> torch.Tensor:
+    """Zeroed uint8 page pool [num_pages, Hkv, C, 32] (pages of 32 tokens)."""
+    return torch.zeros((num_pages, Hkv, C, 32), dtype=torch.uint8, device=device or "cuda")
+
+
+def dq_append_kv_paged(tab: Tables, k: torch.Tensor, v: torch.Tensor, start_pos: torch.Tensor,
+                       kpool: torch.Tensor, vpool: torch.Tensor, page_table: torch.Tensor,
+                       stats: torch.Tensor | None = None, stream=None,
+                       workspace: torch.Tensor | None = None) -> None:
+    """Append into page pools [num_pages, Hkv, C, 32] through page_table
+    int32 [B, max_pages] (see dq_append_kv for the other arguments)."""
+    B, Hkv, n_new, d = k.shape
+    assert d == 128 and v.shape == k.shape and k.dtype == v.dtype
+    assert k.is_contiguous() and v.is_contiguous() and kpool.is_contiguous() and vpool.is_contiguous()
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous() and page_table.shape[0] == B
+    if workspace is None:
+        nbytes = dq_append_workspace_bytes(tab, B, Hkv, n_new)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=kpool.device)
+    _check("dq_append_kv_paged", load().dq_append_kv_paged(
+        tab.handle, _ptr(k), _ptr(v), _dtype_code(k), B, Hkv, n_new, _ptr(start_pos),
+        _ptr(kpool), _ptr(vpool), kpool.shape[0], _ptr(page_table), page_table.shape[1],
+        _ptr(workspace), workspace.numel(), _ptr(stats), _stream(stream)))
+
+
+def dq_decode_attention_paged(tab: Tables, q: torch.Tensor, kpool: torch.Tensor, vpool: torch.Tensor,
+                              page_table: torch.Tensor, seq_lens: torch.Tensor, T_max: int,
+                              out: torch.Tensor, workspace: torch.Tensor, sm_scale: float | None = None,
+                              stats: torch.Tensor | None = None, stream=None) -> None:
+    """Decode attention over page pools (see dq_decode_attention)."""
+    B, Hq, d = q.shape
+    Hkv = kpool.shape[1]
+    assert d == 128 and q.is_contiguous() and out.is_contiguous() and seq_lens.dtype == torch.int32
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous()
+    if sm_scale is None:
+        sm_scale = 128 ** -0.5
+    _check("dq_decode_attention_paged", load().dq_decode_attention_paged(
+        tab.handle, _ptr(q), _dtype_code(q), _ptr(kpool), _ptr(vpool), kpool.shape[0],
+        _ptr(page_table), page_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, T_max, float(sm_scale),
+        _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(), _ptr(stats),
+        _stream(stream)))

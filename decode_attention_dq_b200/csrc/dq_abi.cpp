@@ -326,9 +326,11 @@ int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype, in
                          d_stats, stream);
 }
 
-int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv, int n_new,
-                    const int32_t *d_start_pos, uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
-                    void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream) {
+// Shared by dq_append_kv_ws (page_table NULL) and dq_append_kv_paged.
+static int append_core(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv, int n_new,
+                       const int32_t *d_start_pos, uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
+                       void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream,
+                       const int32_t *page_table, int64_t max_pages, int64_t num_pages) {
   try {
     if (!t || !k || !v || !d_start_pos || !d_kcache || !d_vcache) return DQ_ERR_NULL;
     if (dtype != DQ_F32 && dtype != DQ_BF16) return DQ_ERR_DTYPE;
@@ -365,6 +367,9 @@ int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype,
       a.drift_list = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(d_workspace) + 256);
       a.list_cap = nvec;
     }
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.num_pages = num_pages;
     int e = dqi::launch_append(a, stream);
     return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
   } catch (...) {
@@ -372,15 +377,36 @@ int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype,
   }
 }
 
+int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv, int n_new,
+                    const int32_t *d_start_pos, uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
+                    void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream) {
+  return append_core(t, k, v, dtype, B, Hkv, n_new, d_start_pos, d_kcache, d_vcache, T_cap, d_workspace, ws_bytes,
+                     d_stats, stream, nullptr, 0, 0);
+}
+
+int dq_append_kv_paged(const dq_tables *t, const void *k, const void *v, int dtype, int B, int Hkv, int n_new,
+                       const int32_t *d_start_pos, uint8_t *d_kpool, uint8_t *d_vpool, int64_t num_pages,
+                       const int32_t *d_page_table, int64_t max_pages, void *d_workspace, size_t ws_bytes,
+                       dq_stats *d_stats, void *stream) {
+  if (!d_page_table) return DQ_ERR_NULL;
+  if (num_pages < 1 || max_pages < 1 || max_pages > (int64_t(1) << 40) || num_pages > (int64_t(1) << 31))
+    return DQ_ERR_SHAPE;
+  if (!aligned(d_page_table, 4)) return DQ_ERR_ALIGN;
+  return append_core(t, k, v, dtype, B, Hkv, n_new, d_start_pos, d_kpool, d_vpool, 32 * max_pages, d_workspace,
+                     ws_bytes, d_stats, stream, d_page_table, max_pages, num_pages);
+}
+
 size_t dq_decode_workspace_bytes(const dq_tables *t, int B, int Hq, int Hkv, int64_t T_max) {
   if (!t || B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv || T_max < 0) return 0;
   return ws_layout(t, B, Hkv, Hq / Hkv).total;
 }
 
-int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
-                        const uint8_t *d_vcache, const int32_t *d_seq_lens, int B, int Hq, int Hkv,
-                        int64_t T_cap, int64_t T_max, float sm_scale, void *out, int out_dtype,
-                        void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream) {
+// Shared by dq_decode_attention (page_table NULL) and dq_decode_attention_paged.
+static int decode_core(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
+                       const uint8_t *d_vcache, const int32_t *d_seq_lens, int B, int Hq, int Hkv,
+                       int64_t T_cap, int64_t T_max, float sm_scale, void *out, int out_dtype,
+                       void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream,
+                       const int32_t *page_table, int64_t max_pages, int64_t num_pages) {
   try {
     if (!t || !q || !d_kcache || !d_vcache || !d_seq_lens || !out || !d_workspace) return DQ_ERR_NULL;
     if ((q_dtype != DQ_F32 && q_dtype != DQ_BF16) || (out_dtype != DQ_F32 && out_dtype != DQ_BF16))
@@ -427,11 +453,35 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const ui
     a.two_k = has_small_freq(t->k);
     a.two_v = has_small_freq(t->v);
     a.stats = d_stats;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.num_pages = num_pages;
     int e = dqi::launch_decode_attention(a, stream);
     return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
   } catch (...) {
     return DQ_ERR_CUDA;
   }
+}
+
+int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
+                        const uint8_t *d_vcache, const int32_t *d_seq_lens, int B, int Hq, int Hkv,
+                        int64_t T_cap, int64_t T_max, float sm_scale, void *out, int out_dtype,
+                        void *d_workspace, size_t ws_bytes, dq_stats *d_stats, void *stream) {
+  return decode_core(t, q, q_dtype, d_kcache, d_vcache, d_seq_lens, B, Hq, Hkv, T_cap, T_max, sm_scale, out,
+                     out_dtype, d_workspace, ws_bytes, d_stats, stream, nullptr, 0, 0);
+}
+
+int dq_decode_attention_paged(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kpool,
+                              const uint8_t *d_vpool, int64_t num_pages, const int32_t *d_page_table,
+                              int64_t max_pages, const int32_t *d_seq_lens, int B, int Hq, int Hkv,
+                              int64_t T_max, float sm_scale, void *out, int out_dtype, void *d_workspace,
+                              size_t ws_bytes, dq_stats *d_stats, void *stream) {
+  if (!d_page_table) return DQ_ERR_NULL;
+  if (num_pages < 1 || max_pages < 1 || max_pages > (int64_t(1) << 40) || num_pages > (int64_t(1) << 31))
+    return DQ_ERR_SHAPE;
+  if (!aligned(d_page_table, 4)) return DQ_ERR_ALIGN;
+  return decode_core(t, q, q_dtype, d_kpool, d_vpool, d_seq_lens, B, Hq, Hkv, 32 * max_pages, T_max, sm_scale,
+                     out, out_dtype, d_workspace, ws_bytes, d_stats, stream, d_page_table, max_pages, num_pages);
 }
 
 int dq_decode_symbols(const dq_tables *t, const uint8_t *d_cache, int stream_kind,

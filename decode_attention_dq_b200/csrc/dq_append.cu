@@ -295,16 +295,29 @@ struct StreamCtx {
   __device__ int head_of(const AppendArgs &a, int64_t v) const {
     return static_cast<int>((v % per_seq) / a.n_new);
   }
-  // Byte 0 of vector v's container (block pos / 32 of row (b, h), lane
-  // pos % 32), or null when the position is outside the cache.
-  __device__ uint8_t *dst_of(const AppendArgs &a, int64_t v, bool *dropped) const {
+  // Byte 0 of vector v's container (lane pos % 32 of the 32-token block
+  // holding position pos), or null when the position is outside the cache
+  // (dropped) or its page-table entry is out of range (also *bad_page).
+  __device__ uint8_t *dst_of(const AppendArgs &a, int64_t v, bool *dropped, bool *bad_page = nullptr) const {
     const int b = static_cast<int>(v / per_seq);
     const int h = head_of(a, v);
     const int j = static_cast<int>(v % a.n_new);
     const int64_t pos = static_cast<int64_t>(a.start_pos[b]) + j;
     *dropped = pos < 0 || pos >= a.T_cap;
     if (*dropped) return nullptr;
-    return cache + ((static_cast<int64_t>(b) * a.Hkv + h) * a.T_cap + (pos & ~int64_t(31))) * C + (pos & 31);
+    int64_t block;
+    if (a.page_table) {
+      const int32_t pg = a.page_table[static_cast<int64_t>(b) * a.max_pages + (pos >> 5)];
+      if (pg < 0 || pg >= a.num_pages) {
+        *dropped = true;
+        if (bad_page) *bad_page = true;
+        return nullptr;
+      }
+      block = static_cast<int64_t>(pg) * a.Hkv + h;
+    } else {
+      block = (static_cast<int64_t>(b) * a.Hkv + h) * (a.T_cap >> 5) + (pos >> 5);
+    }
+    return cache + block * 32 * C + (pos & 31);
   }
 };
 
@@ -448,8 +461,9 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
 }
 
 __device__ __forceinline__ void add_stats(const AppendArgs &a, bool is_v, const DriftCount &dc, unsigned nf,
-                                          unsigned drops) {
+                                          unsigned drops, unsigned bad_pages = 0) {
   if (!a.stats) return;
+  if (bad_pages) atomicAdd(&a.stats->bad_pages, (unsigned long long)bad_pages);
   if (dc.moves) atomicAdd(is_v ? &a.stats->v_syms_drifted : &a.stats->k_syms_drifted, (unsigned long long)dc.moves);
   if (dc.containers)
     atomicAdd(is_v ? &a.stats->v_cont_drifted : &a.stats->k_cont_drifted, (unsigned long long)dc.containers);
@@ -472,7 +486,7 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
   // ---- phases 1 and 2: lane per vector ----
   uint8_t *stk = W.stack + lane;
   uint16_t n16 = 0;
-  bool nf = false, dropped = false, too_long = false;
+  bool nf = false, dropped = false, too_long = false, bad_page = false;
   if (valid) {
     const int h = c.head_of(a, v);
     uint32_t sw[4];
@@ -484,12 +498,13 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
     const int len = encode_bf<kTwo, true>([&](int i) { return __byte_perm(pk[i >> 2], 0u, 0x4440u + (i & 3)); },
                                           T.es, stk, &x);
     too_long = len > c.P;
-    uint8_t *dst = c.dst_of(a, v, &dropped);
+    uint8_t *dst = c.dst_of(a, v, &dropped, &bad_page);
     if (!too_long && dst) store_container(dst, c.C, n16, x, stk, len);
   }
   unsigned drift_mask = __ballot_sync(kFull, too_long);
   const unsigned nf_mask = __ballot_sync(kFull, valid && nf);
   const unsigned drops = __ballot_sync(kFull, dropped);
+  const unsigned bads = __ballot_sync(kFull, bad_page);
   DriftCount dc;
 
   if (a.drift_list) {
@@ -515,7 +530,7 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
     // Most containers need a few moves: rank 8 first (throughput).
     drift_one<kTwo>(a, c, T, W, vd, n16v, u, lane, 8, dc);
   }
-  if (lane == 0) add_stats(a, is_v, dc, __popc(nf_mask), __popc(drops));
+  if (lane == 0) add_stats(a, is_v, dc, __popc(nf_mask), __popc(drops), __popc(bads));
 }
 
 // Warp-per-vector body for small appends (a decode step): many warps with
@@ -535,8 +550,8 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   uint8_t *stk = W.stack + lane;
   uint32_t x = 0;
   const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(W.q[i]); }, T.es, stk, &x);
-  bool dropped = false;
-  uint8_t *dst = c.dst_of(a, v, &dropped);
+  bool dropped = false, bad_page = false;
+  uint8_t *dst = c.dst_of(a, v, &dropped, &bad_page);
   DriftCount dc;
   if (len <= c.P) {
     if (lane == 0 && dst) store_container(dst, c.C, n16, x, stk, len);
@@ -545,7 +560,7 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
     // One pass of 32 in most cases (latency of a small append).
     drift_one<kTwo>(a, c, T, W, v, n16, u, lane, 32, dc);
   }
-  if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u);
+  if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u, bad_page ? 1u : 0u);
 }
 
 // E6 for the containers listed by the lane-per-vector kernel: each warp of

@@ -94,11 +94,10 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
-// Copies the 32-token block starting at token t0 (a multiple of 32) of one
-// cache row into shared memory, 16 bytes per copy (32 C is a multiple of 16).
-__device__ __forceinline__ void stage_group(uint8_t *dst, const uint8_t *row, int64_t t0, int C, int lane) {
+// Copies one 32-token block (32 C bytes, a multiple of 16) of a cache into
+// shared memory, 16 bytes per copy.
+__device__ __forceinline__ void stage_block(uint8_t *dst, const uint8_t *src, int C, int lane) {
   const int chunks = (kTile * C) >> 4;
-  const uint8_t *src = row + t0 * C;
   for (int c = lane; c < chunks; c += 32) cp_async16(dst + c * 16, src + c * 16);
 }
 
@@ -363,6 +362,7 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
   const int64_t g_end = warp_first(wid + 1, W, N);
   if (g >= g_end) return;
   unsigned bad_count = 0;
+  unsigned bad_pages = 0;
 
   // Sequence holding flat group g: the largest b with prefix[b] * Hkv <= g
   // (it has tokens, since g < prefix[b + 1] * Hkv).
@@ -403,10 +403,26 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
       }
     }
 
-    const uint8_t *krow = a.kcache + bh * a.T_cap * ck;
-    const uint8_t *vrow = a.vcache + bh * a.T_cap * cv;
     const int64_t tseg = j0 * kTile;
     auto group_t0 = [&](int64_t j) { return tseg + j * kTile; };
+    // Cache block (32 tokens of one KV head) holding group j of the segment:
+    // block b of a cache sits at byte 32 C b. Contiguous caches: row bh,
+    // token block t / 32. Paged caches: page_table[b][t / 32] * Hkv + h; an
+    // entry out of range is counted and read as page 0 (garbage, no fault).
+    auto block_of = [&](int64_t j) -> int64_t {
+      const int64_t tb = (tseg >> 5) + j;
+      if (a.page_table) {
+        int64_t pg = a.page_table[static_cast<int64_t>(b) * a.max_pages + tb];
+        if (pg < 0 || pg >= a.num_pages) {
+          ++bad_pages;
+          pg = 0;
+        }
+        return pg * Hkv + h;
+      }
+      return bh * (a.T_cap / kTile) + tb;
+    };
+    auto kblock = [&](int64_t blk) { return a.kcache + blk * kTile * ck; };
+    auto vblock = [&](int64_t blk) { return a.vcache + blk * kTile * cv; };
 
     WarpAcc<G> acc;
 #pragma unroll
@@ -422,14 +438,18 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
     // Prologue: K(0), V(0) into slot 0 and K(1) into K slot 1. Invariant at
     // the top of iteration j: V(j) sits in V slot j%2 and K(j+1) in K slot
     // (j+1)%2, both complete; iteration j prefetches K(j+2) and V(j+1).
+    // Block ids run one iteration ahead of their use: bj1 = block of group
+    // j+1, bj2 = block of group j+2 at the top of iteration j.
+    int64_t bj1 = 0, bj2 = 0;
     {
-      const int64_t t0 = group_t0(0);
-      stage_group(kst, krow, t0, ck, lane);
-      stage_group(vst, vrow, t0, cv, lane);
+      const int64_t b0 = block_of(0);
+      stage_block(kst, kblock(b0), ck, lane);
+      stage_block(vst, vblock(b0), cv, lane);
       if (n > 1) {
-        const int64_t t1 = group_t0(1);
-        stage_group(kst + kTile * ck, krow, t1, ck, lane);
+        bj1 = block_of(1);
+        stage_block(kst + kTile * ck, kblock(bj1), ck, lane);
       }
+      if (n > 2) bj2 = block_of(2);
       cp_async_commit();
       cp_async_wait_0();
       __syncwarp();  // staged bytes and q~ visible to the whole warp
@@ -483,15 +503,11 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
           }
       }
       // Prefetch K(j+2) into slot cur and V(j+1) into slot nxt.
-      if (j + 2 < n) {
-        const int64_t t2 = group_t0(j + 2);
-        stage_group(kst + cur * kTile * ck, krow, t2, ck, lane);
-      }
-      if (has_next) {
-        const int64_t t1 = group_t0(j + 1);
-        stage_group(vst + nxt * kTile * cv, vrow, t1, cv, lane);
-      }
+      if (j + 2 < n) stage_block(kst + cur * kTile * ck, kblock(bj2), ck, lane);
+      if (has_next) stage_block(vst + nxt * kTile * cv, vblock(bj1), cv, lane);
       cp_async_commit();
+      bj1 = bj2;
+      if (j + 3 < n) bj2 = block_of(j + 3);
 
       const uint8_t *kb = kst + nxt * kTile * ck + lane;
       const uint8_t *vb = vst + cur * kTile * cv + lane;
@@ -580,6 +596,7 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
     }
   }
   if (a.stats && lane == 0 && bad_count) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(bad_count));
+  if (a.stats && lane == 0 && bad_pages) atomicAdd(&a.stats->bad_pages, static_cast<unsigned long long>(bad_pages));
 }
 
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a) {

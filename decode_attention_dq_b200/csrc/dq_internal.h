@@ -83,6 +83,11 @@ struct AppendArgs {
   uint32_t *drift_list;
   uint32_t *drift_count;
   int64_t list_cap;
+  // Paged caches (nullptr: contiguous caches of T_cap tokens per row): token
+  // t of sequence b is in page page_table[b * max_pages + t / 32] of a pool
+  // laid out [num_pages][Hkv][C][32]; T_cap = 32 max_pages.
+  const int32_t *page_table;
+  int64_t max_pages, num_pages;
 };
 // Bytes of the optional append workspace for nvec vectors per stream.
 size_t append_workspace_bytes(int64_t nvec);
@@ -108,6 +113,9 @@ struct DecodeArgs {
   int ck, cv;
   bool two_k, two_v;  // the stream's table has a symbol with f < 16
   dq_stats *stats;
+  // Paged caches, as in AppendArgs (nullptr: contiguous).
+  const int32_t *page_table;
+  int64_t max_pages, num_pages;
 };
 int launch_decode_attention(const DecodeArgs &a, void *stream);
 // Warps per CTA of the split kernel for these shapes (0 if unsupported).

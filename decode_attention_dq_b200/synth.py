@@ -140,15 +140,23 @@ def scaled(w: Workload, **changes) -> Workload:
 
 
 def prefill_cache(tab, w: Workload, kcache, vcache, n_tokens: int, seqs_per_call: int = 8,
-                  threads: int = 16, stats=None, timings: list | None = None):
+                  threads: int = 16, stats=None, timings: list | None = None, page_table=None):
     """Fill positions [0, n_tokens) of every sequence's cache with the
     workload's seeded K/V, appended through dq_append_kv in batches of
     sequences (the inputs are drawn on the host, then copied to the device).
     With `timings`, each dq_append_kv call is bracketed by CUDA events on the
     current stream and (start event, end event, vectors per stream) is
     appended to the list; the first call is then made twice and only its
-    second run is timed (the first also loads the kernels)."""
-    from ._native import dq_append_kv  # local import: synth itself needs no GPU
+    second run is timed (the first also loads the kernels). With `page_table`
+    (int32 [B, max_pages]) kcache and vcache are page pools and the tokens go
+    through dq_append_kv_paged."""
+    from ._native import dq_append_kv, dq_append_kv_paged  # local import: synth itself needs no GPU
+
+    def append(kt, vt, start, b0, b1, st):
+        if page_table is None:
+            dq_append_kv(tab, kt, vt, start, kcache[b0:b1], vcache[b0:b1], stats=st)
+        else:
+            dq_append_kv_paged(tab, kt, vt, start, kcache, vcache, page_table[b0:b1], stats=st)
 
     for b0 in range(0, w.B, seqs_per_call):
         b1 = min(w.B, b0 + seqs_per_call)
@@ -162,10 +170,10 @@ def prefill_cache(tab, w: Workload, kcache, vcache, n_tokens: int, seqs_per_call
         start = torch.zeros(b1 - b0, dtype=torch.int32, device=kcache.device)
         if timings is not None:
             if b0 == 0:  # untimed first run (same inputs, same containers)
-                dq_append_kv(tab, kt, vt, start, kcache[b0:b1], vcache[b0:b1])
+                append(kt, vt, start, b0, b1, None)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-        dq_append_kv(tab, kt, vt, start, kcache[b0:b1], vcache[b0:b1], stats=stats)
+        append(kt, vt, start, b0, b1, stats)
         if timings is not None:
             e1.record()
             timings.append((e0, e1, (b1 - b0) * w.Hkv * n_tokens))

@@ -101,6 +101,7 @@ typedef struct {
   unsigned long long nonfinite_inputs;   /* input vectors treated as zero    */
   unsigned long long dropped_writes;     /* append positions >= T_cap        */
   unsigned long long clamped_lengths;    /* seq_len > T_max or > T_cap       */
+  unsigned long long bad_pages;          /* page-table entries out of range  */
 } dq_stats;
 
 typedef struct dq_tables dq_tables; /* opaque, library-owned */
@@ -229,6 +230,41 @@ int dq_decode_attention(const dq_tables *t, const void *q, int q_dtype,
                         int64_t T_cap, int64_t T_max, float sm_scale,
                         void *out, int out_dtype, void *d_workspace,
                         size_t ws_bytes, dq_stats *d_stats, void *stream);
+
+/* Paged caches. The pages' serving results ([news] "The Numbers": batch 128
+ * at an 8K prompt on one GPU) come from a serving engine, and such engines
+ * hand out KV memory in fixed-size pages through a per-sequence page table;
+ * the D-Quant pages describe no page table themselves. A page here is one
+ * 32-token block of every KV head: a pool of num_pages pages is laid out
+ * [num_pages][Hkv][C][32] (the 32 containers of a block byte-interleaved as
+ * in the contiguous cache), and token t of sequence b lives in page
+ * d_page_table[b * max_pages + t / 32], at lane t % 32 of its blocks.
+ *   d_kpool, d_vpool  device pools of C_k- and C_v-byte containers, 16-byte
+ *                     aligned (DQ_ERR_ALIGN)
+ *   num_pages         pages in each pool, 1 .. 2^31
+ *   d_page_table      device int32 [B][max_pages], 4-byte aligned; entries
+ *                     outside [0, num_pages) are never dereferenced: they
+ *                     are counted in bad_pages (an append drops the token,
+ *                     the decoder reads page 0 instead)
+ *   max_pages         pages per sequence; a sequence holds up to
+ *                     32 * max_pages tokens (the T_cap of the contiguous calls)
+ * Everything else is as in dq_append_kv_ws and dq_decode_attention (the
+ * decode workspace is dq_decode_workspace_bytes, the append workspace is
+ * optional); containers and outputs are the same as with a contiguous cache
+ * holding the same tokens. */
+int dq_append_kv_paged(const dq_tables *t, const void *k, const void *v, int dtype,
+                       int B, int Hkv, int n_new, const int32_t *d_start_pos,
+                       uint8_t *d_kpool, uint8_t *d_vpool, int64_t num_pages,
+                       const int32_t *d_page_table, int64_t max_pages,
+                       void *d_workspace, size_t ws_bytes, dq_stats *d_stats,
+                       void *stream);
+int dq_decode_attention_paged(const dq_tables *t, const void *q, int q_dtype,
+                              const uint8_t *d_kpool, const uint8_t *d_vpool,
+                              int64_t num_pages, const int32_t *d_page_table,
+                              int64_t max_pages, const int32_t *d_seq_lens,
+                              int B, int Hq, int Hkv, int64_t T_max, float sm_scale,
+                              void *out, int out_dtype, void *d_workspace,
+                              size_t ws_bytes, dq_stats *d_stats, void *stream);
 
 /* Decode attention without a caller-provided workspace. The D-Quant pages
  * have no counterpart to this call: it exists for callers that cannot
