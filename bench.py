@@ -49,13 +49,13 @@ ENCODE_OPS_PER_VECTOR = 2560
 LAUNCHES_PER_STEP = 4
 # DRAM traffic of decode_split_kernel from one ncu capture (dram__bytes_read
 # + dram__bytes_write) of the 32-sequence, 8192-token workload with 36-byte
-# containers: 151.37 MB + 3.74 MB per launch over 32*8*8192 token-heads. It
+# containers: 151.44 MB + 6.80 MB per launch over 32*8*8192 token-heads. It
 # scales with the token-heads a launch processes (reads are the containers,
 # writes the partial states). It belongs to one version of the kernel source:
 # for any other, or other container sizes, traffic is reported as null.
 DECODE_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_decode.cu",
-                  "sha256_16": "2badf4fff5fba524", "ck": 36, "cv": 36,
-                  "bytes_per_token_head": (151.367168e6 + 3.742464e6) / (32 * 8 * 8192)}
+                  "sha256_16": "6d0be282ac859e1f", "ck": 36, "cv": 36,
+                  "bytes_per_token_head": (151.442944e6 + 6.804992e6) / (32 * 8 * 8192)}
 
 
 def decode_traffic(token_heads, ck, cv):
