@@ -31,7 +31,9 @@
 //     first, ties to the lower index), and lane m encodes the string with the
 //     first m+1 moves applied; the smallest m that fits is the greedy result.
 //     The first pass tries 8 move counts (32 in the warp-per-vector
-//     kernel), later ones 32.
+//     kernel), later ones 32. The separate drift kernel ranks 8 moves for
+//     each of 4 containers and tries all 32 (container, count) pairs in one
+//     encode pass.
 #include "dq_device.cuh"
 
 namespace dqi {
@@ -362,22 +364,24 @@ struct DriftCount {
   unsigned moves = 0, containers = 0, fallbacks = 0;
 };
 
-// E6 for one over-long container, by the whole warp. On entry W.q holds the
-// symbols and u[k] this lane's coordinates lane + 32 k.
+// E6 for one over-long container, by the whole warp. On entry q[] holds the
+// symbols and u[k] this lane's coordinates lane + 32 k; rank[] and tgt[] are
+// scratch, stack the warp's push stacks.
 template <bool kTwo>
-__device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T, WarpArea &W,
-                                          int64_t vd, uint16_t n16v, const float (&u)[4], int lane, int first_batch,
+__device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
+                                          uint8_t *stack, const uint8_t *q, uint8_t *rank, uint8_t *tgt, int64_t vd,
+                                          uint16_t n16v, const float (&u)[4], int lane, int first_batch,
                                           DriftCount &dc) {
-  uint8_t *stk = W.stack + lane;
+  uint8_t *stk = stack + lane;
   // Best move and key of the 4 symbols this lane owns (i = lane + 32 k).
   float key[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int i = lane + 32 * k;
     int tj;
-    key[k] = best_move(T, c.nl, W.q[i], u[k], &tj);
-    W.rank[i] = kNoRank;
-    W.tgt[i] = static_cast<uint8_t>(tj);
+    key[k] = best_move(T, c.nl, q[i], u[k], &tj);
+    rank[i] = kNoRank;
+    tgt[i] = static_cast<uint8_t>(tj);
   }
   __syncwarp();
   int ranked = 0;    // moves ranked so far
@@ -405,7 +409,7 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           if (bi == lane + 32 * k) key[k] = INFINITY;
-        W.rank[bi] = static_cast<uint8_t>(ranked + added);
+        rank[bi] = static_cast<uint8_t>(ranked + added);
       }
     }
     __syncwarp();
@@ -415,9 +419,9 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
     uint32_t x = 0;
     const int len = encode_bf<kTwo, false>(
         [&](int i) {
-          const uint32_t r = W.rank[i];
-          return (r != kNoRank && static_cast<int>(r) <= m_moves) ? static_cast<uint32_t>(W.tgt[i])
-                                                                  : static_cast<uint32_t>(W.q[i]);
+          const uint32_t r = rank[i];
+          return (r != kNoRank && static_cast<int>(r) <= m_moves) ? static_cast<uint32_t>(tgt[i])
+                                                                  : static_cast<uint32_t>(q[i]);
         },
         T.es, stk, &x);
     const unsigned fit = __ballot_sync(kFull, lane < added && len <= c.P);
@@ -442,8 +446,8 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
     uint32_t x = 0;
     const int len = encode_bf<kTwo, false>(
         [&](int i) {
-          const uint32_t r = W.rank[i];
-          const uint32_t s = (r != kNoRank) ? W.tgt[i] : W.q[i];
+          const uint32_t r = rank[i];
+          const uint32_t s = (r != kNoRank) ? tgt[i] : q[i];
           return static_cast<uint32_t>(s >= static_cast<uint32_t>(hlf) ? hlf : hlf - 1);
         },
         T.es, stk, &x);
@@ -528,7 +532,7 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
     warp_prepare(a, c.src, vd, c.head_of(a, vd), c.t, lane, u, W.q, &n16v, &nfv);
     __syncwarp();
     // Most containers need a few moves: rank 8 first (throughput).
-    drift_one<kTwo>(a, c, T, W, vd, n16v, u, lane, 8, dc);
+    drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, vd, n16v, u, lane, 8, dc);
   }
   if (lane == 0) add_stats(a, is_v, dc, __popc(nf_mask), __popc(drops), __popc(bads));
 }
@@ -558,30 +562,143 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   } else {
     __syncwarp();
     // One pass of 32 in most cases (latency of a small append).
-    drift_one<kTwo>(a, c, T, W, v, n16, u, lane, 32, dc);
+    drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 32, dc);
   }
   if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u, bad_page ? 1u : 0u);
 }
 
+// Drift kernel scratch: kBatch containers per warp are prepared and ranked,
+// then their first kFirst candidate move counts are tried in one encode
+// pass (lane 8 c + k tries container c with moves 0..k).
+constexpr int kBatch = 4;
+constexpr int kFirst = 8;
+static_assert(kBatch * kFirst == 32, "one trial per lane");
+
+struct DriftArea {
+  uint8_t stack[kStackSlots * 32];
+  uint8_t q[kBatch][kD], rank[kBatch][kD], tgt[kBatch][kD];
+  int64_t vd[kBatch];
+  int32_t added[kBatch];
+  uint16_t n16[kBatch];
+};
+
+// Ranks up to kFirst best moves of one container (u: this lane's coordinates,
+// q: symbols) into rank[] / tgt[] (repeated warp arg-min over (key, index),
+// as in drift_one). Returns how many were ranked.
+__device__ __forceinline__ int rank_first(const AppendTables &T, int nl, const float (&u)[4], const uint8_t *q,
+                                          uint8_t *rank, uint8_t *tgt, int lane) {
+  float key[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = lane + 32 * k;
+    int tj;
+    key[k] = best_move(T, nl, q[i], u[k], &tj);
+    rank[i] = kNoRank;
+    tgt[i] = static_cast<uint8_t>(tj);
+  }
+  __syncwarp();
+  int added = 0;
+  for (; added < kFirst; ++added) {
+    float bk = key[0];
+    int bi = lane;
+#pragma unroll
+    for (int k = 1; k < 4; ++k)
+      if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ok = __shfl_xor_sync(kFull, bk, off);
+      const int oi = __shfl_xor_sync(kFull, bi, off);
+      if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
+    }
+    if (bk == INFINITY) break;  // no candidate left
+    if ((bi & 31) == lane) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (bi == lane + 32 * k) key[k] = INFINITY;
+      rank[bi] = static_cast<uint8_t>(added);
+    }
+  }
+  __syncwarp();
+  return added;
+}
+
 // E6 for the containers listed by the lane-per-vector kernel: each warp of
-// a persistent grid takes list entries gridDim.x * kAW apart.
+// a persistent grid takes kBatch list entries at a time. A container whose
+// first kFirst moves are not enough goes through drift_one.
 template <bool kTwo>
-__device__ __forceinline__ void drift_body(const AppendArgs &a, AppendTables &T, WarpArea &W, bool is_v) {
+__device__ __forceinline__ void drift_body(const AppendArgs &a, AppendTables &T, DriftArea &A, bool is_v) {
   const int lane = threadIdx.x & 31;
   const StreamCtx c = stream_setup(a, T, is_v);
   __syncthreads();
   const uint32_t n = a.drift_count[is_v ? 1 : 0];
   const uint32_t *list = a.drift_list + (is_v ? a.list_cap : 0);
-  const uint32_t stride = gridDim.x * kAW;
+  const uint32_t stride = gridDim.x * kAW * kBatch;
+  uint8_t *stk = A.stack + lane;
   DriftCount dc;
-  for (uint32_t i = blockIdx.x * kAW + (threadIdx.x >> 5); i < n; i += stride) {
-    const int64_t vd = list[i];
-    float u[4];
-    uint16_t n16;
-    bool nf;
-    warp_prepare(a, c.src, vd, c.head_of(a, vd), c.t, lane, u, W.q, &n16, &nf);
+  for (uint32_t base = (blockIdx.x * kAW + (threadIdx.x >> 5)) * kBatch; base < n; base += stride) {
+    const int nb = (n - base) < static_cast<uint32_t>(kBatch) ? static_cast<int>(n - base) : kBatch;
+    // Loops over the batch stay rolled: the kernel's code has to fit the
+    // instruction caches shared by its warps.
+#pragma unroll 1
+    for (int cb = 0; cb < nb; ++cb) {
+      const int64_t v = list[base + cb];
+      float u[4];
+      uint16_t n16v;
+      bool nf;
+      warp_prepare(a, c.src, v, c.head_of(a, v), c.t, lane, u, A.q[cb], &n16v, &nf);
+      __syncwarp();
+      const int ad = rank_first(T, c.nl, u, A.q[cb], A.rank[cb], A.tgt[cb], lane);
+      if (lane == 0) {
+        A.vd[cb] = v;
+        A.n16[cb] = n16v;
+        A.added[cb] = ad;
+      }
+    }
     __syncwarp();
-    drift_one<kTwo>(a, c, T, W, vd, n16, u, lane, 8, dc);
+    // Lane 8 cb + k encodes container cb with its moves 0..k applied.
+    const int cm = (lane / kFirst) < nb ? lane / kFirst : 0, km = lane % kFirst;
+    const uint8_t *q = A.q[cm], *rk = A.rank[cm], *tg = A.tgt[cm];
+    uint32_t x = 0;
+    const int len = encode_bf<kTwo, false>(
+        [&](int i) {
+          const uint32_t r = rk[i];
+          return (r != kNoRank && static_cast<int>(r) <= km) ? static_cast<uint32_t>(tg[i]) : static_cast<uint32_t>(q[i]);
+        },
+        T.es, stk, &x);
+    const unsigned fit =
+        __ballot_sync(kFull, lane / kFirst < nb && km < A.added[cm] && len <= c.P);
+    // The first fitting lane of each container stores it.
+    {
+      const int cb = lane / kFirst;
+      const unsigned fc = (fit >> (kFirst * cb)) & ((1u << kFirst) - 1u);
+      if (cb < nb && fc && km == __ffs(fc) - 1) {
+        bool dr = false;
+        uint8_t *dst = c.dst_of(a, A.vd[cb], &dr);
+        if (dst) store_container(dst, c.C, A.n16[cb], x, stk, len);
+      }
+    }
+#pragma unroll 1
+    for (int cb = 0; cb < nb; ++cb) {
+      const unsigned fc = (fit >> (kFirst * cb)) & ((1u << kFirst) - 1u);
+      if (fc) {
+        dc.moves += static_cast<unsigned>(__ffs(fc));
+        dc.containers += 1;
+      }
+    }
+    __syncwarp();
+    // Containers that need more moves (or run out of candidates): the full
+    // greedy search, which ranks its moves again from the first.
+#pragma unroll 1
+    for (int cb = 0; cb < nb; ++cb) {
+      if ((fit >> (kFirst * cb)) & ((1u << kFirst) - 1u)) continue;
+      const int64_t v = A.vd[cb];
+      float u[4];
+      uint16_t n16v;
+      bool nf;
+      warp_prepare(a, c.src, v, c.head_of(a, v), c.t, lane, u, A.q[0], &n16v, &nf);
+      __syncwarp();
+      drift_one<kTwo>(a, c, T, A.stack, A.q[0], A.rank[0], A.tgt[0], v, n16v, u, lane, 32, dc);
+    }
   }
   if (lane == 0) add_stats(a, is_v, dc, 0u, 0u);
 }
@@ -589,9 +706,9 @@ __device__ __forceinline__ void drift_body(const AppendArgs &a, AppendTables &T,
 template <bool kTwoK, bool kTwoV>
 __global__ void __launch_bounds__(kAW * 32) append_drift_kernel(const AppendArgs a) {
   __shared__ AppendTables T;
-  __shared__ WarpArea W[kAW];
+  __shared__ DriftArea A[kAW];
   const bool is_v = blockIdx.y == 1;
-  WarpArea &w = W[threadIdx.x >> 5];
+  DriftArea &w = A[threadIdx.x >> 5];
   if constexpr (kTwoK == kTwoV) {
     drift_body<kTwoK>(a, T, w, is_v);
   } else {
