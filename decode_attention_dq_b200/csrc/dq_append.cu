@@ -60,10 +60,12 @@ struct AppendTables {
   uint32_t freq[kMaxLevels], cum[kMaxLevels];
 };
 
-// Per-warp shared memory: push stacks (byte j of lane l at [j][l]) and the
-// symbols, move ranks and targets of the container being drifted.
+// Per-warp shared memory: push stacks (byte j of lane l at [j][l]), the
+// lanes' packed symbols (word w of lane l at [w][l]) and the symbols, move
+// ranks and targets of the container being drifted.
 struct WarpArea {
   uint8_t stack[kStackSlots * 32];
+  uint32_t syms[kD / 4][32];
   uint8_t q[kD], rank[kD], tgt[kD];
 };
 
@@ -496,11 +498,18 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
     uint32_t sw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
-    uint32_t pk[32];
-    lane_prepare<kBF16>(c.src, v, sw, c.t, pk, &n16, &nf);
+    {
+      uint32_t pk[32];
+      lane_prepare<kBF16>(c.src, v, sw, c.t, pk, &n16, &nf);
+#pragma unroll
+      for (int w2 = 0; w2 < kD / 4; ++w2) W.syms[w2][lane] = pk[w2];
+    }
+    // The encode loop reads the symbols back from shared memory so that it
+    // can stay rolled (a fully unrolled loop adds ~40 KB of code).
+    const uint8_t *sy = reinterpret_cast<const uint8_t *>(&W.syms[0][lane]);
     uint32_t x = 0;
-    const int len = encode_bf<kTwo, true>([&](int i) { return __byte_perm(pk[i >> 2], 0u, 0x4440u + (i & 3)); },
-                                          T.es, stk, &x);
+    const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(sy[(i >> 2) * 128 + (i & 3)]); },
+                                           T.es, stk, &x);
     too_long = len > c.P;
     uint8_t *dst = c.dst_of(a, v, &dropped, &bad_page);
     if (!too_long && dst) store_container(dst, c.C, n16, x, stk, len);
