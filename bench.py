@@ -12,8 +12,10 @@ per step); the HBM rate of the compressed bytes and the dominant kernel's
 roofline fraction are reported beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dq|reference]
-                  [--workload NAME] [--paged]
---paged keeps the caches in page pools behind a shuffled page table.
+                  [--workload NAME] [--paged] [--layers L] [--graph]
+--paged keeps the caches in page pools behind a shuffled page table; --layers
+runs an L-layer attention-only decode loop (one cache per layer); --graph also
+times the step captured once as a CUDA graph and replayed.
 Under torchrun every rank runs an independent replica (no data-path
 collective): value = all ranks' KV tokens / the slowest rank's time.
 """
@@ -248,29 +250,37 @@ def run_dq(args):
 
     app_ws = torch.empty(max(16, dq.dq_append_workspace_bytes(tab, w.B, w.Hkv, 1)), dtype=torch.uint8,
                          device=dev)
+    # Serving loop of L layers: one cache per layer (the same prefilled
+    # contents), each step appends to and attends over every layer in turn.
+    L = max(1, args.layers)
+    caches = [(kc, vc)] + [(kc.clone(), vc.clone()) for _ in range(L - 1)]
 
-    def append(i):
+    def append(i, layer, st):
+        kl, vl = caches[layer]
         if page_table is None:
-            dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kc, vc, stats=stats, stream=stream, workspace=app_ws)
+            dq.dq_append_kv(tab, dev_k[i], dev_v[i], start, kl, vl, stats=stats, stream=st, workspace=app_ws)
         else:
-            dq.dq_append_kv_paged(tab, dev_k[i], dev_v[i], start, kc, vc, page_table, stats=stats,
-                                  stream=stream, workspace=app_ws)
+            dq.dq_append_kv_paged(tab, dev_k[i], dev_v[i], start, kl, vl, page_table, stats=stats,
+                                  stream=st, workspace=app_ws)
 
-    def decode(i):
+    def decode(i, layer, st):
+        kl, vl = caches[layer]
         if page_table is None:
-            dq.dq_decode_attention(tab, dev_q[i], kc, vc, seq, T, out, wsp, stats=stats, stream=stream)
+            dq.dq_decode_attention(tab, dev_q[i], kl, vl, seq, T, out, wsp, stats=stats, stream=st)
         else:
-            dq.dq_decode_attention_paged(tab, dev_q[i], kc, vc, page_table, seq, T, out, wsp, stats=stats,
-                                         stream=stream)
+            dq.dq_decode_attention_paged(tab, dev_q[i], kl, vl, page_table, seq, T, out, wsp, stats=stats,
+                                         stream=st)
 
-    def step(s, e_dec0=None, e_dec1=None):
+    def step(s, ev=None, st=None):
+        st = stream if st is None else st
         i = s % nsteps_inputs
-        append(i)
-        if e_dec0 is not None:
-            e_dec0.record(stream)
-        decode(i)
-        if e_dec1 is not None:
-            e_dec1.record(stream)
+        for layer in range(L):
+            append(i, layer, st)
+            if ev is not None:
+                ev[layer][0].record(st)
+            decode(i, layer, st)
+            if ev is not None:
+                ev[layer][1].record(st)
 
     def barrier():
         if dist is not None:
@@ -281,8 +291,8 @@ def run_dq(args):
     torch.cuda.synchronize()
 
     # ---- timed region: device-resident inputs ----
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+    ev_dec = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(L)] for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -291,16 +301,34 @@ def run_dq(args):
     torch.cuda.synchronize()
     e0.record(stream)
     for s in range(args.steps):
-        step(s, *ev_dec[s])
+        step(s, ev_dec[s])
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     elapsed_ms = e0.elapsed_time(e1)
-    dec_ms = sum(a.elapsed_time(b) for a, b in ev_dec) / args.steps
+    dec_ms = sum(a.elapsed_time(b) for evs in ev_dec for a, b in evs) / (args.steps * L)  # per decode call
+
+    # ---- optional: the same step captured once as a CUDA graph and replayed ----
+    graph_ms = None
+    if args.graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(0, st=torch.cuda.current_stream())
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = max_over_ranks([g0.elapsed_time(g1) / args.steps], dist, dev)[0]
+        del g
     elapsed_ms, dec_ms = max_over_ranks([elapsed_ms, dec_ms], dist, dev)
     ms_per_step = elapsed_ms / args.steps
-    kv_tokens_step = w.B * T
+    kv_tokens_step = w.B * T * L
     value = whole_job_rate(kv_tokens_step, ws, ms_per_step)
 
     # ---- e2e: host buffers, copies inside the timed region ----
@@ -309,8 +337,9 @@ def run_dq(args):
         dev_k[i].copy_(host_k[i], non_blocking=True)
         dev_v[i].copy_(host_v[i], non_blocking=True)
         dev_q[i].copy_(host_q[i], non_blocking=True)
-        append(i)
-        decode(i)
+        for layer in range(L):
+            append(i, layer, stream)
+            decode(i, layer, stream)
         out_host.copy_(out, non_blocking=True)
 
     for s in range(2):
@@ -352,6 +381,7 @@ def run_dq(args):
                        "k_container_bytes": ck, "v_container_bytes": cv,
                        "l2": "inputs larger than L2 (%.0f MB of containers read per step)" % (comp_bytes / 1e6),
                        "cache": "paged: 32-token pages in a shuffled order" if args.paged else "contiguous",
+                       "layers": L,
                        "parallelism": "replicas x%d" % ws},
             "hbm_gbs": hbm_gbs,
             "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tlaneop/s",
@@ -365,7 +395,7 @@ def run_dq(args):
                          "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": peaks.get("hbm_gbs"),
                                  "frac": hbm_gbs / float(peaks.get("hbm_gbs", 6650.0))}},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * L * args.steps,
             "clocks": clk,
             "drift": {"prefill_k_syms_pct": 100.0 * pstats["k_syms_drifted"] / (token_heads * 128),
                       "prefill_v_syms_pct": 100.0 * pstats["v_syms_drifted"] / (token_heads * 128),
@@ -375,6 +405,11 @@ def run_dq(args):
             "integrity_errors": st["integrity_errors"],
             "prefill_s": prefill_s,
             "encode": encode_report(enc_ms, enc_vectors, w, ck, cv, alu_peak, peaks),
+            "serving": {"what": "attention-only decode loop over %d layer(s): append 1 token + decode "
+                                "attention per layer, %d sequences of %d tokens" % (L, w.B, T),
+                        "tokens_per_s": whole_job_rate(w.B, ws, ms_per_step),
+                        "graph_ms_per_step": graph_ms,
+                        "graph_tokens_per_s": None if graph_ms is None else whole_job_rate(w.B, ws, graph_ms)},
         }
         if ws == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(w, tab_seed=0, seconds=args.cpu_seconds)
@@ -513,6 +548,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--paged", action="store_true", help="page pools and a shuffled page table")
+    ap.add_argument("--layers", type=int, default=1, help="layers of the decode loop (one cache each)")
+    ap.add_argument("--graph", action="store_true", help="also time the step captured as a CUDA graph")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
