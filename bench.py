@@ -464,38 +464,62 @@ def oracle_sample_step(w, tabs, rows, cache_rows):
 
 
 def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512):
-    """The oracle, as it stands, on the host: bounded sample of the step."""
+    """The oracle, as it stands, on the host: a bounded sample of the step,
+    once on one thread (BLAS limited to one thread too) and once on all host
+    cores (a thread per (sequence, KV head) row; the oracle's C calls and
+    numpy's kernels release the GIL)."""
+    from concurrent.futures import ThreadPoolExecutor
+
     import numpy as np
+    from threadpoolctl import threadpool_limits
+
     from decode_attention_dq_b200 import synth
     from oracle import oracle as o
 
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
                     v_container_bytes=o.container_bytes(w.v_bits), sign_seed=tab_seed)
-    # Containers for a few sampled rows, encoded by the oracle (setup, untimed).
-    rng = np.random.default_rng(0)
-    cand = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, max_rows), rng.integers(0, w.Hkv, max_rows))]
-    prepared = []
-    t_setup = time.time()
-    for b, h in cand:
-        K = synth.kv_row(w, "k", b, h)
-        V = synth.kv_row(w, "v", b, h)
-        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
-        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
-        prepared.append(((b, h), (kc, vc)))
-        if time.time() - t_setup > seconds:
-            break
-    done = 0
-    t0 = time.time()
-    for (bh, cc) in prepared:
-        oracle_sample_step(w, tabs, [bh], [cc])
-        done += 1
-        if time.time() - t0 > seconds:
-            break
-    dt = time.time() - t0
-    kv_tokens = done * w.T / w.Hkv  # one KV token = one position across all KV heads
-    return {"value": kv_tokens / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d (sequence, KV head) rows of %s: append 1 token + fp64 decode attention "
-                      "over %d tokens each, single thread, %.1f s" % (done, w.name, w.T, dt)}
+    ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    with threadpool_limits(limits=1):
+        # Containers for sampled rows, encoded by the oracle (setup, untimed).
+        rng = np.random.default_rng(0)
+        cand = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, max_rows), rng.integers(0, w.Hkv, max_rows))]
+
+        def prepare(bh):
+            b, h = bh
+            K = synth.kv_row(w, "k", b, h)
+            V = synth.kv_row(w, "v", b, h)
+            kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
+            vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+            return (bh, (kc, vc))
+
+        prepared = []
+        t_setup = time.time()
+        with ThreadPoolExecutor(ncores) as ex:
+            for i in range(0, len(cand), ncores):
+                prepared.extend(ex.map(prepare, cand[i:i + ncores]))
+                if time.time() - t_setup > seconds:
+                    break
+        # One thread.
+        done = 0
+        t0 = time.time()
+        for (bh, cc) in prepared:
+            oracle_sample_step(w, tabs, [bh], [cc])
+            done += 1
+            if time.time() - t0 > seconds / 2:
+                break
+        dt = time.time() - t0
+        # All cores, over the same rows.
+        rows = prepared[:max(done, min(len(prepared), ncores))]
+        t1 = time.time()
+        with ThreadPoolExecutor(ncores) as ex:
+            list(ex.map(lambda p: oracle_sample_step(w, tabs, [p[0]], [p[1]]), rows))
+        dt_all = time.time() - t1
+    per_row = w.T / w.Hkv  # one KV token = one position across all KV heads
+    return {"value": done * per_row / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d (sequence, KV head) rows of %s: append 1 token + fp64 decode attention over %d "
+                      "tokens each, one thread, %.1f s" % (done, w.name, w.T, dt),
+            "all_cores": {"value": len(rows) * per_row / dt_all, "unit": UNIT, "cores": ncores,
+                          "sample": "%d rows, one thread per row, %.1f s" % (len(rows), dt_all)}}
 
 
 def run_reference(args):
@@ -517,12 +541,14 @@ def run_reference(args):
         kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
         vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
         prepared.append(((b, h), (kc, vc)))
-    for i in range(args.warmup):
-        oracle_sample_step(w, tabs, [prepared[i][0]], [prepared[i][1]])
-    t0 = time.time()
-    for i in range(args.warmup, args.warmup + args.steps):
-        oracle_sample_step(w, tabs, [prepared[i][0]], [prepared[i][1]])
-    dt = time.time() - t0
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):  # one thread, BLAS included
+        for i in range(args.warmup):
+            oracle_sample_step(w, tabs, [prepared[i][0]], [prepared[i][1]])
+        t0 = time.time()
+        for i in range(args.warmup, args.warmup + args.steps):
+            oracle_sample_step(w, tabs, [prepared[i][0]], [prepared[i][1]])
+        dt = time.time() - t0
     kv_tokens = args.steps * w.T / w.Hkv
     value = kv_tokens / dt
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
