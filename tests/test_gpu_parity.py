@@ -98,6 +98,10 @@ APPEND_CASES = [
     ("qwen3_8b_b16_t8k", 4096, 2.26, 2.26),
     ("llama_b32_t32k_1p96", 4096, 1.96, 1.96),
     ("llama_b32_t32k_3p0", 4096, 3.0, 3.0),
+    # asymmetric budgets (48-byte K, 31-byte V) and the largest container (64 bytes)
+    ("qwen3_8b_b16_t8k", 300, 3.0, 1.96),
+    ("qwen3_8b_b16_t8k", 4096, 1.96, 3.0),
+    ("qwen3_8b_b16_t8k", 300, 4.0, 4.0),
 ]
 
 
@@ -205,6 +209,24 @@ def test_attention_parity(wname, B, Hkv, G, T, seq, q_dtype):
     stats = dq.new_stats()
     got = cm.gpu_attention(lib, q, kc, vc, seq, q_dtype=q_dtype, stats=stats)
     cm.assert_attention_close(got, ref, what=str((wname, B, Hkv, G, T)))
+    assert dq.stats_dict(stats)["integrity_errors"] == 0
+
+
+@pytest.mark.parametrize("kb,vb", [(3.0, 1.96), (1.96, 3.0), (4.0, 4.0)])
+def test_attention_parity_other_budgets(kb, vb):
+    w = synth.scaled(synth.WORKLOADS["qwen3_8b_b16_t8k"], B=3, Hkv=2, Hq=8, T=700)
+    K, V, q = cm.inputs(w)
+    ref_t = cm.oracle_tables(2, kb, vb)
+    lib = cm.lib_tables(2, kb, vb)
+    rk, rv, _, _, _, _ = o.encode_cache(ref_t, K, V)
+    kc, vc = cm.gpu_append_all(lib, K, V, w.torch_dtype)
+    np.testing.assert_array_equal(cm.flat(kc)[:, :, :700], rk)
+    np.testing.assert_array_equal(cm.flat(vc)[:, :, :700], rv)
+    seq = [700, 255, 1]
+    ref = o.attention_fp64(ref_t, q, rk, rv, seq)
+    stats = dq.new_stats()
+    got = cm.gpu_attention(lib, q, kc, vc, seq, stats=stats)
+    cm.assert_attention_close(got, ref, what="budgets %s/%s" % (kb, vb))
     assert dq.stats_dict(stats)["integrity_errors"] == 0
 
 
