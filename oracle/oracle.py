@@ -374,3 +374,48 @@ def attention_fp64(tab: Tables, q: np.ndarray, kcache: np.ndarray, vcache: np.nd
             p /= p.sum()
             out[b, h * G + g] = p @ vh
     return out
+
+
+def attention_prefill_fp64(tab: Tables, q: np.ndarray, kcache: np.ndarray, vcache: np.ndarray,
+                           q_start, sm_scale: float | None = None, rows=None) -> np.ndarray:
+    """Causal attention of a prompt chunk over the dequantised cache, fp64.
+
+    [news] "D-Quant: Entropy Coding Meets KV Cache at 2.26 Bits", "The
+    Numbers": long prompts are processed chunk by chunk; the chunk's own K
+    and V are in the cache before it attends. q [B, n_q, Hq, 128]; query
+    token i of sequence b sits at position p = q_start[b] + i and attends to
+    cache positions 0 .. p (softmax(sm_scale q K^T) V over those rows of the
+    dequantised cache). A position outside [0, T_cap) gives 0. Query head hq
+    reads KV head hq // (Hq / Hkv). ``rows`` optionally limits the work to a
+    list of (b, h_kv) pairs (other outputs are NaN)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, n_q, Hq, _ = q.shape
+    Hkv, T_cap = kcache.shape[1], kcache.shape[2]
+    G = Hq // Hkv
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    out = np.full((B, n_q, Hq, D), np.nan)
+    if rows is None:
+        rows = [(b, h) for b in range(B) for h in range(Hkv)]
+    for b, h in rows:
+        pos = int(q_start[b]) + np.arange(n_q)
+        ok = (pos >= 0) & (pos < T_cap)
+        out[b, :, h * G:(h + 1) * G] = 0.0
+        if not ok.any():
+            continue
+        T = int(pos[ok].max()) + 1
+        ks, kn, kstat = decode_containers(tab.k, kcache[b, h, :T])
+        vs, vn, vstat = decode_containers(tab.v, vcache[b, h, :T])
+        assert not kstat.any() and not vstat.any(), "corrupt container in oracle input"
+        kh = dequantize(tab.k, ks, kn, tab.signs[h])
+        vh = dequantize(tab.v, vs, vn, tab.signs[h])
+        qi = np.nonzero(ok)[0]                            # query tokens with a valid position
+        mask = np.arange(T)[None, :] <= pos[qi, None]     # [rows, T]: key t visible to query i
+        for g in range(G):
+            a = sm_scale * (q[b, qi, h * G + g] @ kh.T)  # [rows, T]
+            a = np.where(mask, a, -np.inf)
+            a = a - a.max(axis=1, keepdims=True)
+            p = np.exp(a)                                  # exp(-inf) = 0 outside the mask
+            p /= p.sum(axis=1, keepdims=True)
+            out[b, qi, h * G + g] = p @ vh
+    return out
