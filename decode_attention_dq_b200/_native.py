@@ -19,12 +19,13 @@ DQ_F32, DQ_BF16 = 0, 1
 DQ_STREAM_K, DQ_STREAM_V = 0, 1
 STATS_FIELDS = ("k_syms_drifted", "v_syms_drifted", "k_cont_drifted", "v_cont_drifted",
                 "overflow_fallbacks", "integrity_errors", "nonfinite_inputs",
-                "dropped_writes", "clamped_lengths", "bad_pages")
+                "dropped_writes", "clamped_lengths", "bad_pages", "wait_timeouts")
 EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_stream_table",
             "dq_get_stream_design", "dq_get_signs", "dq_append_kv", "dq_decode_workspace_bytes",
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",
             "dq_design_stream", "dq_decode_attention_noalloc", "dq_append_workspace_bytes",
-            "dq_append_kv_ws", "dq_append_kv_paged", "dq_decode_attention_paged")
+            "dq_append_kv_ws", "dq_append_kv_paged", "dq_decode_attention_paged",
+            "dq_prefill_attention", "dq_prefill_attention_paged")
 
 
 class DqConfig(C.Structure):
@@ -86,6 +87,10 @@ def load():
     lib.dq_decode_symbols.argtypes = [vp, vp, C.c_int, i64, vp, vp, vp, vp, vp]
     lib.dq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int,
                                                 C.c_int, i64, i64, C.c_float, vp, C.c_int, vp, vp]
+    lib.dq_prefill_attention.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int, C.c_int,
+                                         C.c_int, i64, C.c_float, vp, C.c_int, vp, vp]
+    lib.dq_prefill_attention_paged.argtypes = [vp, vp, C.c_int, vp, vp, i64, vp, i64, vp, C.c_int,
+                                               C.c_int, C.c_int, C.c_int, C.c_float, vp, C.c_int, vp, vp]
     lib.dq_error_string.argtypes = [C.c_int]
     lib.dq_error_string.restype = C.c_char_p
     lib.dq_last_cuda_error.argtypes = []
@@ -285,6 +290,40 @@ def dq_decode_attention_noalloc(tab: Tables, q: torch.Tensor, kcache: torch.Tens
         tab.handle, _ptr(q), _dtype_code(q), _ptr(kcache), _ptr(vcache), _ptr(seq_lens), B, Hq,
         Hkv, T_cap, T_max, float(sm_scale), _ptr(out), _dtype_code(out), _ptr(stats),
         _stream(stream)))
+
+
+def dq_prefill_attention(tab: Tables, q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
+                         q_start: torch.Tensor, out: torch.Tensor, sm_scale: float | None = None,
+                         stats: torch.Tensor | None = None, stream=None) -> None:
+    """Chunked-prefill attention: q [B, n_q, Hq, 128] (query token i of
+    sequence b at position q_start[b] + i, causal over the cache); caches
+    uint8 [B, Hkv, T_cap, C]; q_start int32 [B]; out [B, n_q, Hq, 128]."""
+    B, n_q, Hq, d = q.shape
+    Hkv, T_cap = kcache.shape[1], kcache.shape[2]
+    assert d == 128 and q.is_contiguous() and out.is_contiguous() and q_start.dtype == torch.int32
+    assert out.shape == q.shape
+    if sm_scale is None:
+        sm_scale = 128 ** -0.5
+    _check("dq_prefill_attention", load().dq_prefill_attention(
+        tab.handle, _ptr(q), _dtype_code(q), _ptr(kcache), _ptr(vcache), _ptr(q_start), B, n_q, Hq,
+        Hkv, T_cap, float(sm_scale), _ptr(out), _dtype_code(out), _ptr(stats), _stream(stream)))
+
+
+def dq_prefill_attention_paged(tab: Tables, q: torch.Tensor, kpool: torch.Tensor, vpool: torch.Tensor,
+                               page_table: torch.Tensor, q_start: torch.Tensor, out: torch.Tensor,
+                               sm_scale: float | None = None, stats: torch.Tensor | None = None,
+                               stream=None) -> None:
+    """Chunked-prefill attention over page pools (see dq_prefill_attention)."""
+    B, n_q, Hq, d = q.shape
+    Hkv = kpool.shape[1]
+    assert d == 128 and q.is_contiguous() and out.is_contiguous() and q_start.dtype == torch.int32
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous() and out.shape == q.shape
+    if sm_scale is None:
+        sm_scale = 128 ** -0.5
+    _check("dq_prefill_attention_paged", load().dq_prefill_attention_paged(
+        tab.handle, _ptr(q), _dtype_code(q), _ptr(kpool), _ptr(vpool), kpool.shape[0],
+        _ptr(page_table), page_table.shape[1], _ptr(q_start), B, n_q, Hq, Hkv, float(sm_scale),
+        _ptr(out), _dtype_code(out), _ptr(stats), _stream(stream)))
 
 
 def dq_decode_symbols(tab: Tables, cache: torch.Tensor, kind: int, syms: torch.Tensor,

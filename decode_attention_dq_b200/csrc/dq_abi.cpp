@@ -95,6 +95,39 @@ void choose_tile_scale(const dqi::StreamDesign &d, dqi::DevStream *s) {
     s->level16[i] = i < d.n_levels ? f32_to_f16_rn(static_cast<float>(best_k * static_cast<double>(d.levels[i]))) : 0u;
 }
 
+// Scale kappa in [1, 2) (steps of 2^-16) for the prefill score operand:
+// minimises sum_s f_s |fp16(kappa y_s) / kappa - y_s|, the expected absolute
+// error of a coordinate's level, so the frequent inner levels are the exact
+// ones; the smallest such kappa on ties.
+void choose_score_scale(const dqi::StreamDesign &d, dqi::DevStream *s) {
+  double best_err = INFINITY;
+  double best_k = 1.0;
+  for (int j = 0; j < 65536; ++j) {
+    const double kappa = 1.0 + j / 65536.0;
+    double err = 0.0;
+    for (int i = 0; i < d.n_levels; ++i) {
+      const double y = static_cast<double>(d.levels[i]);
+      const double h = f16_to_double(f32_to_f16_rn(static_cast<float>(kappa * y)));
+      err += static_cast<double>(d.freq[i]) * std::fabs(h / kappa - y);
+    }
+    if (err < best_err) {
+      best_err = err;
+      best_k = kappa;
+    }
+  }
+  double worst = 0.0;
+  for (int i = 0; i < dqi::kMaxLevels; ++i) {
+    s->score16[i] = 0u;
+    if (i >= d.n_levels) continue;
+    const double y = static_cast<double>(d.levels[i]);
+    s->score16[i] = f32_to_f16_rn(static_cast<float>(best_k * y));
+    if (y != 0.0) worst = std::max(worst, std::fabs(f16_to_double(static_cast<uint16_t>(s->score16[i])) - best_k * y) /
+                                              std::fabs(best_k * y));
+  }
+  s->score_scale = static_cast<float>(best_k);
+  s->score_err = static_cast<float>(worst);
+}
+
 void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
   std::memset(s, 0, sizeof(*s));
   for (int sym = 0; sym < d.n_levels; ++sym)
@@ -108,6 +141,7 @@ void fill_dev_stream(const dqi::StreamDesign &d, dqi::DevStream *s) {
     s->cum[i] = i < d.n_levels ? d.cum[i] : dqi::kM;
   }
   choose_tile_scale(d, s);
+  choose_score_scale(d, s);
   s->n_levels = d.n_levels;
   s->container_bytes = d.container_bytes;
   s->payload_bytes = d.payload_bytes;
@@ -482,6 +516,80 @@ int dq_decode_attention_paged(const dq_tables *t, const void *q, int q_dtype, co
   if (!aligned(d_page_table, 4)) return DQ_ERR_ALIGN;
   return decode_core(t, q, q_dtype, d_kpool, d_vpool, d_seq_lens, B, Hq, Hkv, 32 * max_pages, T_max, sm_scale,
                      out, out_dtype, d_workspace, ws_bytes, d_stats, stream, d_page_table, max_pages, num_pages);
+}
+
+static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
+                        const uint8_t *d_vcache, const int32_t *d_q_start, int B, int n_q, int Hq, int Hkv,
+                        int64_t T_cap, float sm_scale, void *out, int out_dtype, dq_stats *d_stats, void *stream,
+                        const int32_t *page_table, int64_t max_pages, int64_t num_pages) {
+  try {
+    if (!t || !q || !d_kcache || !d_vcache || !d_q_start || !out) return DQ_ERR_NULL;
+    if ((q_dtype != DQ_F32 && q_dtype != DQ_BF16) || (out_dtype != DQ_F32 && out_dtype != DQ_BF16))
+      return DQ_ERR_DTYPE;
+    if (B < 0 || n_q < 0 || Hkv != t->cfg.n_kv_heads || Hq < Hkv || Hq % Hkv) return DQ_ERR_SHAPE;
+    const int G = Hq / Hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return DQ_ERR_SHAPE;
+    if (T_cap < 0) return DQ_ERR_SHAPE;
+    if (T_cap % 32 || !aligned(d_kcache, 16) || !aligned(d_vcache, 16) || !aligned(q, 4) || !aligned(out, 4) ||
+        !aligned(d_q_start, 4))
+      return DQ_ERR_ALIGN;
+    if (!std::isfinite(sm_scale)) return DQ_ERR_SHAPE;
+    const int nd = dqi::prefill_decoder_warps(t->k.container_bytes, t->v.container_bytes);
+    if (nd <= 0) return DQ_ERR_SHAPE;
+    if (dqi::prefill_grid(B, Hkv, G, n_q) > 0x7FFFFFFF) return DQ_ERR_SHAPE;
+    int rc = check_device(t);
+    if (rc != DQ_OK) return rc;
+    if (B == 0 || n_q == 0) return DQ_OK;
+    dqi::PrefillArgs a{};
+    a.tabs = t->d_tabs;
+    a.sign_bits = t->d_sign_bits;
+    a.q = q;
+    a.q_dtype = q_dtype;
+    a.kcache = d_kcache;
+    a.vcache = d_vcache;
+    a.q_start = d_q_start;
+    a.B = B;
+    a.n_q = n_q;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = G;
+    a.T_cap = T_cap;
+    a.sm_scale = sm_scale;
+    a.out = out;
+    a.out_dtype = out_dtype;
+    a.ck = t->k.container_bytes;
+    a.cv = t->v.container_bytes;
+    a.two_k = has_small_freq(t->k);
+    a.two_v = has_small_freq(t->v);
+    a.nd = nd;
+    a.stats = d_stats;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.num_pages = num_pages;
+    int e = dqi::launch_prefill_attention(a, stream);
+    return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
+  } catch (...) {
+    return DQ_ERR_CUDA;
+  }
+}
+
+int dq_prefill_attention(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
+                         const uint8_t *d_vcache, const int32_t *d_q_start, int B, int n_q, int Hq, int Hkv,
+                         int64_t T_cap, float sm_scale, void *out, int out_dtype, dq_stats *d_stats, void *stream) {
+  return prefill_core(t, q, q_dtype, d_kcache, d_vcache, d_q_start, B, n_q, Hq, Hkv, T_cap, sm_scale, out,
+                      out_dtype, d_stats, stream, nullptr, 0, 0);
+}
+
+int dq_prefill_attention_paged(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kpool,
+                               const uint8_t *d_vpool, int64_t num_pages, const int32_t *d_page_table,
+                               int64_t max_pages, const int32_t *d_q_start, int B, int n_q, int Hq, int Hkv,
+                               float sm_scale, void *out, int out_dtype, dq_stats *d_stats, void *stream) {
+  if (!d_page_table) return DQ_ERR_NULL;
+  if (num_pages < 1 || max_pages < 1 || max_pages > (int64_t(1) << 40) || num_pages > (int64_t(1) << 31))
+    return DQ_ERR_SHAPE;
+  if (!aligned(d_page_table, 4)) return DQ_ERR_ALIGN;
+  return prefill_core(t, q, q_dtype, d_kpool, d_vpool, d_q_start, B, n_q, Hq, Hkv, 32 * max_pages, sm_scale, out,
+                      out_dtype, d_stats, stream, d_page_table, max_pages, num_pages);
 }
 
 int dq_decode_symbols(const dq_tables *t, const uint8_t *d_cache, int stream_kind,

@@ -56,6 +56,13 @@ struct alignas(16) DevStream {
   uint32_t level16[kMaxLevels];
   float tile_scale, tile_rel_err;
   int32_t n_levels, container_bytes, payload_bytes, pad;
+  // Levels for the fp16 K operand of the prefill score MMA: score16[s] holds
+  // the fp16 bits of score_scale * levels[s], with score_scale in [1, 2)
+  // chosen to minimise the frequency-weighted absolute error of the levels
+  // (the frequent inner levels come out exact to about 1e-6); score_err is
+  // the largest relative error left (on a rare outer level).
+  uint32_t score16[kMaxLevels];
+  float score_scale, score_err;
 };
 
 struct DevTables {
@@ -120,6 +127,32 @@ struct DecodeArgs {
 int launch_decode_attention(const DecodeArgs &a, void *stream);
 // Warps per CTA of the split kernel for these shapes (0 if unsupported).
 int decode_warps_per_cta(int G, int ck, int cv);
+
+// Chunked-prefill attention (dq_prefill.cu).
+struct PrefillArgs {
+  const DevTables *tabs;
+  const uint32_t *sign_bits;
+  const void *q;       // [B][n_q][Hq][128]
+  int q_dtype;
+  const uint8_t *kcache, *vcache;
+  const int32_t *q_start;  // [B]: position of query token 0 of each sequence
+  int B, n_q, Hq, Hkv, G;
+  int64_t T_cap;
+  float sm_scale;
+  void *out;           // [B][n_q][Hq][128]
+  int out_dtype;
+  int ck, cv;
+  bool two_k, two_v;
+  int nd;              // decoder warps per CTA (prefill_decoder_warps)
+  dq_stats *stats;
+  const int32_t *page_table;  // paged caches as in AppendArgs (nullptr: contiguous)
+  int64_t max_pages, num_pages;
+};
+int launch_prefill_attention(const PrefillArgs &a, void *stream);
+// Decoder warps per CTA for these container sizes (0 if unsupported).
+int prefill_decoder_warps(int ck, int cv);
+// CTAs of one call: B * Hkv * ceil(n_q / (128 / G)).
+int64_t prefill_grid(int B, int Hkv, int G, int n_q);
 
 struct SymbolsArgs {
   const DevStream *tab;

@@ -1,0 +1,716 @@
+// dq_prefill.cu -- chunked-prefill attention over the compressed KV cache,
+// on the sm_100 tensor cores (tcgen05, accumulators in tensor memory).
+//
+// [abstract] "D-Quant: Driftable Entropy Coding for KV Cache Quantization":
+// fixed-size bitstreams give regular memory access and parallel
+// dequantisation within attention kernels. [news] "D-Quant: Entropy Coding
+// Meets KV Cache at 2.26 Bits", "The Numbers": the method is evaluated on
+// long prompts (8K to 128K); a prompt processed in chunks attends, chunk by
+// chunk, over the compressed cache that already holds the chunk's own keys
+// and values. Query token i of sequence b sits at position q_start[b] + i and
+// attends causally to cache positions 0 .. q_start[b] + i.
+//
+// One CTA per (b, KV head h, block of 128 query rows); a row is one query
+// token of the chunk with one of the G query heads of h (rows are token-major:
+// row r = token r / G, head r % G). Warp roles:
+//   warps 0-3  softmax: thread r owns row r, which is lane r of tensor memory.
+//              It rotates its query (q~ = H D q, fp32, times a power of two),
+//              splits it into fp16 hi + lo and stores both into tensor memory
+//              (the A operand of the score MMA); per 32-token group it reads
+//              its 32 scores, applies the key norms, the scale and the causal
+//              mask, runs the online softmax, rescales its row of O in tensor
+//              memory when the running maximum grows, and stores the weights
+//              w = p ||v|| as fp16 hi + lo into tensor memory (the A operand of
+//              the P.V MMA). At the end it applies 1 / (128 l kappa_V), the
+//              inverse rotation D H and writes the output row.
+//   warp 4     owns the tensor memory; one lane issues the MMAs:
+//              S_j = Q~hi K_j^T + Q~lo K_j^T        (M 128, N 32, K 128)
+//              O  += W_j,hi V_j + W_j,lo V_j         (M 128, N 128, K 32)
+//              both of kind f16 with fp32 accumulation, A from tensor memory
+//              and B from shared memory (no swizzle, 8 x 16-byte core
+//              matrices).
+//   warps 5..  decoders: decoder d takes groups d, d + nd, ... of 32 tokens,
+//              stages the group's byte-interleaved K and V containers with
+//              cp.async (one group ahead), rANS-decodes them one lane per
+//              token (K and V chains interleaved) and writes fp16 levels into
+//              its ring slot: kappa_K y for K (kappa_K minimises the
+//              frequency-weighted level error) and kappa_V y for V, with the
+//              tokens' norms beside them.
+// Hand-offs use mbarriers; every wait is bounded, and a CTA that gives up
+// counts the event in wait_timeouts, skips the rest of its work and still
+// frees its tensor memory after its MMAs have drained.
+#include <type_traits>
+
+#include "dq_device.cuh"
+
+namespace dqi {
+namespace {
+
+constexpr int kRows = 128;          // query rows per CTA (the MMA's M)
+constexpr int kGrp = 32;            // tokens per cache block (one per decoder lane)
+constexpr int kSoftWarps = 4;       // warps 0..3
+constexpr int kMmaWarp = 4;         // warp 4
+constexpr int kFirstDec = 5;        // warps 5..5+nd-1
+constexpr int kMaxDec = 7;
+constexpr int kMaxThreads = 32 * (kFirstDec + kMaxDec);
+constexpr uint32_t kTmemCols = 512;
+// Tensor-memory columns (32-bit each; 128 lanes = rows).
+constexpr uint32_t kColO = 0;       // O: 128 fp32 columns
+constexpr uint32_t kColS = 128;     // S: 2 buffers x 32 fp32 columns
+constexpr uint32_t kColP = 192;     // W: 2 buffers x (16 hi + 16 lo) columns of packed fp16 pairs
+constexpr uint32_t kColQh = 256;    // q~ hi: 64 columns of packed fp16 pairs
+constexpr uint32_t kColQl = 320;    // q~ lo: 64 columns
+constexpr int kTileBytes = kGrp * kD * 2;   // one fp16 tile: 32 tokens x 128 coordinates
+constexpr int kSlotBytes = 2 * kTileBytes + 2 * kGrp * 4;  // K tile, V tile, K norms, V norms
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kSpin = 1u << 24;  // bound on each mbarrier wait loop
+// Barrier slots.
+constexpr int kBarFull = 0, kBarEmpty = 8, kBarSFull = 16, kBarSFree = 18, kBarPFull = 20, kBarPvDone = 22,
+              kBarQFull = 24, kBarDrain = 25, kNumBars = 32;
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct PrefillSmem {
+  size_t lut_k, lut_v, lev, bars, misc, ring, stage;
+  size_t kslot, vslot, stage_bytes;  // per decoder warp: K slots 0, 1 then V slots 0, 1
+  size_t total;
+};
+
+__host__ __device__ inline PrefillSmem prefill_smem_layout(int ck, int cv, int nd) {
+  PrefillSmem s;
+  s.lut_k = 0;
+  s.lut_v = s.lut_k + kM * 4;
+  s.lev = s.lut_v + kM * 4;                   // [0..7] K score levels, [8..15] V tile levels (fp16 bits)
+  s.bars = s.lev + 2 * kMaxLevels * 4;
+  s.misc = s.bars + kNumBars * 8;             // tensor-memory base, abort flag
+  s.ring = align_up(s.misc + 16, 128);
+  s.kslot = align_up(static_cast<size_t>(kGrp) * ck, 16);
+  s.vslot = align_up(static_cast<size_t>(kGrp) * cv, 16);
+  s.stage_bytes = 2 * s.kslot + 2 * s.vslot;
+  s.stage = s.ring + static_cast<size_t>(nd) * kSlotBytes;
+  const size_t end = s.stage + static_cast<size_t>(nd) * s.stage_bytes;
+  // A corrupt container moves its decoder's cursor by at most 2 bytes per
+  // symbol (byte 5 + 2 * 128 at most), 32 bytes apart in the interleaved
+  // layout: reads from the last V slot stay inside the allocation.
+  const size_t reach = end - s.vslot + static_cast<size_t>(kGrp) * (kHeaderBytes + 2 * kD + 1);
+  s.total = (reach > end ? align_up(reach, 16) : end) + 256;
+  // At least 116 KB so that one CTA holds an SM (and its tensor memory).
+  if (s.total < 116 * 1024) s.total = 116 * 1024;
+  return s;
+}
+
+// ---- PTX wrappers -------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(smem_u32(bar)) : "memory");
+}
+// Waits for the phase with the given parity to complete. Gives up after
+// kSpin polls, or as soon as another thread of the CTA has given up.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t it = 0; it < kSpin; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\nselp.u32 %0, 1, 0, P;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((it & 255u) == 255u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// d (+)= a b^T: A (M 128 x K 16 fp16) from tensor memory, B from a shared
+// memory descriptor, fp32 accumulators in tensor memory.
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "r"(a), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Shared-memory matrix descriptor, no swizzle: start address, leading and
+// stride byte offsets (16-byte units), version 1 (bits 46-47).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// Instruction descriptor, kind f16: fp32 accumulators (bit 4), A and B fp16,
+// A K-major, B K-major (0) or MN-major (1) at bit 16, N / 8 at bits 17-22,
+// M / 16 at bits 24-28.
+__host__ __device__ constexpr uint32_t instr_desc(int M, int N, int b_mn) {
+  return (1u << 4) | (static_cast<uint32_t>(b_mn) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// 32 consecutive fp32 columns of this warp's 32 lanes (one row per thread).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// fp16 hi + lo of a pair of fp32 values, packed (first value in the low half).
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
+// Unnormalised Walsh-Hadamard transform of 128 values in registers (stages
+// h = 1, 2, ..., 64, butterfly (a, b) -> (a + b, a - b)).
+__device__ __forceinline__ void wht128_regs(float (&v)[kD]) {
+#pragma unroll
+  for (int h = 1; h < kD; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < kD; ++i)
+      if ((i & h) == 0) {
+        const float a0 = v[i], a1 = v[i + h];
+        v[i] = __fadd_rn(a0, a1);
+        v[i + h] = __fsub_rn(a0, a1);
+      }
+}
+
+// ---- rANS decoding (one lane per token of a staged 32-token block) ------
+
+struct RansLane {
+  uint32_t x;
+  uint32_t p;  // shared-memory offset of the next byte
+};
+
+__device__ __forceinline__ RansLane rans_open(const uint8_t *smem, uint32_t off) {
+  RansLane r;
+  r.x = static_cast<uint32_t>(smem[off + 2 * kGrp]) | (static_cast<uint32_t>(smem[off + 3 * kGrp]) << 8) |
+        (static_cast<uint32_t>(smem[off + 4 * kGrp]) << 16);
+  r.p = off + kHeaderBytes * kGrp;
+  return r;
+}
+
+// One decode step (table entry: bits 0..10 slot - c_s, 11..13 s, 20..31 f_s):
+// x = f (x >> 12) + slot - c_s, then arithmetic byte renormalisation (one
+// byte, or two for tables with a symbol of f < 16). Returns 4 s.
+template <bool kTwo>
+__device__ __forceinline__ uint32_t rans_step(RansLane &r, const uint32_t *lut, const uint8_t *smem) {
+  const uint32_t e = lut[r.x & (kM - 1)];
+  uint32_t x = (e >> 20) * (r.x >> kProbBits) + (e & 0x7FFu);
+  const uint32_t b0 = smem[r.p];
+  const uint32_t b1 = kTwo ? static_cast<uint32_t>(smem[r.p + kGrp]) : 0u;
+  const uint32_t n0 = __umulhi(x - kL, 2u);
+  x += n0 * (x * 255u + b0);
+  uint32_t adv = n0;
+  if constexpr (kTwo) {
+    const uint32_t n1 = __umulhi(x - kL, 2u);
+    x += n1 * (x * 255u + b1);
+    adv += n1;
+  }
+  r.p += adv * kGrp;
+  r.x = x;
+  return (e >> 9) & 0x1Cu;
+}
+
+__device__ __forceinline__ float norm_of(const uint8_t *cb) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(cb[0] | (cb[kGrp] << 8))));
+}
+
+template <bool kTwoK, bool kTwoV>
+__global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int nd = a.nd;
+  const PrefillSmem L = prefill_smem_layout(a.ck, a.cv, nd);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t *lut_k = reinterpret_cast<uint32_t *>(smem + L.lut_k);
+  uint32_t *lut_v = reinterpret_cast<uint32_t *>(smem + L.lut_v);
+  uint32_t *lev = reinterpret_cast<uint32_t *>(smem + L.lev);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + L.misc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 4);
+  auto slot_base = [&](int d) { return smem + L.ring + static_cast<size_t>(d) * kSlotBytes; };
+
+  // Work item; late query blocks (the longest causal ranges) first.
+  const int G = a.G, Mt = kRows / G;
+  const int nqb = (a.n_q + Mt - 1) / Mt;
+  const int64_t BH = static_cast<int64_t>(a.B) * a.Hkv;
+  const int64_t bid = blockIdx.x;
+  const int qb = nqb - 1 - static_cast<int>(bid / BH);
+  const int64_t bh = bid % BH;
+  const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
+  const int64_t qs = a.q_start[b];
+  const int i_lo = qb * Mt;
+  const int i_hi = min(i_lo + Mt, a.n_q) - 1;
+  const int64_t lo_pos = max(qs + i_lo, int64_t(0));
+  const int64_t hi_pos = min(qs + i_hi, a.T_cap - 1);
+  const int64_t nG = lo_pos <= hi_pos ? hi_pos / kGrp + 1 : 0;
+  // Tokens whose integrity this CTA reports: those the previous query block
+  // of (b, h) does not reach, so each container is counted once.
+  const int64_t prev_hi = qb == 0 ? int64_t(-1) : min(qs + i_lo - 1, a.T_cap - 1);
+
+  // ---- set-up ----
+  {
+    const uint4 *sk = reinterpret_cast<const uint4 *>(a.tabs->k.lut);
+    const uint4 *sv = reinterpret_cast<const uint4 *>(a.tabs->v.lut);
+    uint4 *dk = reinterpret_cast<uint4 *>(lut_k);
+    uint4 *dv = reinterpret_cast<uint4 *>(lut_v);
+    for (int i = tid; i < static_cast<int>(kM / 4); i += blockDim.x) {
+      dk[i] = __ldg(sk + i);
+      dv[i] = __ldg(sv + i);
+    }
+    if (tid < kMaxLevels) {
+      lev[tid] = a.tabs->k.score16[tid];
+      lev[kMaxLevels + tid] = a.tabs->v.level16[tid];
+    }
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  if (tid == 0) {
+    for (int d = 0; d < nd; ++d) {
+      mbar_init(bars + kBarFull + d, 32);
+      mbar_init(bars + kBarEmpty + d, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + kBarSFull + i, 1);
+      mbar_init(bars + kBarSFree + i, kRows);
+      mbar_init(bars + kBarPFull + i, kRows);
+      mbar_init(bars + kBarPvDone + i, 1);
+    }
+    mbar_init(bars + kBarQFull, kRows);
+    mbar_init(bars + kBarDrain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+  unsigned timeouts = 0, bad = 0, bad_pages = 0, clamped = 0;
+
+  if (warp < kSoftWarps) {
+    // ================= softmax warpgroup: thread = row =================
+    const int r = tid;
+    const uint32_t tl = tbase + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lanes
+    const int ti = i_lo + r / G, g = r % G;
+    const bool in_chunk = ti <= i_hi;
+    const int64_t pos = qs + ti;
+    const bool row_ok = in_chunk && pos >= 0 && pos < a.T_cap;
+    if (in_chunk && !row_ok) ++clamped;
+    const int hq = h * G + g;
+    const int64_t qbase = ((static_cast<int64_t>(b) * a.n_q + (in_chunk ? ti : 0)) * a.Hq + hq) * kD;
+    // D1: q~ = H D q (unnormalised), times 2^e so that max |q~| is in [2^13, 2^14).
+    float crow = 0.0f;
+    {
+      float v[kD];
+      uint32_t sw[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
+#pragma unroll
+      for (int c = 0; c < kD; ++c) {
+        const float x = in_chunk ? load_elem(a.q, qbase + c, a.q_dtype) : 0.0f;
+        v[c] = ((sw[c >> 5] >> (c & 31)) & 1u) ? -x : x;
+      }
+      wht128_regs(v);
+      float amax = 0.0f;
+#pragma unroll
+      for (int c = 0; c < kD; ++c) amax = fmaxf(amax, fabsf(v[c]));
+      float sc = 1.0f;
+      if (amax > 0.0f && amax < INFINITY) {
+        int ex;
+        frexpf(amax, &ex);
+        sc = ldexpf(1.0f, 14 - ex);
+      }
+      // logit (log2 units) = S * ||k|| * crow, with S = sum (q~ sc)(kappa_K y)
+      crow = row_ok ? a.sm_scale * kLog2e / (static_cast<float>(kD) * sc * a.tabs->k.score_scale) : 0.0f;
+#pragma unroll
+      for (int c16 = 0; c16 < kD; c16 += 16) {
+        uint32_t hi[8], lo[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) split_pair(v[c16 + 2 * p] * sc, v[c16 + 2 * p + 1] * sc, hi[p], lo[p]);
+        tmem_st8(tl + kColQh + c16 / 2, hi);
+        tmem_st8(tl + kColQl + c16 / 2, lo);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    mbar_arrive(bars + kBarQFull);
+
+    float m_run = -INFINITY, l_run = 0.0f;
+    bool alive = true;
+    for (int64_t j = 0; j < nG && alive; ++j) {
+      const int sb = static_cast<int>(j & 1);
+      const int rb = static_cast<int>(j % nd);
+      bool ok = mbar_wait(bars + kBarSFull + sb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) &&
+                mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / nd) & 1), abort_flag);
+      if (!__all_sync(kFull, ok)) {
+        ++timeouts;
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      float s[32];
+      tmem_ld32(tl + kColS + 32 * sb, s);
+      tc_fence_before();
+      mbar_arrive(bars + kBarSFree + sb);
+      const float *nk = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes);
+      const float *nv = nk + kGrp;
+      const int64_t t0 = j * kGrp;
+      float mx = m_run;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const bool valid = row_ok && t0 + t <= pos;
+        s[t] = valid ? s[t] * nk[t] * crow : -INFINITY;
+        mx = fmaxf(mx, s[t]);
+      }
+      float alpha = 1.0f;
+      uint32_t whi[16], wlo[16];
+      float psum = 0.0f;
+      if (mx == -INFINITY) {
+#pragma unroll
+        for (int p = 0; p < 16; ++p) whi[p] = wlo[p] = 0u;
+      } else {
+        if (m_run != -INFINITY) alpha = exp2f(m_run - mx);
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float p0 = exp2f(s[2 * p] - mx), p1 = exp2f(s[2 * p + 1] - mx);
+          psum += p0 + p1;
+          const float w0 = p0 > 0.0f ? p0 * nv[2 * p] : 0.0f;
+          const float w1 = p1 > 0.0f ? p1 * nv[2 * p + 1] : 0.0f;
+          split_pair(w0, w1, whi[p], wlo[p]);
+        }
+        m_run = mx;
+      }
+      l_run = l_run * alpha + psum;
+      // O and the W buffer are free once P.V of the previous group is done.
+      if (j > 0) {
+        ok = mbar_wait(bars + kBarPvDone + ((j - 1) & 1), static_cast<uint32_t>(((j - 1) >> 1) & 1), abort_flag);
+        if (!__all_sync(kFull, ok)) {
+          ++timeouts;
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(kFull, alpha != 1.0f)) {
+#pragma unroll 1
+          for (int c = 0; c < kD; c += 32) {
+            float o[32];
+            tmem_ld32(tl + kColO + c, o);
+            uint32_t w[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * alpha);
+            uint32_t w0[16], w1[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              w0[e] = w[e];
+              w1[e] = w[16 + e];
+            }
+            tmem_st16(tl + kColO + c, w0);
+            tmem_st16(tl + kColO + c + 16, w1);
+          }
+        }
+      }
+      tmem_st16(tl + kColP + 32 * sb, whi);
+      tmem_st16(tl + kColP + 32 * sb + 16, wlo);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bars + kBarPFull + sb);
+    }
+    // D7: o = D H o_rot / 128 with o_rot = O / (l kappa_V).
+    bool have_o = alive && nG > 0;
+    if (have_o) {
+      const int64_t jl = nG - 1;
+      const bool ok =
+          mbar_wait(bars + kBarPvDone + (jl & 1), static_cast<uint32_t>((jl >> 1) & 1), abort_flag);
+      if (!__all_sync(kFull, ok)) {
+        ++timeouts;
+        have_o = false;
+      }
+    }
+    {
+      float v[kD];
+      if (have_o) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kD; c += 32) {
+          float o[32];
+          tmem_ld32(tl + kColO + c, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[c + e] = o[e];
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kD; ++c) v[c] = 0.0f;
+      }
+      const float inv =
+          (have_o && row_ok && l_run > 0.0f) ? 1.0f / (l_run * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
+#pragma unroll
+      for (int c = 0; c < kD; ++c) v[c] *= inv;
+      wht128_regs(v);
+      if (in_chunk) {
+        uint32_t sw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
+#pragma unroll
+        for (int c = 0; c < kD; ++c) {
+          const float o = ((sw[c >> 5] >> (c & 31)) & 1u) ? -v[c] : v[c];
+          store_elem(a.out, qbase + c, o, a.out_dtype);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issue (one lane) =================
+    if (lane == 0 && nG > 0) {
+      const uint32_t idS = instr_desc(kRows, kGrp, 0);
+      const uint32_t idO = instr_desc(kRows, kD, 1);
+      bool alive = mbar_wait(bars + kBarQFull, 0, abort_flag);
+      if (!alive) ++timeouts;
+      tc_fence_after();
+      // W_jj V_jj into O: A = W hi / lo (tensor memory, 8 columns per 16
+      // tokens), B = V tile, MN-major: token groups of 8 at 128 bytes (LBO),
+      // coordinate chunks of 8 at 512 bytes (SBO).
+      auto issue_pv = [&](int64_t jj) -> bool {
+        if (!mbar_wait(bars + kBarPFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vt = smem_u32(slot_base(static_cast<int>(jj % nd)) + kTileBytes);
+        const uint32_t wp = tbase + kColP + 32 * static_cast<uint32_t>(jj & 1);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const uint64_t bd = smem_desc(vt + ks * 256, 128, 512);
+          mma_ts(tbase + kColO, wp + ks * 8, bd, idO, (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tbase + kColO, wp + 16 + ks * 8, bd, idO, 1u);
+        }
+        tc_commit(bars + kBarPvDone + (jj & 1));
+        tc_commit(bars + kBarEmpty + static_cast<int>(jj % nd));
+        return true;
+      };
+      for (int64_t j = 0; j < nG && alive; ++j) {
+        const int rb = static_cast<int>(j % nd);
+        alive = mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / nd) & 1), abort_flag);
+        if (alive && j >= 2)
+          alive = mbar_wait(bars + kBarSFree + (j & 1), static_cast<uint32_t>(((j - 2) >> 1) & 1), abort_flag);
+        if (!alive) {
+          ++timeouts;
+          break;
+        }
+        tc_fence_after();
+        // S_j = q~ K_j^T: B = K tile, K-major: token groups of 8 at 128 bytes
+        // (SBO), coordinate chunks of 8 at 512 bytes (LBO).
+        const uint32_t kt = smem_u32(slot_base(rb));
+        const uint32_t sd = tbase + kColS + 32 * static_cast<uint32_t>(j & 1);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint64_t bd = smem_desc(kt + ks * 1024, 512, 128);
+          mma_ts(sd, tbase + kColQh + ks * 8, bd, idS, ks > 0 ? 1u : 0u);
+          mma_ts(sd, tbase + kColQl + ks * 8, bd, idS, 1u);
+        }
+        tc_commit(bars + kBarSFull + (j & 1));
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ++timeouts;
+          alive = false;
+        }
+      }
+      if (alive && !issue_pv(nG - 1)) ++timeouts;
+      // Drain: every MMA issued above has completed before tensor memory is freed.
+      tc_commit(bars + kBarDrain);
+      if (!mbar_wait(bars + kBarDrain, 0, abort_flag)) {
+        // The abort path may skip the wait above; wait once more without
+        // looking at the flag, still bounded.
+        const uint32_t da = smem_u32(bars + kBarDrain);
+        for (uint32_t it = 0; it < kSpin; ++it) {
+          uint32_t done;
+          asm volatile(
+              "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], 0;\nselp.u32 %0, 1, 0, P;\n}\n"
+              : "=r"(done)
+              : "r"(da)
+              : "memory");
+          if (done) break;
+        }
+      }
+    }
+  } else {
+    // ================= decoders =================
+    const int d = warp - kFirstDec;
+    uint8_t *stg = smem + L.stage + static_cast<size_t>(d) * L.stage_bytes;
+    auto kslot = [&](int s) { return stg + s * L.kslot; };
+    auto vslot = [&](int s) { return stg + 2 * L.kslot + s * L.vslot; };
+    uint8_t *kt = slot_base(d);
+    uint8_t *vt = kt + kTileBytes;
+    float *nk = reinterpret_cast<float *>(kt + 2 * kTileBytes);
+    float *nv = nk + kGrp;
+    const int ck = a.ck, cv = a.cv;
+    auto block_of = [&](int64_t j) -> int64_t {
+      if (a.page_table) {
+        int64_t pg = a.page_table[static_cast<int64_t>(b) * a.max_pages + j];
+        if (pg < 0 || pg >= a.num_pages) {
+          ++bad_pages;
+          pg = 0;
+        }
+        return pg * a.Hkv + h;
+      }
+      return bh * (a.T_cap / kGrp) + j;
+    };
+    auto stage = [&](int s, int64_t j) {
+      const int64_t blk = block_of(j);
+      const uint8_t *ks = a.kcache + blk * kGrp * ck;
+      const uint8_t *vs = a.vcache + blk * kGrp * cv;
+      for (int c = lane; c < (kGrp * ck) >> 4; c += 32) cp_async16(kslot(s) + c * 16, ks + c * 16);
+      for (int c = lane; c < (kGrp * cv) >> 4; c += 32) cp_async16(vslot(s) + c * 16, vs + c * 16);
+    };
+    int64_t j = d;
+    if (j < nG) stage(0, j);
+    cp_async_commit();
+    for (int k = 0; j < nG; j += nd, ++k) {
+      const int s = k & 1;
+      if (j + nd < nG) stage(s ^ 1, j + nd);
+      cp_async_commit();
+      cp_async_wait_1();
+      __syncwarp();
+      if (k >= 1) {
+        const bool ok = mbar_wait(bars + kBarEmpty + d, static_cast<uint32_t>((k - 1) & 1), abort_flag);
+        if (!__all_sync(kFull, ok)) {
+          ++timeouts;
+          break;
+        }
+      }
+      const uint8_t *kb = kslot(s) + lane;
+      const uint8_t *vb = vslot(s) + lane;
+      RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
+      RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
+#pragma unroll 1
+      for (int i8 = 0; i8 < kD; i8 += 8) {
+        uint32_t hk[8], hv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
+          const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
+          hk[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + ek);
+          hv[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + 4 * kMaxLevels + ev);
+        }
+        // 8 coordinates of this lane's token: 16 bytes at chunk i8 / 8
+        // (512 bytes per chunk of 32 tokens), token offset 16 * lane.
+        const uint32_t off = static_cast<uint32_t>((i8 >> 3) * 512 + lane * 16);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(smem_u32(kt) + off),
+                     "r"(__byte_perm(hk[0], hk[1], 0x5410)), "r"(__byte_perm(hk[2], hk[3], 0x5410)),
+                     "r"(__byte_perm(hk[4], hk[5], 0x5410)), "r"(__byte_perm(hk[6], hk[7], 0x5410))
+                     : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(smem_u32(vt) + off),
+                     "r"(__byte_perm(hv[0], hv[1], 0x5410)), "r"(__byte_perm(hv[2], hv[3], 0x5410)),
+                     "r"(__byte_perm(hv[4], hv[5], 0x5410)), "r"(__byte_perm(hv[6], hv[7], 0x5410))
+                     : "memory");
+      }
+      nk[lane] = norm_of(kb);
+      nv[lane] = norm_of(vb);
+      const int64_t tok = j * kGrp + lane;
+      if (tok > prev_hi && tok <= hi_pos) bad += (rk.x != kL) + (rv.x != kL);
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      mbar_arrive(bars + kBarFull + d);
+    }
+    cp_async_wait_0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tbase), "r"(kTmemCols) : "memory");
+  }
+  if (a.stats) {
+    const unsigned t_w = __reduce_add_sync(kFull, timeouts);
+    const unsigned b_w = __reduce_add_sync(kFull, bad);
+    const unsigned p_w = __reduce_add_sync(kFull, bad_pages);
+    const unsigned c_w = __reduce_add_sync(kFull, clamped);
+    if (lane == 0) {
+      if (t_w) atomicAdd(&a.stats->wait_timeouts, static_cast<unsigned long long>(t_w));
+      if (b_w) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(b_w));
+      if (p_w) atomicAdd(&a.stats->bad_pages, static_cast<unsigned long long>(p_w));
+      if (c_w) atomicAdd(&a.stats->clamped_lengths, static_cast<unsigned long long>(c_w));
+    }
+  }
+}
+
+template <bool kTwoK, bool kTwoV>
+int launch_prefill_t(const PrefillArgs &a, int64_t grid, cudaStream_t st) {
+  const PrefillSmem L = prefill_smem_layout(a.ck, a.cv, a.nd);
+  auto kern = prefill_kernel<kTwoK, kTwoV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  if (e != cudaSuccess) return static_cast<int>(e);
+  kern<<<static_cast<unsigned>(grid), 32 * (kFirstDec + a.nd), L.total, st>>>(a);
+  return static_cast<int>(cudaGetLastError());
+}
+
+}  // namespace
+
+int prefill_decoder_warps(int ck, int cv) {
+  if (ck < 1 || cv < 1 || ck > kMaxContainer || cv > kMaxContainer) return 0;
+  // At least two decoders: group j + 1 is decoded while P.V of group j still
+  // reads its slot (the MMA loop issues P.V of group j after S of group j + 1).
+  for (int nd = kMaxDec; nd >= 2; --nd)
+    if (prefill_smem_layout(ck, cv, nd).total <= 227 * 1024) return nd;
+  return 0;
+}
+
+int64_t prefill_grid(int B, int Hkv, int G, int n_q) {
+  const int Mt = kRows / G;
+  return static_cast<int64_t>(B) * Hkv * ((n_q + Mt - 1) / Mt);
+}
+
+int launch_prefill_attention(const PrefillArgs &a, void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (a.nd < 2 || a.nd > kMaxDec || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8))
+    return static_cast<int>(cudaErrorInvalidValue);
+  const int64_t grid = prefill_grid(a.B, a.Hkv, a.G, a.n_q);
+  if (grid < 1 || grid > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidValue);
+  if (a.two_k && a.two_v) return launch_prefill_t<true, true>(a, grid, st);
+  if (a.two_k) return launch_prefill_t<true, false>(a, grid, st);
+  if (a.two_v) return launch_prefill_t<false, true>(a, grid, st);
+  return launch_prefill_t<false, false>(a, grid, st);
+}
+
+}  // namespace dqi

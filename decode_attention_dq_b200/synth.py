@@ -131,6 +131,12 @@ def q_block(w: Workload, step: int = 0) -> np.ndarray:
     return np.stack([q_rows(w, b, step) for b in range(w.B)])
 
 
+def q_chunk(w: Workload, n_q: int, first_step: int = 0) -> np.ndarray:
+    """Queries of a prompt chunk: float32 [B, n_q, Hq, 128]; query token i of
+    sequence b is q_rows(w, b, first_step + i)."""
+    return np.stack([np.stack([q_rows(w, b, first_step + i) for i in range(n_q)]) for b in range(w.B)])
+
+
 def scaled(w: Workload, **changes) -> Workload:
     """The same recipe at other sizes (for tests at sizes the oracle finishes)."""
     d = dict(name=w.name + "_small", B=w.B, Hkv=w.Hkv, Hq=w.Hq, T=w.T, dtype=w.dtype,
