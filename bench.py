@@ -12,10 +12,13 @@ per step); the HBM rate of the compressed bytes and the dominant kernel's
 roofline fraction are reported beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dq|reference]
-                  [--workload NAME] [--paged] [--layers L] [--graph]
+                  [--workload NAME] [--paged] [--layers L] [--graph] [--prefill N_Q]
 --paged keeps the caches in page pools behind a shuffled page table; --layers
 runs an L-layer attention-only decode loop (one cache per layer); --graph also
-times the step captured once as a CUDA graph and replayed.
+times the step captured once as a CUDA graph and replayed. --prefill N_Q
+switches to the chunked-prefill step (append an N_Q-token chunk to every
+sequence, then causal attention of its queries over the compressed context)
+and its own metric, query tokens/s, with a tensor-core roofline.
 Under torchrun every rank runs an independent replica (no data-path
 collective): value = all ranks' KV tokens / the slowest rank's time.
 """
@@ -522,6 +525,260 @@ def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512):
                           "sample": "%d rows, one thread per row, %.1f s" % (len(rows), dt_all)}}
 
 
+PREFILL_METRIC = "chunked-prefill attention over the compressed KV cache: query tokens/s"
+PREFILL_UNIT = "query tokens/s"
+# Useful tensor work per (query row, visible key): q.k and p.v, 128
+# multiply-adds each.
+FLOPS_PER_PAIR = 4 * 128
+# Kernel launches of one prefill step: dq_append_kv of the chunk (encode +
+# drift kernels) and dq_prefill_attention (one kernel).
+PREFILL_LAUNCHES_PER_STEP = 3
+
+
+def chunk_pairs(B, Hq, q_start, n_q):
+    """(query row, visible key) pairs of a causal chunk: sum over its query
+    tokens i of (q_start + i + 1) keys, for every sequence and query head."""
+    return B * Hq * (n_q * (q_start + 1) + n_q * (n_q - 1) // 2)
+
+
+def run_prefill(args):
+    """One step = append an n_q-token chunk to every sequence (dq_append_kv)
+    + chunked-prefill attention of its n_q queries over the context, the
+    chunk itself included (dq_prefill_attention); the chunk is the last
+    n_q positions of the workload's context."""
+    import numpy as np
+    import torch
+
+    import decode_attention_dq_b200 as dq
+    from decode_attention_dq_b200 import synth
+
+    ws, rank, local = dist_setup(args)
+    dist = None
+    if ws > 1:
+        import torch.distributed as dist
+    w = replica_workload(synth.WORKLOADS[args.workload], rank)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
+    ck, cv = tab.k.container_bytes, tab.v.container_bytes
+    T, n_q = w.T, args.prefill
+    q_start = T - n_q
+    T_cap = (T + 31) // 32 * 32
+    kc = torch.zeros((w.B, w.Hkv, T_cap, ck), dtype=torch.uint8, device=dev)
+    vc = torch.zeros((w.B, w.Hkv, T_cap, cv), dtype=torch.uint8, device=dev)
+    synth.prefill_cache(tab, w, kc, vc, q_start, threads=args.threads)
+    rows = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    # The chunk's tokens: a seeded stream of their own (step index 1 of the
+    # generator), and its queries.
+    host_k = torch.from_numpy(synth.kv_block(w, "k", rows, n=n_q, step=1, threads=args.threads)
+                              ).to(w.torch_dtype).view(w.B, w.Hkv, n_q, 128).pin_memory()
+    host_v = torch.from_numpy(synth.kv_block(w, "v", rows, n=n_q, step=1, threads=args.threads)
+                              ).to(w.torch_dtype).view(w.B, w.Hkv, n_q, 128).pin_memory()
+    host_q = torch.from_numpy(synth.q_chunk(w, n_q)).to(w.torch_dtype).pin_memory()
+    dk, dv, dqq = host_k.to(dev), host_v.to(dev), host_q.to(dev)
+    out = torch.empty((w.B, n_q, w.Hq, 128), dtype=torch.float32, device=dev)
+    out_host = torch.empty_like(out, device="cpu").pin_memory()
+    start = torch.full((w.B,), q_start, dtype=torch.int32, device=dev)
+    app_ws = torch.empty(max(16, dq.dq_append_workspace_bytes(tab, w.B, w.Hkv, n_q)), dtype=torch.uint8,
+                         device=dev)
+    stats = dq.new_stats(dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        dq.dq_append_kv(tab, dk, dv, start, kc, vc, stats=stats, workspace=app_ws)
+        if ev is not None:
+            ev[0].record(stream)
+        dq.dq_prefill_attention(tab, dqq, kc, vc, start, out, stats=stats)
+        if ev is not None:
+            ev[1].record(stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    attn_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    elapsed_ms, attn_ms = max_over_ranks([elapsed_ms, attn_ms], dist, dev)
+    ms_per_step = elapsed_ms / args.steps
+    qtok = w.B * n_q
+    value = whole_job_rate(qtok, ws, ms_per_step)
+
+    def step_e2e():
+        dk.copy_(host_k, non_blocking=True)
+        dv.copy_(host_v, non_blocking=True)
+        dqq.copy_(host_q, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+
+    step_e2e()
+    torch.cuda.synchronize()
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        step_e2e()
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks([f0.elapsed_time(f1)], dist, dev)[0]
+    st = dq.stats_dict(stats)
+    result = None
+    if rank == 0:
+        peaks, src = measured_peaks()
+        flops = chunk_pairs(w.B, w.Hq, q_start, n_q) * FLOPS_PER_PAIR
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        peak = float(peaks.get("bf16_tflops", 1590.0))
+        peak_sus = float(peaks.get("bf16_tflops_sustained", peak))
+        comp_bytes = w.B * w.Hkv * T * (ck + cv)
+        io_bytes = 2 * dqq.numel() * dqq.element_size() + out.numel() * out.element_size()
+        h2d = (host_k.numel() + host_v.numel() + host_q.numel()) * host_k.element_size()
+        result = {
+            "metric": PREFILL_METRIC, "value": value, "unit": PREFILL_UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16x2 tensor / f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
+                       "context": T, "chunk": n_q, "q_start": q_start, "input_dtype": w.dtype,
+                       "k_container_bytes": ck, "v_container_bytes": cv,
+                       "l2": "inputs larger than L2 (%.0f MB of containers, %.0f MB of queries and outputs)"
+                             % (comp_bytes / 1e6, io_bytes / 1e6),
+                       "parallelism": "replicas x%d" % ws},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "frac_of_sustained": achieved / peak_sus,
+                         "traffic": None,
+                         "useful_flops": flops, "flops_convention": "4 x 128 per (query row, visible key)",
+                         "kernel": "prefill_kernel (dq_prefill_attention)", "kernel_ms": attn_ms,
+                         "peak_source": "%s bf16 dense GEMM (fp16 runs at the same rate)" % src},
+            "e2e": {"value": whole_job_rate(qtok, ws, e2e_ms / args.steps), "unit": PREFILL_UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+            "gpu_launches": PREFILL_LAUNCHES_PER_STEP * args.steps,
+            "clocks": clk,
+            "integrity_errors": st["integrity_errors"], "wait_timeouts": st["wait_timeouts"],
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = prefill_cpu_baseline(w, n_q, seconds=args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def oracle_prefill_row(w, tabs, bh, n_q, ctx):
+    """The oracle's prefill step for one (sequence, KV head) row: encode the
+    chunk's K and V, then fp64 causal attention of the chunk's queries (the G
+    heads of this KV head) over context + chunk."""
+    import numpy as np
+
+    from decode_attention_dq_b200 import synth
+    from oracle import oracle as o
+    b, h = bh
+    kc, vc = ctx
+    T = kc.shape[0]
+    G = w.Hq // w.Hkv
+    k_new = synth.kv_row(w, "k", b, h, n=n_q, step=1)
+    v_new = synth.kv_row(w, "v", b, h, n=n_q, step=1)
+    hh = np.full(n_q, h, np.int32)
+    kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, hh)
+    vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, hh)
+    kfull = np.zeros((1, w.Hkv, T, kc.shape[1]), np.uint8)
+    vfull = np.zeros((1, w.Hkv, T, vc.shape[1]), np.uint8)
+    kfull[0, h, :T - n_q] = kc[:T - n_q]
+    vfull[0, h, :T - n_q] = vc[:T - n_q]
+    kfull[0, h, T - n_q:] = kk
+    vfull[0, h, T - n_q:] = vv
+    q = np.zeros((1, n_q, w.Hq, 128))
+    q[0, :, h * G:(h + 1) * G] = np.stack([synth.q_rows(w, b, i)[h * G:(h + 1) * G] for i in range(n_q)])
+    o.attention_prefill_fp64(tabs, q, kfull, vfull, [T - n_q], rows=[(0, h)])
+
+
+def prefill_contexts(w, tabs, n_rows, seconds):
+    """Oracle containers of the context of sampled rows (setup, untimed)."""
+    import numpy as np
+
+    from decode_attention_dq_b200 import synth
+    from oracle import oracle as o
+    rows = [(s % w.B, (s * 3) % w.Hkv) for s in range(n_rows)]
+    out = []
+    t0 = time.time()
+    for b, h in rows:
+        K = synth.kv_row(w, "k", b, h)
+        V = synth.kv_row(w, "v", b, h)
+        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
+        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+        out.append(((b, h), (kc, vc)))
+        if time.time() - t0 > seconds:
+            break
+    return out
+
+
+def prefill_cpu_baseline(w, n_q, seconds=12.0):
+    """The oracle's prefill step on one host thread (BLAS limited to one
+    thread), on a bounded sample of (sequence, KV head) rows."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import oracle as o
+    tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
+                    v_container_bytes=o.container_bytes(w.v_bits))
+    with threadpool_limits(limits=1):
+        ctx = prefill_contexts(w, tabs, 16, seconds / 2)
+        done = 0
+        t0 = time.time()
+        for bh, cc in ctx:
+            oracle_prefill_row(w, tabs, bh, n_q, cc)
+            done += 1
+            if time.time() - t0 > seconds / 2:
+                break
+        dt = time.time() - t0
+    return {"value": done * n_q / w.Hkv / dt, "unit": PREFILL_UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d (sequence, KV head) rows of %s: encode a %d-token chunk + fp64 causal attention of "
+                      "its queries over %d tokens, one thread, %.1f s" % (done, w.name, n_q, w.T, dt)}
+
+
+def run_reference_prefill(args, w):
+    """Reference arm of the prefill mode: the oracle's prefill step, one
+    (sequence, KV head) row per step, one thread."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import oracle as o
+    n_q = args.prefill
+    tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
+                    v_container_bytes=o.container_bytes(w.v_bits))
+    with threadpool_limits(limits=1):
+        ctx = prefill_contexts(w, tabs, args.warmup + args.steps, 1e9)
+        for i in range(args.warmup):
+            oracle_prefill_row(w, tabs, ctx[i][0], n_q, ctx[i][1])
+        t0 = time.time()
+        for i in range(args.warmup, args.warmup + args.steps):
+            oracle_prefill_row(w, tabs, ctx[i][0], n_q, ctx[i][1])
+        dt = time.time() - t0
+    value = args.steps * n_q / w.Hkv / dt
+    sample = ("per step: one (sequence, KV head) row of %s, encode a %d-token chunk + fp64 causal attention "
+              "over %d tokens, single thread" % (w.name, n_q, w.T))
+    return {"impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": PREFILL_UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
+                       "context": w.T, "chunk": n_q, "sample_per_step": "one (sequence, KV head) row"},
+            "cpu_baseline": {"value": value, "unit": PREFILL_UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def run_reference(args):
     """Reference arm: the CPU oracle on the host cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -529,6 +786,8 @@ def run_reference(args):
         return None
     from decode_attention_dq_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.prefill:
+        return run_reference_prefill(args, w)
     import numpy as np
     from oracle import oracle as o
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
@@ -576,10 +835,15 @@ def main():
     ap.add_argument("--paged", action="store_true", help="page pools and a shuffled page table")
     ap.add_argument("--layers", type=int, default=1, help="layers of the decode loop (one cache each)")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as a CUDA graph")
+    ap.add_argument("--prefill", type=int, default=0, metavar="N_Q",
+                    help="chunked-prefill mode: append an N_Q-token chunk and attend its queries causally")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    res = run_reference(args) if args.impl == "reference" else run_dq(args)
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_prefill(args) if args.prefill else run_dq(args)
     if res is not None:
         print(json.dumps(res), flush=True)
 
