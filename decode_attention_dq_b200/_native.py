@@ -25,7 +25,7 @@ EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_st
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",
             "dq_design_stream", "dq_decode_attention_noalloc", "dq_append_workspace_bytes",
             "dq_append_kv_ws", "dq_append_kv_paged", "dq_decode_attention_paged",
-            "dq_prefill_attention", "dq_prefill_attention_paged")
+            "dq_prefill_attention", "dq_prefill_attention_paged", "dq_prefill_workspace_bytes")
 
 
 class DqConfig(C.Structure):
@@ -87,10 +87,13 @@ def load():
     lib.dq_decode_symbols.argtypes = [vp, vp, C.c_int, i64, vp, vp, vp, vp, vp]
     lib.dq_decode_attention_noalloc.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int,
                                                 C.c_int, i64, i64, C.c_float, vp, C.c_int, vp, vp]
+    lib.dq_prefill_workspace_bytes.argtypes = [vp, C.c_int, C.c_int, i64]
+    lib.dq_prefill_workspace_bytes.restype = C.c_size_t
     lib.dq_prefill_attention.argtypes = [vp, vp, C.c_int, vp, vp, vp, C.c_int, C.c_int, C.c_int,
-                                         C.c_int, i64, C.c_float, vp, C.c_int, vp, vp]
+                                         C.c_int, i64, C.c_float, vp, C.c_int, vp, C.c_size_t, vp, vp]
     lib.dq_prefill_attention_paged.argtypes = [vp, vp, C.c_int, vp, vp, i64, vp, i64, vp, C.c_int,
-                                               C.c_int, C.c_int, C.c_int, C.c_float, vp, C.c_int, vp, vp]
+                                               C.c_int, C.c_int, C.c_int, C.c_float, vp, C.c_int, vp,
+                                               C.c_size_t, vp, vp]
     lib.dq_error_string.argtypes = [C.c_int]
     lib.dq_error_string.restype = C.c_char_p
     lib.dq_last_cuda_error.argtypes = []
@@ -292,27 +295,43 @@ def dq_decode_attention_noalloc(tab: Tables, q: torch.Tensor, kcache: torch.Tens
         _stream(stream)))
 
 
+def dq_prefill_workspace_bytes(tab: Tables, B: int, Hkv: int, T_cap: int) -> int:
+    """Bytes of the dq_prefill_attention workspace (decoded tiles)."""
+    return int(load().dq_prefill_workspace_bytes(tab.handle, B, Hkv, T_cap))
+
+
+def _prefill_ws(tab, workspace, B, Hkv, T_cap, device):
+    need = dq_prefill_workspace_bytes(tab, B, Hkv, T_cap)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    return workspace
+
+
 def dq_prefill_attention(tab: Tables, q: torch.Tensor, kcache: torch.Tensor, vcache: torch.Tensor,
-                         q_start: torch.Tensor, out: torch.Tensor, sm_scale: float | None = None,
-                         stats: torch.Tensor | None = None, stream=None) -> None:
+                         q_start: torch.Tensor, out: torch.Tensor, workspace: torch.Tensor | None = None,
+                         sm_scale: float | None = None, stats: torch.Tensor | None = None,
+                         stream=None) -> None:
     """Chunked-prefill attention: q [B, n_q, Hq, 128] (query token i of
     sequence b at position q_start[b] + i, causal over the cache); caches
-    uint8 [B, Hkv, T_cap, C]; q_start int32 [B]; out [B, n_q, Hq, 128]."""
+    uint8 [B, Hkv, T_cap, C]; q_start int32 [B]; out [B, n_q, Hq, 128];
+    workspace uint8 of dq_prefill_workspace_bytes (allocated if None)."""
     B, n_q, Hq, d = q.shape
     Hkv, T_cap = kcache.shape[1], kcache.shape[2]
     assert d == 128 and q.is_contiguous() and out.is_contiguous() and q_start.dtype == torch.int32
     assert out.shape == q.shape
     if sm_scale is None:
         sm_scale = 128 ** -0.5
+    workspace = _prefill_ws(tab, workspace, B, Hkv, T_cap, q.device)
     _check("dq_prefill_attention", load().dq_prefill_attention(
         tab.handle, _ptr(q), _dtype_code(q), _ptr(kcache), _ptr(vcache), _ptr(q_start), B, n_q, Hq,
-        Hkv, T_cap, float(sm_scale), _ptr(out), _dtype_code(out), _ptr(stats), _stream(stream)))
+        Hkv, T_cap, float(sm_scale), _ptr(out), _dtype_code(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(stats), _stream(stream)))
 
 
 def dq_prefill_attention_paged(tab: Tables, q: torch.Tensor, kpool: torch.Tensor, vpool: torch.Tensor,
                                page_table: torch.Tensor, q_start: torch.Tensor, out: torch.Tensor,
-                               sm_scale: float | None = None, stats: torch.Tensor | None = None,
-                               stream=None) -> None:
+                               workspace: torch.Tensor | None = None, sm_scale: float | None = None,
+                               stats: torch.Tensor | None = None, stream=None) -> None:
     """Chunked-prefill attention over page pools (see dq_prefill_attention)."""
     B, n_q, Hq, d = q.shape
     Hkv = kpool.shape[1]
@@ -320,10 +339,12 @@ def dq_prefill_attention_paged(tab: Tables, q: torch.Tensor, kpool: torch.Tensor
     assert page_table.dtype == torch.int32 and page_table.is_contiguous() and out.shape == q.shape
     if sm_scale is None:
         sm_scale = 128 ** -0.5
+    workspace = _prefill_ws(tab, workspace, B, Hkv, 32 * page_table.shape[1], q.device)
     _check("dq_prefill_attention_paged", load().dq_prefill_attention_paged(
         tab.handle, _ptr(q), _dtype_code(q), _ptr(kpool), _ptr(vpool), kpool.shape[0],
         _ptr(page_table), page_table.shape[1], _ptr(q_start), B, n_q, Hq, Hkv, float(sm_scale),
-        _ptr(out), _dtype_code(out), _ptr(stats), _stream(stream)))
+        _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(stats), _stream(stream)))
 
 
 def dq_decode_symbols(tab: Tables, cache: torch.Tensor, kind: int, syms: torch.Tensor,

@@ -520,10 +520,11 @@ int dq_decode_attention_paged(const dq_tables *t, const void *q, int q_dtype, co
 
 static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
                         const uint8_t *d_vcache, const int32_t *d_q_start, int B, int n_q, int Hq, int Hkv,
-                        int64_t T_cap, float sm_scale, void *out, int out_dtype, dq_stats *d_stats, void *stream,
-                        const int32_t *page_table, int64_t max_pages, int64_t num_pages) {
+                        int64_t T_cap, float sm_scale, void *out, int out_dtype, void *d_workspace,
+                        size_t ws_bytes, dq_stats *d_stats, void *stream, const int32_t *page_table,
+                        int64_t max_pages, int64_t num_pages) {
   try {
-    if (!t || !q || !d_kcache || !d_vcache || !d_q_start || !out) return DQ_ERR_NULL;
+    if (!t || !q || !d_kcache || !d_vcache || !d_q_start || !out || !d_workspace) return DQ_ERR_NULL;
     if ((q_dtype != DQ_F32 && q_dtype != DQ_BF16) || (out_dtype != DQ_F32 && out_dtype != DQ_BF16))
       return DQ_ERR_DTYPE;
     if (B < 0 || n_q < 0 || Hkv != t->cfg.n_kv_heads || Hq < Hkv || Hq % Hkv) return DQ_ERR_SHAPE;
@@ -531,15 +532,22 @@ static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const ui
     if (G != 1 && G != 2 && G != 4 && G != 8) return DQ_ERR_SHAPE;
     if (T_cap < 0) return DQ_ERR_SHAPE;
     if (T_cap % 32 || !aligned(d_kcache, 16) || !aligned(d_vcache, 16) || !aligned(q, 4) || !aligned(out, 4) ||
-        !aligned(d_q_start, 4))
+        !aligned(d_q_start, 4) || !aligned(d_workspace, 16))
       return DQ_ERR_ALIGN;
     if (!std::isfinite(sm_scale)) return DQ_ERR_SHAPE;
-    const int nd = dqi::prefill_decoder_warps(t->k.container_bytes, t->v.container_bytes);
-    if (nd <= 0) return DQ_ERR_SHAPE;
+    if (!dqi::prefill_supported(t->k.container_bytes, t->v.container_bytes)) return DQ_ERR_SHAPE;
     if (dqi::prefill_grid(B, Hkv, G, n_q) > 0x7FFFFFFF) return DQ_ERR_SHAPE;
+    if (ws_bytes < dqi::prefill_workspace_bytes(B, Hkv, T_cap)) return DQ_ERR_WORKSPACE;
     int rc = check_device(t);
     if (rc != DQ_OK) return rc;
-    if (B == 0 || n_q == 0) return DQ_OK;
+    if (B == 0 || n_q == 0 || T_cap == 0) {
+      if (B > 0 && n_q > 0) {  // no cache: every row is outside it, out = 0
+        const size_t n = static_cast<size_t>(B) * n_q * Hq * dqi::kD * (out_dtype == DQ_F32 ? 4 : 2);
+        cudaError_t e = cudaMemsetAsync(out, 0, n, static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e);
+      }
+      return DQ_OK;
+    }
     dqi::PrefillArgs a{};
     a.tabs = t->d_tabs;
     a.sign_bits = t->d_sign_bits;
@@ -561,7 +569,10 @@ static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const ui
     a.cv = t->v.container_bytes;
     a.two_k = has_small_freq(t->k);
     a.two_v = has_small_freq(t->v);
-    a.nd = nd;
+    a.tiles = static_cast<uint8_t *>(d_workspace);
+    a.nslots = dqi::prefill_ring_slots();
+    const int64_t rows = static_cast<int64_t>(B) * Hkv * (T_cap / 32);
+    a.tile_grid = static_cast<int>(std::min<int64_t>(t->sm_count, (rows + 19) / 20));
     a.stats = d_stats;
     a.page_table = page_table;
     a.max_pages = max_pages;
@@ -573,23 +584,30 @@ static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const ui
   }
 }
 
+size_t dq_prefill_workspace_bytes(const dq_tables *t, int B, int Hkv, int64_t T_cap) {
+  if (!t || B < 0 || Hkv < 1 || T_cap < 0 || T_cap % 32) return 0;
+  return std::max<size_t>(16, dqi::prefill_workspace_bytes(B, Hkv, T_cap));
+}
+
 int dq_prefill_attention(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kcache,
                          const uint8_t *d_vcache, const int32_t *d_q_start, int B, int n_q, int Hq, int Hkv,
-                         int64_t T_cap, float sm_scale, void *out, int out_dtype, dq_stats *d_stats, void *stream) {
+                         int64_t T_cap, float sm_scale, void *out, int out_dtype, void *d_workspace,
+                         size_t ws_bytes, dq_stats *d_stats, void *stream) {
   return prefill_core(t, q, q_dtype, d_kcache, d_vcache, d_q_start, B, n_q, Hq, Hkv, T_cap, sm_scale, out,
-                      out_dtype, d_stats, stream, nullptr, 0, 0);
+                      out_dtype, d_workspace, ws_bytes, d_stats, stream, nullptr, 0, 0);
 }
 
 int dq_prefill_attention_paged(const dq_tables *t, const void *q, int q_dtype, const uint8_t *d_kpool,
                                const uint8_t *d_vpool, int64_t num_pages, const int32_t *d_page_table,
                                int64_t max_pages, const int32_t *d_q_start, int B, int n_q, int Hq, int Hkv,
-                               float sm_scale, void *out, int out_dtype, dq_stats *d_stats, void *stream) {
+                               float sm_scale, void *out, int out_dtype, void *d_workspace, size_t ws_bytes,
+                               dq_stats *d_stats, void *stream) {
   if (!d_page_table) return DQ_ERR_NULL;
   if (num_pages < 1 || max_pages < 1 || max_pages > (int64_t(1) << 40) || num_pages > (int64_t(1) << 31))
     return DQ_ERR_SHAPE;
   if (!aligned(d_page_table, 4)) return DQ_ERR_ALIGN;
   return prefill_core(t, q, q_dtype, d_kpool, d_vpool, d_q_start, B, n_q, Hq, Hkv, 32 * max_pages, sm_scale, out,
-                      out_dtype, d_stats, stream, d_page_table, max_pages, num_pages);
+                      out_dtype, d_workspace, ws_bytes, d_stats, stream, d_page_table, max_pages, num_pages);
 }
 
 int dq_decode_symbols(const dq_tables *t, const uint8_t *d_cache, int stream_kind,

@@ -143,16 +143,20 @@ struct PrefillArgs {
   int out_dtype;
   int ck, cv;
   bool two_k, two_v;
-  int nd;              // decoder warps per CTA (prefill_decoder_warps)
+  uint8_t *tiles;      // workspace: decoded slots [B][Hkv][T_cap / 32]
+  int nslots;          // ring depth of the attention kernel (prefill_ring_slots)
+  int tile_grid;       // CTAs of the tile kernel
   dq_stats *stats;
   const int32_t *page_table;  // paged caches as in AppendArgs (nullptr: contiguous)
   int64_t max_pages, num_pages;
 };
 int launch_prefill_attention(const PrefillArgs &a, void *stream);
-// Decoder warps per CTA for these container sizes (0 if unsupported).
-int prefill_decoder_warps(int ck, int cv);
-// CTAs of one call: B * Hkv * ceil(n_q / (128 / G)).
+int prefill_ring_slots();
+// CTAs of the attention kernel: B * Hkv * ceil(n_q / (128 / G)).
 int64_t prefill_grid(int B, int Hkv, int G, int n_q);
+// Bytes of decoded slots for B x Hkv rows of T_cap tokens.
+size_t prefill_workspace_bytes(int B, int Hkv, int64_t T_cap);
+bool prefill_supported(int ck, int cv);
 
 struct SymbolsArgs {
   const DevStream *tab;

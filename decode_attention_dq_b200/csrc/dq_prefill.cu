@@ -10,35 +10,41 @@
 // and values. Query token i of sequence b sits at position q_start[b] + i and
 // attends causally to cache positions 0 .. q_start[b] + i.
 //
-// One CTA per (b, KV head h, block of 128 query rows); a row is one query
-// token of the chunk with one of the G query heads of h (rows are token-major:
-// row r = token r / G, head r % G). Warp roles:
-//   warps 0-3  softmax: thread r owns row r, which is lane r of tensor memory.
-//              It rotates its query (q~ = H D q, fp32, times a power of two),
-//              splits it into fp16 hi + lo and stores both into tensor memory
-//              (the A operand of the score MMA); per 32-token group it reads
-//              its 32 scores, applies the key norms, the scale and the causal
-//              mask, runs the online softmax, rescales its row of O in tensor
-//              memory when the running maximum grows, and stores the weights
-//              w = p ||v|| as fp16 hi + lo into tensor memory (the A operand of
-//              the P.V MMA). At the end it applies 1 / (128 l kappa_V), the
-//              inverse rotation D H and writes the output row.
-//   warp 4     owns the tensor memory; one lane issues the MMAs:
-//              S_j = Q~hi K_j^T + Q~lo K_j^T        (M 128, N 32, K 128)
-//              O  += W_j,hi V_j + W_j,lo V_j         (M 128, N 128, K 32)
-//              both of kind f16 with fp32 accumulation, A from tensor memory
-//              and B from shared memory (no swizzle, 8 x 16-byte core
-//              matrices).
-//   warps 5..  decoders: decoder d takes groups d, d + nd, ... of 32 tokens,
-//              stages the group's byte-interleaved K and V containers with
-//              cp.async (one group ahead), rANS-decodes them one lane per
-//              token (K and V chains interleaved) and writes fp16 levels into
-//              its ring slot: kappa_K y for K (kappa_K minimises the
-//              frequency-weighted level error) and kappa_V y for V, with the
-//              tokens' norms beside them.
-// Hand-offs use mbarriers; every wait is bounded, and a CTA that gives up
-// counts the event in wait_timeouts, skips the rest of its work and still
-// frees its tensor memory after its MMAs have drained.
+// Two kernels.
+//
+// prefill_tiles_kernel decodes every 32-token block of K and V that the chunk
+// attends to, once per (b, KV head), into the workspace: one slot per block
+// holds a K tile and a V tile (32 tokens x 128 coordinates, fp16 levels in the
+// tensor cores' no-swizzle core-matrix layout: token t, coordinate i at byte
+// (t/8)*128 + (i/8)*512 + (t%8)*16 + (i%8)*2) and the tokens' K and V norms.
+// K levels are kappa_K y with kappa_K chosen to minimise the frequency-
+// weighted level error, V levels kappa_V y as in decode attention. Every warp
+// of a persistent grid takes blocks in a strided order; a lane decodes one
+// token's K and V (two interleaved rANS chains) from the byte-interleaved
+// containers staged in shared memory with cp.async, one block ahead.
+//
+// prefill_kernel: one CTA per (b, KV head h, block of 128 query rows); a row is
+// one query token of the chunk with one of the G query heads of h (row r =
+// token r / G, head r % G). The CTAs of one (b, h) are launched together (the
+// longest causal ranges first) so that its tiles are read from L2. Warps:
+//   0-3  softmax: thread r owns row r = lane r of tensor memory. It rotates
+//        its query (q~ = H D q in fp32, times a power of two), splits it into
+//        fp16 hi + lo and stores both into tensor memory; per block j it reads
+//        its 32 scores, applies the key norms, the scale and the causal mask,
+//        runs the online softmax, rescales its row of O in tensor memory when
+//        the running maximum grows, and stores the weights w = p ||v|| as fp16
+//        hi + lo into tensor memory. At the end it applies 1 / (128 l kappa_V),
+//        the inverse rotation D H and writes the output row.
+//   4    owns the tensor memory; one lane issues the MMAs
+//          S_j = q~hi K_j^T + q~lo K_j^T        (M 128, N 32, K 128)
+//          O  += W_j,hi V_j + W_j,lo V_j         (M 128, N 128, K 32)
+//        kind::f16 with fp32 accumulators, A from tensor memory, B (K tile
+//        K-major, V tile MN-major) from shared memory.
+//   5    one lane streams the slots into a ring in shared memory with bulk
+//        copies counted on mbarriers.
+// Every wait is bounded; a CTA that gives up counts it in wait_timeouts,
+// skips the rest of its work and still frees its tensor memory after its MMAs
+// and copies have drained.
 #include <type_traits>
 
 #include "dq_device.cuh"
@@ -47,12 +53,13 @@ namespace dqi {
 namespace {
 
 constexpr int kRows = 128;          // query rows per CTA (the MMA's M)
-constexpr int kGrp = 32;            // tokens per cache block (one per decoder lane)
+constexpr int kGrp = 32;            // tokens per cache block
 constexpr int kSoftWarps = 4;       // warps 0..3
 constexpr int kMmaWarp = 4;         // warp 4
-constexpr int kFirstDec = 5;        // warps 5..5+nd-1
-constexpr int kMaxDec = 7;
-constexpr int kMaxThreads = 32 * (kFirstDec + kMaxDec);
+constexpr int kLoadWarp = 5;        // warp 5
+constexpr int kAttnThreads = 32 * 6;
+constexpr int kMaxSlots = 12;       // ring depth of prefill_kernel
+constexpr int kTileWarps = 20;      // warps per CTA of prefill_tiles_kernel
 constexpr uint32_t kTmemCols = 512;
 // Tensor-memory columns (32-bit each; 128 lanes = rows).
 constexpr uint32_t kColO = 0;       // O: 128 fp32 columns
@@ -60,43 +67,61 @@ constexpr uint32_t kColS = 128;     // S: 2 buffers x 32 fp32 columns
 constexpr uint32_t kColP = 192;     // W: 2 buffers x (16 hi + 16 lo) columns of packed fp16 pairs
 constexpr uint32_t kColQh = 256;    // q~ hi: 64 columns of packed fp16 pairs
 constexpr uint32_t kColQl = 320;    // q~ lo: 64 columns
-constexpr int kTileBytes = kGrp * kD * 2;   // one fp16 tile: 32 tokens x 128 coordinates
+constexpr int kTileBytes = kGrp * kD * 2;                  // one fp16 tile: 32 tokens x 128 coordinates
 constexpr int kSlotBytes = 2 * kTileBytes + 2 * kGrp * 4;  // K tile, V tile, K norms, V norms
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kSpin = 1u << 24;  // bound on each mbarrier wait loop
-// Barrier slots.
-constexpr int kBarFull = 0, kBarEmpty = 8, kBarSFull = 16, kBarSFree = 18, kBarPFull = 20, kBarPvDone = 22,
-              kBarQFull = 24, kBarDrain = 25, kNumBars = 32;
+// Barrier slots of prefill_kernel.
+constexpr int kBarFull = 0, kBarEmpty = kMaxSlots, kBarSFull = 2 * kMaxSlots, kBarSFree = kBarSFull + 2,
+              kBarPFull = kBarSFull + 4, kBarPvDone = kBarSFull + 6, kBarQFull = kBarSFull + 8,
+              kBarDrain = kBarSFull + 9, kNumBars = kBarSFull + 10;
+static_assert(kSlotBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-struct PrefillSmem {
-  size_t lut_k, lut_v, lev, bars, misc, ring, stage;
-  size_t kslot, vslot, stage_bytes;  // per decoder warp: K slots 0, 1 then V slots 0, 1
-  size_t total;
+// Shared memory of prefill_tiles_kernel: decode tables, then per warp two
+// staging slots for K and two for V.
+struct TilesSmem {
+  size_t lut_k, lut_v, lev, stage, kslot, vslot, stage_bytes, total;
 };
 
-__host__ __device__ inline PrefillSmem prefill_smem_layout(int ck, int cv, int nd) {
-  PrefillSmem s;
+__host__ __device__ inline TilesSmem tiles_smem_layout(int ck, int cv) {
+  TilesSmem s;
   s.lut_k = 0;
   s.lut_v = s.lut_k + kM * 4;
-  s.lev = s.lut_v + kM * 4;                   // [0..7] K score levels, [8..15] V tile levels (fp16 bits)
-  s.bars = s.lev + 2 * kMaxLevels * 4;
-  s.misc = s.bars + kNumBars * 8;             // tensor-memory base, abort flag
-  s.ring = align_up(s.misc + 16, 128);
+  s.lev = s.lut_v + kM * 4;  // [0..7] K score levels, [8..15] V tile levels (fp16 bits)
+  s.stage = align_up(s.lev + 2 * kMaxLevels * 4, 128);
   s.kslot = align_up(static_cast<size_t>(kGrp) * ck, 16);
   s.vslot = align_up(static_cast<size_t>(kGrp) * cv, 16);
   s.stage_bytes = 2 * s.kslot + 2 * s.vslot;
-  s.stage = s.ring + static_cast<size_t>(nd) * kSlotBytes;
-  const size_t end = s.stage + static_cast<size_t>(nd) * s.stage_bytes;
+  const size_t end = s.stage + static_cast<size_t>(kTileWarps) * s.stage_bytes;
   // A corrupt container moves its decoder's cursor by at most 2 bytes per
   // symbol (byte 5 + 2 * 128 at most), 32 bytes apart in the interleaved
   // layout: reads from the last V slot stay inside the allocation.
   const size_t reach = end - s.vslot + static_cast<size_t>(kGrp) * (kHeaderBytes + 2 * kD + 1);
   s.total = (reach > end ? align_up(reach, 16) : end) + 256;
-  // At least 116 KB so that one CTA holds an SM (and its tensor memory).
-  if (s.total < 116 * 1024) s.total = 116 * 1024;
   return s;
+}
+
+// Shared memory of prefill_kernel: barriers, tensor-memory base and abort
+// flag, then the ring of slots.
+struct AttnSmem {
+  size_t bars, misc, ring, total;
+};
+
+__host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
+  AttnSmem s;
+  s.bars = 0;
+  s.misc = s.bars + kNumBars * 8;
+  s.ring = align_up(s.misc + 16, 128);
+  s.total = s.ring + static_cast<size_t>(nslots) * kSlotBytes;
+  return s;
+}
+
+// Last attended position of sequence b (-1: none) and its 32-token blocks.
+__host__ __device__ __forceinline__ int64_t last_position(int64_t qs, int n_q, int64_t T_cap) {
+  if (qs > T_cap - 1 || qs + n_q - 1 < 0) return -1;
+  return qs + n_q - 1 < T_cap - 1 ? qs + n_q - 1 : T_cap - 1;
 }
 
 // ---- PTX wrappers -------------------------------------------------------
@@ -135,6 +160,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   return false;
 }
 
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("{\n.reg .b64 st;\nmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// Bulk copy (no tensor map, no multicast) of `bytes` (a multiple of 16, both
+// addresses 16-byte aligned) from global to this CTA's shared memory;
+// completion is counted on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_commit(uint64_t *bar) {
@@ -194,6 +233,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// 2^x with the hardware approximation (relative error about 2^-22; x <= 0
+// here, results below 2^-126 flush to 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // fp16 hi + lo of a pair of fp32 values, packed (first value in the low half).
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo) {
@@ -259,27 +306,140 @@ __device__ __forceinline__ float norm_of(const uint8_t *cb) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(cb[0] | (cb[kGrp] << 8))));
 }
 
+
 template <bool kTwoK, bool kTwoV>
-__global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillArgs a) {
+__global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int nd = a.nd;
-  const PrefillSmem L = prefill_smem_layout(a.ck, a.cv, nd);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const TilesSmem L = tiles_smem_layout(a.ck, a.cv);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t *lut_k = reinterpret_cast<uint32_t *>(smem + L.lut_k);
   uint32_t *lut_v = reinterpret_cast<uint32_t *>(smem + L.lut_v);
   uint32_t *lev = reinterpret_cast<uint32_t *>(smem + L.lev);
+  {
+    const uint4 *sk = reinterpret_cast<const uint4 *>(a.tabs->k.lut);
+    const uint4 *sv = reinterpret_cast<const uint4 *>(a.tabs->v.lut);
+    uint4 *dk = reinterpret_cast<uint4 *>(lut_k);
+    uint4 *dv = reinterpret_cast<uint4 *>(lut_v);
+    for (int i = threadIdx.x; i < static_cast<int>(kM / 4); i += blockDim.x) {
+      dk[i] = __ldg(sk + i);
+      dv[i] = __ldg(sv + i);
+    }
+    if (threadIdx.x < kMaxLevels) {
+      lev[threadIdx.x] = a.tabs->k.score16[threadIdx.x];
+      lev[kMaxLevels + threadIdx.x] = a.tabs->v.level16[threadIdx.x];
+    }
+  }
+  __syncthreads();
+
+  const int ck = a.ck, cv = a.cv;
+  const int64_t gcap = a.T_cap / kGrp;
+  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * gcap;  // slot s = (b Hkv + h) gcap + j
+  const int64_t W = static_cast<int64_t>(gridDim.x) * kTileWarps;
+  uint8_t *stg = smem + L.stage + static_cast<size_t>(warp) * L.stage_bytes;
+  auto kslot = [&](int s) { return stg + s * L.kslot; };
+  auto vslot = [&](int s) { return stg + 2 * L.kslot + s * L.vslot; };
+  unsigned bad = 0, bad_pages = 0;
+  // Next slot >= s (in steps of W) that the chunk attends to.
+  auto next_valid = [&](int64_t s) -> int64_t {
+    for (; s < total; s += W) {
+      const int64_t bh = s / gcap, j = s % gcap;
+      const int64_t hi = last_position(a.q_start[bh / a.Hkv], a.n_q, a.T_cap);
+      if (hi >= 0 && j <= hi / kGrp) return s;
+    }
+    return total;
+  };
+  auto block_of = [&](int64_t s) -> int64_t {
+    if (a.page_table) {
+      const int64_t bh = s / gcap, j = s % gcap;
+      int64_t pg = a.page_table[(bh / a.Hkv) * a.max_pages + j];
+      if (pg < 0 || pg >= a.num_pages) {
+        ++bad_pages;
+        pg = 0;
+      }
+      return pg * a.Hkv + bh % a.Hkv;
+    }
+    return s;
+  };
+  auto stage = [&](int sl, int64_t s) {
+    const int64_t blk = block_of(s);
+    const uint8_t *ks = a.kcache + blk * kGrp * ck;
+    const uint8_t *vs = a.vcache + blk * kGrp * cv;
+    for (int c = lane; c < (kGrp * ck) >> 4; c += 32) cp_async16(kslot(sl) + c * 16, ks + c * 16);
+    for (int c = lane; c < (kGrp * cv) >> 4; c += 32) cp_async16(vslot(sl) + c * 16, vs + c * 16);
+  };
+
+  int64_t s = next_valid(static_cast<int64_t>(blockIdx.x) * kTileWarps + warp);
+  if (s < total) stage(0, s);
+  cp_async_commit();
+  for (int k = 0; s < total; ++k) {
+    const int sl = k & 1;
+    const int64_t s_next = next_valid(s + W);
+    if (s_next < total) stage(sl ^ 1, s_next);
+    cp_async_commit();
+    cp_async_wait_1();
+    __syncwarp();
+    const uint8_t *kb = kslot(sl) + lane;
+    const uint8_t *vb = vslot(sl) + lane;
+    RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
+    RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
+    uint8_t *dst = a.tiles + s * kSlotBytes;
+#pragma unroll 1
+    for (int i8 = 0; i8 < kD; i8 += 8) {
+      uint32_t hk[8], hv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
+        const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
+        hk[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + ek);
+        hv[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + 4 * kMaxLevels + ev);
+      }
+      // 8 coordinates of this lane's token: 16 bytes at chunk i8 / 8 (512
+      // bytes per chunk of 32 tokens), token offset 16 * lane.
+      const size_t off = static_cast<size_t>((i8 >> 3) * 512 + lane * 16);
+      *reinterpret_cast<uint4 *>(dst + off) =
+          make_uint4(__byte_perm(hk[0], hk[1], 0x5410), __byte_perm(hk[2], hk[3], 0x5410),
+                     __byte_perm(hk[4], hk[5], 0x5410), __byte_perm(hk[6], hk[7], 0x5410));
+      *reinterpret_cast<uint4 *>(dst + kTileBytes + off) =
+          make_uint4(__byte_perm(hv[0], hv[1], 0x5410), __byte_perm(hv[2], hv[3], 0x5410),
+                     __byte_perm(hv[4], hv[5], 0x5410), __byte_perm(hv[6], hv[7], 0x5410));
+    }
+    const int64_t bh = s / gcap;
+    const int64_t hi = last_position(a.q_start[bh / a.Hkv], a.n_q, a.T_cap);
+    const int64_t tok = (s % gcap) * kGrp + lane;
+    // Tokens past the last attended position keep zero norms: their bytes may
+    // be anything, and the softmax multiplies the weights by these norms.
+    float *nrm = reinterpret_cast<float *>(dst + 2 * kTileBytes);
+    nrm[lane] = tok <= hi ? norm_of(kb) : 0.0f;
+    nrm[kGrp + lane] = tok <= hi ? norm_of(vb) : 0.0f;
+    if (tok <= hi) bad += (rk.x != kL) + (rv.x != kL);
+    __syncwarp();  // the staging slot is refilled next iteration
+    s = s_next;
+  }
+  cp_async_wait_0();
+  if (a.stats) {
+    const unsigned b_w = __reduce_add_sync(kFull, bad);
+    const unsigned p_w = __reduce_add_sync(kFull, bad_pages);
+    if (lane == 0 && b_w) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(b_w));
+    if (lane == 0 && p_w) atomicAdd(&a.stats->bad_pages, static_cast<unsigned long long>(p_w));
+  }
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int ns = a.nslots;
+  const AttnSmem L = attn_smem_layout(ns);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + L.misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 4);
   auto slot_base = [&](int d) { return smem + L.ring + static_cast<size_t>(d) * kSlotBytes; };
 
-  // Work item; late query blocks (the longest causal ranges) first.
+  // Work item: the query blocks of one (b, h) are consecutive, latest first.
   const int G = a.G, Mt = kRows / G;
   const int nqb = (a.n_q + Mt - 1) / Mt;
-  const int64_t BH = static_cast<int64_t>(a.B) * a.Hkv;
   const int64_t bid = blockIdx.x;
-  const int qb = nqb - 1 - static_cast<int>(bid / BH);
-  const int64_t bh = bid % BH;
+  const int64_t bh = bid / nqb;
+  const int qb = nqb - 1 - static_cast<int>(bid % nqb);
   const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
   const int64_t qs = a.q_start[b];
   const int i_lo = qb * Mt;
@@ -287,25 +447,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
   const int64_t lo_pos = max(qs + i_lo, int64_t(0));
   const int64_t hi_pos = min(qs + i_hi, a.T_cap - 1);
   const int64_t nG = lo_pos <= hi_pos ? hi_pos / kGrp + 1 : 0;
-  // Tokens whose integrity this CTA reports: those the previous query block
-  // of (b, h) does not reach, so each container is counted once.
-  const int64_t prev_hi = qb == 0 ? int64_t(-1) : min(qs + i_lo - 1, a.T_cap - 1);
+  const int64_t gcap = a.T_cap / kGrp;
 
   // ---- set-up ----
-  {
-    const uint4 *sk = reinterpret_cast<const uint4 *>(a.tabs->k.lut);
-    const uint4 *sv = reinterpret_cast<const uint4 *>(a.tabs->v.lut);
-    uint4 *dk = reinterpret_cast<uint4 *>(lut_k);
-    uint4 *dv = reinterpret_cast<uint4 *>(lut_v);
-    for (int i = tid; i < static_cast<int>(kM / 4); i += blockDim.x) {
-      dk[i] = __ldg(sk + i);
-      dv[i] = __ldg(sv + i);
-    }
-    if (tid < kMaxLevels) {
-      lev[tid] = a.tabs->k.score16[tid];
-      lev[kMaxLevels + tid] = a.tabs->v.level16[tid];
-    }
-  }
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
                  "r"(kTmemCols)
@@ -313,8 +457,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
   if (tid == 0) {
-    for (int d = 0; d < nd; ++d) {
-      mbar_init(bars + kBarFull + d, 32);
+    for (int d = 0; d < ns; ++d) {
+      mbar_init(bars + kBarFull + d, 1);
       mbar_init(bars + kBarEmpty + d, 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -332,8 +476,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tslot;
-  unsigned timeouts = 0, bad = 0, bad_pages = 0, clamped = 0;
-
+  unsigned timeouts = 0, clamped = 0;
   if (warp < kSoftWarps) {
     // ================= softmax warpgroup: thread = row =================
     const int r = tid;
@@ -386,9 +529,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
     bool alive = true;
     for (int64_t j = 0; j < nG && alive; ++j) {
       const int sb = static_cast<int>(j & 1);
-      const int rb = static_cast<int>(j % nd);
+      const int rb = static_cast<int>(j % ns);
       bool ok = mbar_wait(bars + kBarSFull + sb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) &&
-                mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / nd) & 1), abort_flag);
+                mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag);
       if (!__all_sync(kFull, ok)) {
         ++timeouts;
         alive = false;
@@ -401,14 +544,25 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
       mbar_arrive(bars + kBarSFree + sb);
       const float *nk = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes);
       const float *nv = nk + kGrp;
-      const int64_t t0 = j * kGrp;
-      float mx = m_run;
+      // u = S ||k|| (the logit divided by crow > 0); tokens past this row's
+      // position are masked, which only happens on the causal diagonal.
+      float u[32];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const bool valid = row_ok && t0 + t <= pos;
-        s[t] = valid ? s[t] * nk[t] * crow : -INFINITY;
-        mx = fmaxf(mx, s[t]);
+      for (int t = 0; t < 32; ++t) u[t] = s[t] * nk[t];
+      const int64_t rel = pos - j * kGrp;
+      const int lim = (!row_ok || rel < 0) ? -1 : (rel > 31 ? 31 : static_cast<int>(rel));
+      if (!__all_sync(kFull, lim >= 31)) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
       }
+      float mu[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) mu[t] = fmaxf(u[t], u[t + 16]);
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int t = 0; t < w; ++t) mu[t] = fmaxf(mu[t], mu[t + w]);
+      const float mx = mu[0] == -INFINITY ? m_run : fmaxf(m_run, mu[0] * crow);
       float alpha = 1.0f;
       uint32_t whi[16], wlo[16];
       float psum = 0.0f;
@@ -416,15 +570,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
 #pragma unroll
         for (int p = 0; p < 16; ++p) whi[p] = wlo[p] = 0u;
       } else {
-        if (m_run != -INFINITY) alpha = exp2f(m_run - mx);
+        if (m_run != -INFINITY) alpha = ex2(m_run - mx);
+        // p = 2^(logit - mx); w = p ||v|| (norms of tokens past the CTA's
+        // range are 0, so masked tokens give exactly 0).
+        float ps[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int p = 0; p < 16; ++p) {
-          const float p0 = exp2f(s[2 * p] - mx), p1 = exp2f(s[2 * p + 1] - mx);
-          psum += p0 + p1;
-          const float w0 = p0 > 0.0f ? p0 * nv[2 * p] : 0.0f;
-          const float w1 = p1 > 0.0f ? p1 * nv[2 * p + 1] : 0.0f;
-          split_pair(w0, w1, whi[p], wlo[p]);
+          const float p0 = ex2(fmaf(u[2 * p], crow, -mx)), p1 = ex2(fmaf(u[2 * p + 1], crow, -mx));
+          ps[p & 1] += p0 + p1;
+          split_pair(p0 * nv[2 * p], p1 * nv[2 * p + 1], whi[p], wlo[p]);
         }
+        psum = ps[0] + ps[1];
         m_run = mx;
       }
       l_run = l_run * alpha + psum;
@@ -518,7 +674,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
       auto issue_pv = [&](int64_t jj) -> bool {
         if (!mbar_wait(bars + kBarPFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag)) return false;
         tc_fence_after();
-        const uint32_t vt = smem_u32(slot_base(static_cast<int>(jj % nd)) + kTileBytes);
+        const uint32_t vt = smem_u32(slot_base(static_cast<int>(jj % ns)) + kTileBytes);
         const uint32_t wp = tbase + kColP + 32 * static_cast<uint32_t>(jj & 1);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks) {
@@ -527,12 +683,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
           mma_ts(tbase + kColO, wp + 16 + ks * 8, bd, idO, 1u);
         }
         tc_commit(bars + kBarPvDone + (jj & 1));
-        tc_commit(bars + kBarEmpty + static_cast<int>(jj % nd));
+        tc_commit(bars + kBarEmpty + static_cast<int>(jj % ns));
         return true;
       };
       for (int64_t j = 0; j < nG && alive; ++j) {
-        const int rb = static_cast<int>(j % nd);
-        alive = mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / nd) & 1), abort_flag);
+        const int rb = static_cast<int>(j % ns);
+        alive = mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag);
         if (alive && j >= 2)
           alive = mbar_wait(bars + kBarSFree + (j & 1), static_cast<uint32_t>(((j - 2) >> 1) & 1), abort_flag);
         if (!alive) {
@@ -574,85 +730,37 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
         }
       }
     }
-  } else {
-    // ================= decoders =================
-    const int d = warp - kFirstDec;
-    uint8_t *stg = smem + L.stage + static_cast<size_t>(d) * L.stage_bytes;
-    auto kslot = [&](int s) { return stg + s * L.kslot; };
-    auto vslot = [&](int s) { return stg + 2 * L.kslot + s * L.vslot; };
-    uint8_t *kt = slot_base(d);
-    uint8_t *vt = kt + kTileBytes;
-    float *nk = reinterpret_cast<float *>(kt + 2 * kTileBytes);
-    float *nv = nk + kGrp;
-    const int ck = a.ck, cv = a.cv;
-    auto block_of = [&](int64_t j) -> int64_t {
-      if (a.page_table) {
-        int64_t pg = a.page_table[static_cast<int64_t>(b) * a.max_pages + j];
-        if (pg < 0 || pg >= a.num_pages) {
-          ++bad_pages;
-          pg = 0;
-        }
-        return pg * a.Hkv + h;
-      }
-      return bh * (a.T_cap / kGrp) + j;
-    };
-    auto stage = [&](int s, int64_t j) {
-      const int64_t blk = block_of(j);
-      const uint8_t *ks = a.kcache + blk * kGrp * ck;
-      const uint8_t *vs = a.vcache + blk * kGrp * cv;
-      for (int c = lane; c < (kGrp * ck) >> 4; c += 32) cp_async16(kslot(s) + c * 16, ks + c * 16);
-      for (int c = lane; c < (kGrp * cv) >> 4; c += 32) cp_async16(vslot(s) + c * 16, vs + c * 16);
-    };
-    int64_t j = d;
-    if (j < nG) stage(0, j);
-    cp_async_commit();
-    for (int k = 0; j < nG; j += nd, ++k) {
-      const int s = k & 1;
-      if (j + nd < nG) stage(s ^ 1, j + nd);
-      cp_async_commit();
-      cp_async_wait_1();
-      __syncwarp();
-      if (k >= 1) {
-        const bool ok = mbar_wait(bars + kBarEmpty + d, static_cast<uint32_t>((k - 1) & 1), abort_flag);
-        if (!__all_sync(kFull, ok)) {
+  } else if (warp == kLoadWarp) {
+    // ================= slot loader (one lane) =================
+    if (lane == 0 && nG > 0) {
+      const uint8_t *src = a.tiles + static_cast<size_t>(bh * gcap) * kSlotBytes;
+      int64_t issued = 0;
+      for (int64_t j = 0; j < nG; ++j) {
+        const int sl = static_cast<int>(j % ns);
+        if (j >= ns && !mbar_wait(bars + kBarEmpty + sl, static_cast<uint32_t>(((j / ns) - 1) & 1), abort_flag)) {
           ++timeouts;
           break;
         }
+        mbar_arrive_expect_tx(bars + kBarFull + sl, kSlotBytes);
+        bulk_g2s(slot_base(sl), src + static_cast<size_t>(j) * kSlotBytes, kSlotBytes, bars + kBarFull + sl);
+        ++issued;
       }
-      const uint8_t *kb = kslot(s) + lane;
-      const uint8_t *vb = vslot(s) + lane;
-      RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
-      RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
-#pragma unroll 1
-      for (int i8 = 0; i8 < kD; i8 += 8) {
-        uint32_t hk[8], hv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
-          const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
-          hk[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + ek);
-          hv[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + 4 * kMaxLevels + ev);
+      // Drain: the last copies into each slot have landed before the CTA
+      // exits (bounded, whatever the abort flag says).
+      for (int64_t j = issued > ns ? issued - ns : 0; j < issued; ++j) {
+        const uint32_t fa = smem_u32(bars + kBarFull + static_cast<int>(j % ns));
+        const uint32_t par = static_cast<uint32_t>((j / ns) & 1);
+        for (uint32_t it = 0; it < kSpin; ++it) {
+          uint32_t done;
+          asm volatile(
+              "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\nselp.u32 %0, 1, 0, P;\n}\n"
+              : "=r"(done)
+              : "r"(fa), "r"(par)
+              : "memory");
+          if (done) break;
         }
-        // 8 coordinates of this lane's token: 16 bytes at chunk i8 / 8
-        // (512 bytes per chunk of 32 tokens), token offset 16 * lane.
-        const uint32_t off = static_cast<uint32_t>((i8 >> 3) * 512 + lane * 16);
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(smem_u32(kt) + off),
-                     "r"(__byte_perm(hk[0], hk[1], 0x5410)), "r"(__byte_perm(hk[2], hk[3], 0x5410)),
-                     "r"(__byte_perm(hk[4], hk[5], 0x5410)), "r"(__byte_perm(hk[6], hk[7], 0x5410))
-                     : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(smem_u32(vt) + off),
-                     "r"(__byte_perm(hv[0], hv[1], 0x5410)), "r"(__byte_perm(hv[2], hv[3], 0x5410)),
-                     "r"(__byte_perm(hv[4], hv[5], 0x5410)), "r"(__byte_perm(hv[6], hv[7], 0x5410))
-                     : "memory");
       }
-      nk[lane] = norm_of(kb);
-      nv[lane] = norm_of(vb);
-      const int64_t tok = j * kGrp + lane;
-      if (tok > prev_hi && tok <= hi_pos) bad += (rk.x != kL) + (rv.x != kL);
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      mbar_arrive(bars + kBarFull + d);
     }
-    cp_async_wait_0();
   }
 
   tc_fence_before();
@@ -663,37 +771,30 @@ __global__ void __launch_bounds__(kMaxThreads, 1) prefill_kernel(const PrefillAr
   }
   if (a.stats) {
     const unsigned t_w = __reduce_add_sync(kFull, timeouts);
-    const unsigned b_w = __reduce_add_sync(kFull, bad);
-    const unsigned p_w = __reduce_add_sync(kFull, bad_pages);
     const unsigned c_w = __reduce_add_sync(kFull, clamped);
     if (lane == 0) {
       if (t_w) atomicAdd(&a.stats->wait_timeouts, static_cast<unsigned long long>(t_w));
-      if (b_w) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(b_w));
-      if (p_w) atomicAdd(&a.stats->bad_pages, static_cast<unsigned long long>(p_w));
       if (c_w) atomicAdd(&a.stats->clamped_lengths, static_cast<unsigned long long>(c_w));
     }
   }
 }
 
 template <bool kTwoK, bool kTwoV>
-int launch_prefill_t(const PrefillArgs &a, int64_t grid, cudaStream_t st) {
-  const PrefillSmem L = prefill_smem_layout(a.ck, a.cv, a.nd);
-  auto kern = prefill_kernel<kTwoK, kTwoV>;
+int launch_tiles_t(const PrefillArgs &a, cudaStream_t st) {
+  const TilesSmem L = tiles_smem_layout(a.ck, a.cv);
+  auto kern = prefill_tiles_kernel<kTwoK, kTwoV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
   if (e != cudaSuccess) return static_cast<int>(e);
-  kern<<<static_cast<unsigned>(grid), 32 * (kFirstDec + a.nd), L.total, st>>>(a);
+  kern<<<a.tile_grid, kTileWarps * 32, L.total, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace
 
-int prefill_decoder_warps(int ck, int cv) {
-  if (ck < 1 || cv < 1 || ck > kMaxContainer || cv > kMaxContainer) return 0;
-  // At least two decoders: group j + 1 is decoded while P.V of group j still
-  // reads its slot (the MMA loop issues P.V of group j after S of group j + 1).
-  for (int nd = kMaxDec; nd >= 2; --nd)
-    if (prefill_smem_layout(ck, cv, nd).total <= 227 * 1024) return nd;
-  return 0;
+int prefill_ring_slots() {
+  int ns = kMaxSlots;
+  while (ns > 2 && attn_smem_layout(ns).total > 227 * 1024) --ns;
+  return ns;
 }
 
 int64_t prefill_grid(int B, int Hkv, int G, int n_q) {
@@ -701,16 +802,33 @@ int64_t prefill_grid(int B, int Hkv, int G, int n_q) {
   return static_cast<int64_t>(B) * Hkv * ((n_q + Mt - 1) / Mt);
 }
 
+size_t prefill_workspace_bytes(int B, int Hkv, int64_t T_cap) {
+  return static_cast<size_t>(B) * Hkv * static_cast<size_t>(T_cap / kGrp) * kSlotBytes;
+}
+
+bool prefill_supported(int ck, int cv) {
+  return ck >= 1 && cv >= 1 && ck <= kMaxContainer && cv <= kMaxContainer &&
+         tiles_smem_layout(ck, cv).total <= 227 * 1024;
+}
+
 int launch_prefill_attention(const PrefillArgs &a, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (a.nd < 2 || a.nd > kMaxDec || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8))
+  if (a.nslots < 2 || a.nslots > kMaxSlots || a.tile_grid < 1 || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8))
     return static_cast<int>(cudaErrorInvalidValue);
   const int64_t grid = prefill_grid(a.B, a.Hkv, a.G, a.n_q);
   if (grid < 1 || grid > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidValue);
-  if (a.two_k && a.two_v) return launch_prefill_t<true, true>(a, grid, st);
-  if (a.two_k) return launch_prefill_t<true, false>(a, grid, st);
-  if (a.two_v) return launch_prefill_t<false, true>(a, grid, st);
-  return launch_prefill_t<false, false>(a, grid, st);
+  int e;
+  if (a.two_k && a.two_v) e = launch_tiles_t<true, true>(a, st);
+  else if (a.two_k) e = launch_tiles_t<true, false>(a, st);
+  else if (a.two_v) e = launch_tiles_t<false, true>(a, st);
+  else e = launch_tiles_t<false, false>(a, st);
+  if (e) return e;
+  const AttnSmem L = attn_smem_layout(a.nslots);
+  cudaError_t ce =
+      cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  if (ce != cudaSuccess) return static_cast<int>(ce);
+  prefill_kernel<<<static_cast<unsigned>(grid), kAttnThreads, L.total, st>>>(a);
+  return static_cast<int>(cudaGetLastError());
 }
 
 }  // namespace dqi

@@ -303,37 +303,44 @@ int dq_decode_attention_noalloc(const dq_tables *t, const void *q, int q_dtype,
  * sequence b sits at position p = d_q_start[b] + i and
  *   out[b][i][hq] = softmax(sm_scale * q[b][i][hq] K^T) V
  * over cache positions 0 .. p (causal), K and V dequantised from their
- * containers inside the kernel. Query head hq reads KV head hq / (Hq/Hkv).
- * One CTA per (b, KV head, block of 128 / G query tokens): its warps rANS-
- * decode each 32-token block once into fp16 tiles that serve all of the
- * block's 128 query rows; scores and P.V run on the tensor cores (tcgen05,
- * fp16 operands split into hi + lo halves where fp32 precision matters,
- * fp32 accumulation in tensor memory).
+ * containers on the GPU. Query head hq reads KV head hq / (Hq/Hkv).
+ * Two kernels: every 32-token block that the chunk attends to is rANS-
+ * decoded once per (b, KV head) into fp16 tiles in the workspace; then one
+ * CTA per (b, KV head, block of 128 / G query tokens) streams the tiles in
+ * and runs the scores and P.V on the tensor cores (tcgen05, fp16 operands
+ * split into hi + lo halves where fp32 precision matters, fp32 accumulation
+ * in tensor memory) with the online softmax in between.
  *   q           device [B][n_q][Hq][128], q_dtype DQ_F32 or DQ_BF16
  *   d_kcache, d_vcache  device caches (interleaved layout), 16-byte aligned,
  *               T_cap % 32 == 0
  *   d_q_start   device int32 [B]; a query row whose position is outside
  *               [0, T_cap) gets out = 0 and is counted in clamped_lengths
  *   out         device [B][n_q][Hq][128], out_dtype DQ_F32 or DQ_BF16
+ *   d_workspace device, >= dq_prefill_workspace_bytes(...) bytes, 16-byte
+ *               aligned, contents need not be initialised (the decoded
+ *               tiles: 520 bytes per token and KV head of the cache)
  *   d_stats     device dq_stats or NULL (integrity_errors: corrupt
- *               containers in the attended range, each counted once;
- *               wait_timeouts: should stay 0)
+ *               containers in the attended range; wait_timeouts: should
+ *               stay 0)
  * Hq / Hkv must be 1, 2, 4 or 8 and Hkv the tables' n_kv_heads; n_q >= 0
- * (0 does nothing). Needs no workspace and allocates nothing. */
+ * (0 does nothing). Calls sharing a workspace must not overlap on the GPU. */
+size_t dq_prefill_workspace_bytes(const dq_tables *t, int B, int Hkv,
+                                  int64_t T_cap);
 int dq_prefill_attention(const dq_tables *t, const void *q, int q_dtype,
                          const uint8_t *d_kcache, const uint8_t *d_vcache,
                          const int32_t *d_q_start, int B, int n_q, int Hq,
                          int Hkv, int64_t T_cap, float sm_scale, void *out,
-                         int out_dtype, dq_stats *d_stats, void *stream);
+                         int out_dtype, void *d_workspace, size_t ws_bytes,
+                         dq_stats *d_stats, void *stream);
 /* The same over paged pools (layout and page-table rules as in
- * dq_decode_attention_paged; T_cap is 32 * max_pages). */
+ * dq_decode_attention_paged; T_cap is 32 * max_pages for the workspace). */
 int dq_prefill_attention_paged(const dq_tables *t, const void *q, int q_dtype,
                                const uint8_t *d_kpool, const uint8_t *d_vpool,
                                int64_t num_pages, const int32_t *d_page_table,
                                int64_t max_pages, const int32_t *d_q_start, int B,
                                int n_q, int Hq, int Hkv, float sm_scale,
-                               void *out, int out_dtype, dq_stats *d_stats,
-                               void *stream);
+                               void *out, int out_dtype, void *d_workspace,
+                               size_t ws_bytes, dq_stats *d_stats, void *stream);
 
 /* Test hook: decodes n flat containers of one stream.
  *   d_cache   device [n][C]; d_syms device uint8 [n][128]; d_norm16 device
