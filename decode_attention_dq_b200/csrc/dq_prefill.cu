@@ -53,28 +53,30 @@ namespace dqi {
 namespace {
 
 constexpr int kRows = 128;          // query rows per CTA (the MMA's M)
-constexpr int kGrp = 32;            // tokens per cache block
-constexpr int kSoftWarps = 4;       // warps 0..3
-constexpr int kMmaWarp = 4;         // warp 4
-constexpr int kLoadWarp = 5;        // warp 5
-constexpr int kAttnThreads = 32 * 6;
-constexpr int kMaxSlots = 12;       // ring depth of prefill_kernel
+constexpr int kGrp = 32;            // tokens per cache block (one decoder warp)
+constexpr int kBlk = 128;           // tokens per workspace slot / attention block (the score MMA's N)
+constexpr int kSoftWarps = 8;       // warps 0..7: warp w and w + 4 share rows 32 (w % 4) ..
+constexpr int kMmaWarp = 8;         // warp 8
+constexpr int kLoadWarp = 9;        // warp 9
+constexpr int kAttnThreads = 32 * 10;
+constexpr int kMaxSlots = 3;        // ring depth of prefill_kernel
 constexpr int kTileWarps = 20;      // warps per CTA of prefill_tiles_kernel
 constexpr uint32_t kTmemCols = 512;
 // Tensor-memory columns (32-bit each; 128 lanes = rows).
 constexpr uint32_t kColO = 0;       // O: 128 fp32 columns
-constexpr uint32_t kColS = 128;     // S: 2 buffers x 32 fp32 columns
-constexpr uint32_t kColP = 192;     // W: 2 buffers x (16 hi + 16 lo) columns of packed fp16 pairs
-constexpr uint32_t kColQh = 256;    // q~ hi: 64 columns of packed fp16 pairs
-constexpr uint32_t kColQl = 320;    // q~ lo: 64 columns
-constexpr int kTileBytes = kGrp * kD * 2;                  // one fp16 tile: 32 tokens x 128 coordinates
-constexpr int kSlotBytes = 2 * kTileBytes + 2 * kGrp * 4;  // K tile, V tile, K norms, V norms
+constexpr uint32_t kColQh = 128;    // q~ hi: 64 columns of packed fp16 pairs
+constexpr uint32_t kColQl = 192;    // q~ lo: 64 columns
+constexpr uint32_t kColS = 256;     // 2 buffers x 128 columns: the scores S (fp32), then in place the
+                                    // weights W: tokens 0..63 hi | lo, tokens 64..127 hi | lo (32 each)
+constexpr int kTileBytes = kBlk * kD * 2;                  // one fp16 tile: 128 tokens x 128 coordinates
+constexpr int kSlotBytes = 2 * kTileBytes + 2 * kBlk * 4;  // K tile, V tile, K norms, V norms
+constexpr int kChunkStride = kBlk / 8 * 128;               // bytes between 8-coordinate chunks of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kSpin = 1u << 24;  // bound on each mbarrier wait loop
 // Barrier slots of prefill_kernel.
-constexpr int kBarFull = 0, kBarEmpty = kMaxSlots, kBarSFull = 2 * kMaxSlots, kBarSFree = kBarSFull + 2,
-              kBarPFull = kBarSFull + 4, kBarPvDone = kBarSFull + 6, kBarQFull = kBarSFull + 8,
-              kBarDrain = kBarSFull + 9, kNumBars = kBarSFull + 10;
+constexpr int kBarFull = 0, kBarEmpty = kMaxSlots, kBarSFull = 2 * kMaxSlots, kBarWFull = kBarSFull + 2,
+              kBarPvDone = kBarSFull + 4, kBarQFull = kBarSFull + 6, kBarDrain = kBarSFull + 7,
+              kNumBars = kBarSFull + 8;
 static_assert(kSlotBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -104,16 +106,19 @@ __host__ __device__ inline TilesSmem tiles_smem_layout(int ck, int cv) {
 }
 
 // Shared memory of prefill_kernel: barriers, tensor-memory base and abort
-// flag, then the ring of slots.
+// flag, the row-max exchange [2 blocks][2 halves][128 rows] and the row-sum
+// exchange [2 halves][128 rows] of the softmax warp pairs, then the ring.
 struct AttnSmem {
-  size_t bars, misc, ring, total;
+  size_t bars, misc, pmax, lsum, ring, total;
 };
 
 __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
   AttnSmem s;
   s.bars = 0;
   s.misc = s.bars + kNumBars * 8;
-  s.ring = align_up(s.misc + 16, 128);
+  s.pmax = align_up(s.misc + 16, 16);
+  s.lsum = s.pmax + 2 * 2 * kRows * 4;
+  s.ring = align_up(s.lsum + 2 * kRows * 4, 128);
   s.total = s.ring + static_cast<size_t>(nslots) * kSlotBytes;
   return s;
 }
@@ -332,25 +337,31 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   __syncthreads();
 
   const int ck = a.ck, cv = a.cv;
-  const int64_t gcap = a.T_cap / kGrp;
-  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * gcap;  // slot s = (b Hkv + h) gcap + j
+  const int64_t gslots = (a.T_cap + kBlk - 1) / kBlk;  // slots per (b, h)
+  constexpr int kQuarters = kBlk / kGrp;
+  // Work unit u = ((b Hkv + h) gslots + slot) * 4 + quarter: one 32-token
+  // group of one slot.
+  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * gslots * kQuarters;
   const int64_t W = static_cast<int64_t>(gridDim.x) * kTileWarps;
   uint8_t *stg = smem + L.stage + static_cast<size_t>(warp) * L.stage_bytes;
   auto kslot = [&](int s) { return stg + s * L.kslot; };
   auto vslot = [&](int s) { return stg + 2 * L.kslot + s * L.vslot; };
   unsigned bad = 0, bad_pages = 0;
-  // Next slot >= s (in steps of W) that the chunk attends to.
-  auto next_valid = [&](int64_t s) -> int64_t {
-    for (; s < total; s += W) {
-      const int64_t bh = s / gcap, j = s % gcap;
-      const int64_t hi = last_position(a.q_start[bh / a.Hkv], a.n_q, a.T_cap);
-      if (hi >= 0 && j <= hi / kGrp) return s;
+  auto last_of = [&](int64_t u) -> int64_t {
+    return last_position(a.q_start[(u / (gslots * kQuarters)) / a.Hkv], a.n_q, a.T_cap);
+  };
+  // Next unit >= u (in steps of W) inside a slot the chunk attends to.
+  auto next_valid = [&](int64_t u) -> int64_t {
+    for (; u < total; u += W) {
+      const int64_t hi = last_of(u);
+      if (hi >= 0 && (u / kQuarters) % gslots <= hi / kBlk) return u;
     }
     return total;
   };
-  auto block_of = [&](int64_t s) -> int64_t {
+  // Cache block (32 tokens) of group j of the unit's (b, h).
+  auto block_of = [&](int64_t u, int64_t j) -> int64_t {
+    const int64_t bh = u / (gslots * kQuarters);
     if (a.page_table) {
-      const int64_t bh = s / gcap, j = s % gcap;
       int64_t pg = a.page_table[(bh / a.Hkv) * a.max_pages + j];
       if (pg < 0 || pg >= a.num_pages) {
         ++bad_pages;
@@ -358,62 +369,77 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
       }
       return pg * a.Hkv + bh % a.Hkv;
     }
-    return s;
+    return bh * (a.T_cap / kGrp) + j;
   };
-  auto stage = [&](int sl, int64_t s) {
-    const int64_t blk = block_of(s);
+  auto group_of = [&](int64_t u) -> int64_t { return ((u / kQuarters) % gslots) * kQuarters + u % kQuarters; };
+  // Units whose group holds an attended token are decoded; the others (past
+  // the last attended position, possibly past the cache) are zero-filled.
+  auto decoded = [&](int64_t u) { return group_of(u) * kGrp <= last_of(u); };
+  auto stage = [&](int sl, int64_t u) {
+    const int64_t blk = block_of(u, group_of(u));
     const uint8_t *ks = a.kcache + blk * kGrp * ck;
     const uint8_t *vs = a.vcache + blk * kGrp * cv;
     for (int c = lane; c < (kGrp * ck) >> 4; c += 32) cp_async16(kslot(sl) + c * 16, ks + c * 16);
     for (int c = lane; c < (kGrp * cv) >> 4; c += 32) cp_async16(vslot(sl) + c * 16, vs + c * 16);
   };
 
-  int64_t s = next_valid(static_cast<int64_t>(blockIdx.x) * kTileWarps + warp);
-  if (s < total) stage(0, s);
+  int64_t u = next_valid(static_cast<int64_t>(blockIdx.x) * kTileWarps + warp);
+  if (u < total && decoded(u)) stage(0, u);
   cp_async_commit();
-  for (int k = 0; s < total; ++k) {
+  for (int k = 0; u < total; ++k) {
     const int sl = k & 1;
-    const int64_t s_next = next_valid(s + W);
-    if (s_next < total) stage(sl ^ 1, s_next);
+    const int64_t u_next = next_valid(u + W);
+    if (u_next < total && decoded(u_next)) stage(sl ^ 1, u_next);
     cp_async_commit();
     cp_async_wait_1();
     __syncwarp();
-    const uint8_t *kb = kslot(sl) + lane;
-    const uint8_t *vb = vslot(sl) + lane;
-    RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
-    RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
-    uint8_t *dst = a.tiles + s * kSlotBytes;
-#pragma unroll 1
-    for (int i8 = 0; i8 < kD; i8 += 8) {
-      uint32_t hk[8], hv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
-        const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
-        hk[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + ek);
-        hv[u] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + 4 * kMaxLevels + ev);
-      }
-      // 8 coordinates of this lane's token: 16 bytes at chunk i8 / 8 (512
-      // bytes per chunk of 32 tokens), token offset 16 * lane.
-      const size_t off = static_cast<size_t>((i8 >> 3) * 512 + lane * 16);
-      *reinterpret_cast<uint4 *>(dst + off) =
-          make_uint4(__byte_perm(hk[0], hk[1], 0x5410), __byte_perm(hk[2], hk[3], 0x5410),
-                     __byte_perm(hk[4], hk[5], 0x5410), __byte_perm(hk[6], hk[7], 0x5410));
-      *reinterpret_cast<uint4 *>(dst + kTileBytes + off) =
-          make_uint4(__byte_perm(hv[0], hv[1], 0x5410), __byte_perm(hv[2], hv[3], 0x5410),
-                     __byte_perm(hv[4], hv[5], 0x5410), __byte_perm(hv[6], hv[7], 0x5410));
-    }
-    const int64_t bh = s / gcap;
-    const int64_t hi = last_position(a.q_start[bh / a.Hkv], a.n_q, a.T_cap);
-    const int64_t tok = (s % gcap) * kGrp + lane;
-    // Tokens past the last attended position keep zero norms: their bytes may
-    // be anything, and the softmax multiplies the weights by these norms.
+    const int q4 = static_cast<int>(u % kQuarters);
+    uint8_t *dst = a.tiles + (u / kQuarters) * static_cast<int64_t>(kSlotBytes);
     float *nrm = reinterpret_cast<float *>(dst + 2 * kTileBytes);
-    nrm[lane] = tok <= hi ? norm_of(kb) : 0.0f;
-    nrm[kGrp + lane] = tok <= hi ? norm_of(vb) : 0.0f;
-    if (tok <= hi) bad += (rk.x != kL) + (rv.x != kL);
+    const int tl = q4 * kGrp + lane;  // token within the slot
+    if (decoded(u)) {
+      const uint8_t *kb = kslot(sl) + lane;
+      const uint8_t *vb = vslot(sl) + lane;
+      RansLane rk = rans_open(smem, static_cast<uint32_t>(kb - smem));
+      RansLane rv = rans_open(smem, static_cast<uint32_t>(vb - smem));
+#pragma unroll 1
+      for (int i8 = 0; i8 < kD; i8 += 8) {
+        uint32_t hk[8], hv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t ek = rans_step<kTwoK>(rk, lut_k, smem);
+          const uint32_t ev = rans_step<kTwoV>(rv, lut_v, smem);
+          hk[e] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + ek);
+          hv[e] = *reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint8_t *>(lev) + 4 * kMaxLevels + ev);
+        }
+        // 8 coordinates of this lane's token: 16 bytes in chunk i8 / 8.
+        const size_t off = static_cast<size_t>((i8 >> 3) * kChunkStride + tl * 16);
+        *reinterpret_cast<uint4 *>(dst + off) =
+            make_uint4(__byte_perm(hk[0], hk[1], 0x5410), __byte_perm(hk[2], hk[3], 0x5410),
+                       __byte_perm(hk[4], hk[5], 0x5410), __byte_perm(hk[6], hk[7], 0x5410));
+        *reinterpret_cast<uint4 *>(dst + kTileBytes + off) =
+            make_uint4(__byte_perm(hv[0], hv[1], 0x5410), __byte_perm(hv[2], hv[3], 0x5410),
+                       __byte_perm(hv[4], hv[5], 0x5410), __byte_perm(hv[6], hv[7], 0x5410));
+      }
+      const int64_t hi = last_of(u);
+      const int64_t tok = group_of(u) * kGrp + lane;
+      // Tokens past the last attended position keep zero norms: their bytes
+      // may be anything, and the softmax multiplies the weights by them.
+      nrm[tl] = tok <= hi ? norm_of(kb) : 0.0f;
+      nrm[kBlk + tl] = tok <= hi ? norm_of(vb) : 0.0f;
+      if (tok <= hi) bad += (rk.x != kL) + (rv.x != kL);
+    } else {
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+      for (int c = 0; c < kD / 8; ++c) {
+        *reinterpret_cast<uint4 *>(dst + c * kChunkStride + tl * 16) = z;
+        *reinterpret_cast<uint4 *>(dst + kTileBytes + c * kChunkStride + tl * 16) = z;
+      }
+      nrm[tl] = 0.0f;
+      nrm[kBlk + tl] = 0.0f;
+    }
     __syncwarp();  // the staging slot is refilled next iteration
-    s = s_next;
+    u = u_next;
   }
   cp_async_wait_0();
   if (a.stats) {
@@ -424,6 +450,8 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   }
 }
 
+__device__ __forceinline__ void pair_sync(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+
 __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int ns = a.nslots;
@@ -432,6 +460,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + L.misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 4);
+  float *pmax = reinterpret_cast<float *>(smem + L.pmax);  // [2][2][128]
+  float *lsum = reinterpret_cast<float *>(smem + L.lsum);  // [2][128]
   auto slot_base = [&](int d) { return smem + L.ring + static_cast<size_t>(d) * kSlotBytes; };
 
   // Work item: the query blocks of one (b, h) are consecutive, latest first.
@@ -446,8 +476,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   const int i_hi = min(i_lo + Mt, a.n_q) - 1;
   const int64_t lo_pos = max(qs + i_lo, int64_t(0));
   const int64_t hi_pos = min(qs + i_hi, a.T_cap - 1);
-  const int64_t nG = lo_pos <= hi_pos ? hi_pos / kGrp + 1 : 0;
-  const int64_t gcap = a.T_cap / kGrp;
+  const int64_t nB = lo_pos <= hi_pos ? hi_pos / kBlk + 1 : 0;  // 128-token blocks to attend
+  const int64_t gslots = (a.T_cap + kBlk - 1) / kBlk;
 
   // ---- set-up ----
   if (warp == kMmaWarp) {
@@ -463,8 +493,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars + kBarSFull + i, 1);
-      mbar_init(bars + kBarSFree + i, kRows);
-      mbar_init(bars + kBarPFull + i, kRows);
+      mbar_init(bars + kBarWFull + i, 32 * kSoftWarps);
       mbar_init(bars + kBarPvDone + i, 1);
     }
     mbar_init(bars + kBarQFull, kRows);
@@ -477,18 +506,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   tc_fence_after();
   const uint32_t tbase = *tslot;
   unsigned timeouts = 0, clamped = 0;
+
   if (warp < kSoftWarps) {
-    // ================= softmax warpgroup: thread = row =================
-    const int r = tid;
-    const uint32_t tl = tbase + (static_cast<uint32_t>(warp * 32) << 16);  // this warp's lanes
+    // ===== softmax: warps w and w + 4 own rows r = 32 (w % 4) + lane; warp w
+    // takes tokens 0..63 of each block, warp w + 4 tokens 64..127 =====
+    const int half = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t tl = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);  // this warp's lanes
     const int ti = i_lo + r / G, g = r % G;
     const bool in_chunk = ti <= i_hi;
     const int64_t pos = qs + ti;
     const bool row_ok = in_chunk && pos >= 0 && pos < a.T_cap;
-    if (in_chunk && !row_ok) ++clamped;
+    if (half == 0 && in_chunk && !row_ok) ++clamped;
     const int hq = h * G + g;
     const int64_t qbase = ((static_cast<int64_t>(b) * a.n_q + (in_chunk ? ti : 0)) * a.Hq + hq) * kD;
     // D1: q~ = H D q (unnormalised), times 2^e so that max |q~| is in [2^13, 2^14).
+    // Both warps of a pair need the row's scale; warp w alone stores q~.
     float crow = 0.0f;
     {
       float v[kD];
@@ -512,70 +545,89 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       }
       // logit (log2 units) = S * ||k|| * crow, with S = sum (q~ sc)(kappa_K y)
       crow = row_ok ? a.sm_scale * kLog2e / (static_cast<float>(kD) * sc * a.tabs->k.score_scale) : 0.0f;
+      if (half == 0) {
 #pragma unroll
-      for (int c16 = 0; c16 < kD; c16 += 16) {
-        uint32_t hi[8], lo[8];
+        for (int c16 = 0; c16 < kD; c16 += 16) {
+          uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) split_pair(v[c16 + 2 * p] * sc, v[c16 + 2 * p + 1] * sc, hi[p], lo[p]);
-        tmem_st8(tl + kColQh + c16 / 2, hi);
-        tmem_st8(tl + kColQl + c16 / 2, lo);
+          for (int p = 0; p < 8; ++p) split_pair(v[c16 + 2 * p] * sc, v[c16 + 2 * p + 1] * sc, hi[p], lo[p]);
+          tmem_st8(tl + kColQh + c16 / 2, hi);
+          tmem_st8(tl + kColQl + c16 / 2, lo);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bars + kBarQFull);
       }
-      tmem_wait_st();
     }
-    tc_fence_before();
-    mbar_arrive(bars + kBarQFull);
 
     float m_run = -INFINITY, l_run = 0.0f;
     bool alive = true;
-    for (int64_t j = 0; j < nG && alive; ++j) {
+    const int pair_id = 1 + (warp & 3);
+    for (int64_t j = 0; j < nB; ++j) {
       const int sb = static_cast<int>(j & 1);
       const int rb = static_cast<int>(j % ns);
-      bool ok = mbar_wait(bars + kBarSFull + sb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) &&
+      bool ok = alive && mbar_wait(bars + kBarSFull + sb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) &&
                 mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag);
-      if (!__all_sync(kFull, ok)) {
-        ++timeouts;
+      ok = __all_sync(kFull, ok);
+      // The two warps of a pair leave the loop together (they meet at the
+      // pair barriers below): agree on going on, through shared memory.
+      pmax[(sb * 2 + half) * kRows + r] = ok ? 0.0f : 1.0f;
+      pair_sync(pair_id);
+      const bool go = ok && pmax[(sb * 2 + (half ^ 1)) * kRows + r] == 0.0f;
+      pair_sync(pair_id);
+      if (!go) {
+        if (alive) ++timeouts;
         alive = false;
         break;
       }
       tc_fence_after();
-      float s[32];
-      tmem_ld32(tl + kColS + 32 * sb, s);
-      tc_fence_before();
-      mbar_arrive(bars + kBarSFree + sb);
-      const float *nk = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes);
-      const float *nv = nk + kGrp;
+      const uint32_t scol = tl + kColS + 128 * sb + 64 * half;  // this warp's 64 score columns
+      float u[64];
+      {
+        float s0[32], s1[32];
+        tmem_ld32(scol, s0);
+        tmem_ld32(scol + 32, s1);
+        const float *nk = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + 64 * half;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          u[t] = s0[t] * nk[t];
+          u[32 + t] = s1[t] * nk[32 + t];
+        }
+      }
       // u = S ||k|| (the logit divided by crow > 0); tokens past this row's
       // position are masked, which only happens on the causal diagonal.
-      float u[32];
+      const int64_t rel = pos - j * kBlk - 64 * half;
+      const int lim = (!row_ok || rel < 0) ? -1 : (rel > 63 ? 63 : static_cast<int>(rel));
+      if (!__all_sync(kFull, lim >= 63)) {
 #pragma unroll
-      for (int t = 0; t < 32; ++t) u[t] = s[t] * nk[t];
-      const int64_t rel = pos - j * kGrp;
-      const int lim = (!row_ok || rel < 0) ? -1 : (rel > 31 ? 31 : static_cast<int>(rel));
-      if (!__all_sync(kFull, lim >= 31)) {
-#pragma unroll
-        for (int t = 0; t < 32; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
+        for (int t = 0; t < 64; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
       }
-      float mu[16];
+      float mu[32];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) mu[t] = fmaxf(u[t], u[t + 16]);
+      for (int t = 0; t < 32; ++t) mu[t] = fmaxf(u[t], u[t + 32]);
 #pragma unroll
-      for (int w = 8; w >= 1; w >>= 1)
+      for (int w2 = 16; w2 >= 1; w2 >>= 1)
 #pragma unroll
-        for (int t = 0; t < w; ++t) mu[t] = fmaxf(mu[t], mu[t + w]);
-      const float mx = mu[0] == -INFINITY ? m_run : fmaxf(m_run, mu[0] * crow);
+        for (int t = 0; t < w2; ++t) mu[t] = fmaxf(mu[t], mu[t + w2]);
+      // Row maximum over both halves: exchange through shared memory.
+      pmax[(sb * 2 + half) * kRows + r] = mu[0];
+      pair_sync(pair_id);
+      const float mrow = fmaxf(mu[0], pmax[(sb * 2 + (half ^ 1)) * kRows + r]);
+      const float mx = mrow == -INFINITY ? m_run : fmaxf(m_run, mrow * crow);
       float alpha = 1.0f;
-      uint32_t whi[16], wlo[16];
+      uint32_t whi[32], wlo[32];
       float psum = 0.0f;
       if (mx == -INFINITY) {
 #pragma unroll
-        for (int p = 0; p < 16; ++p) whi[p] = wlo[p] = 0u;
+        for (int p = 0; p < 32; ++p) whi[p] = wlo[p] = 0u;
       } else {
         if (m_run != -INFINITY) alpha = ex2(m_run - mx);
-        // p = 2^(logit - mx); w = p ||v|| (norms of tokens past the CTA's
-        // range are 0, so masked tokens give exactly 0).
+        // p = 2^(logit - mx); w = p ||v|| (norms of tokens past the last
+        // attended position are 0, so masked tokens give exactly 0).
+        const float *nv = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + kBlk + 64 * half;
         float ps[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
+        for (int p = 0; p < 32; ++p) {
           const float p0 = ex2(fmaf(u[2 * p], crow, -mx)), p1 = ex2(fmaf(u[2 * p + 1], crow, -mx));
           ps[p & 1] += p0 + p1;
           split_pair(p0 * nv[2 * p], p1 * nv[2 * p + 1], whi[p], wlo[p]);
@@ -584,52 +636,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
         m_run = mx;
       }
       l_run = l_run * alpha + psum;
-      // O and the W buffer are free once P.V of the previous group is done.
-      if (j > 0) {
-        ok = mbar_wait(bars + kBarPvDone + ((j - 1) & 1), static_cast<uint32_t>(((j - 1) >> 1) & 1), abort_flag);
-        if (!__all_sync(kFull, ok)) {
-          ++timeouts;
-          alive = false;
-          break;
-        }
+      // O is current once P.V of the previous block is done.
+      ok = j == 0 ||
+           mbar_wait(bars + kBarPvDone + ((j - 1) & 1), static_cast<uint32_t>(((j - 1) >> 1) & 1), abort_flag);
+      ok = __all_sync(kFull, ok);
+      if (ok) {
         tc_fence_after();
-        if (__any_sync(kFull, alpha != 1.0f)) {
+        if (j > 0 && __any_sync(kFull, alpha != 1.0f)) {
 #pragma unroll 1
-          for (int c = 0; c < kD; c += 32) {
+          for (int c = 0; c < 64; c += 32) {
             float o[32];
-            tmem_ld32(tl + kColO + c, o);
-            uint32_t w[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(o[e] * alpha);
+            const uint32_t oc = tl + kColO + 64 * half + c;
+            tmem_ld32(oc, o);
             uint32_t w0[16], w1[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              w0[e] = w[e];
-              w1[e] = w[16 + e];
+              w0[e] = __float_as_uint(o[e] * alpha);
+              w1[e] = __float_as_uint(o[16 + e] * alpha);
             }
-            tmem_st16(tl + kColO + c, w0);
-            tmem_st16(tl + kColO + c + 16, w1);
+            tmem_st16(oc, w0);
+            tmem_st16(oc + 16, w1);
           }
         }
-      }
-      tmem_st16(tl + kColP + 32 * sb, whi);
-      tmem_st16(tl + kColP + 32 * sb + 16, wlo);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bars + kBarPFull + sb);
-    }
-    // D7: o = D H o_rot / 128 with o_rot = O / (l kappa_V).
-    bool have_o = alive && nG > 0;
-    if (have_o) {
-      const int64_t jl = nG - 1;
-      const bool ok =
-          mbar_wait(bars + kBarPvDone + (jl & 1), static_cast<uint32_t>((jl >> 1) & 1), abort_flag);
-      if (!__all_sync(kFull, ok)) {
+        // W in place of this warp's own score columns: hi in the first 32,
+        // lo in the next 32 (the scores were read above).
+        uint32_t w0[16], w1[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          w0[e] = whi[e];
+          w1[e] = whi[16 + e];
+        }
+        tmem_st16(scol, w0);
+        tmem_st16(scol + 16, w1);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          w0[e] = wlo[e];
+          w1[e] = wlo[16 + e];
+        }
+        tmem_st16(scol + 32, w0);
+        tmem_st16(scol + 48, w1);
+        tmem_wait_st();
+      } else {
         ++timeouts;
-        have_o = false;
+        alive = false;  // both warps stop at the next agreement
       }
+      tc_fence_before();
+      mbar_arrive(bars + kBarWFull + sb);  // always, so the MMA warp's count completes
     }
-    {
+    // D7: o = D H o_rot / 128 with o_rot = O / (l kappa_V); l sums both halves.
+    lsum[half * kRows + r] = l_run;
+    pair_sync(pair_id);
+    const float l_all = l_run + lsum[(half ^ 1) * kRows + r];
+    if (half == 0) {
+      bool have_o = alive && nB > 0;
+      if (have_o) {
+        const int64_t jl = nB - 1;
+        const bool ok =
+            mbar_wait(bars + kBarPvDone + (jl & 1), static_cast<uint32_t>((jl >> 1) & 1), abort_flag);
+        if (!__all_sync(kFull, ok)) {
+          ++timeouts;
+          have_o = false;
+        }
+      }
       float v[kD];
       if (have_o) {
         tc_fence_after();
@@ -645,7 +713,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
         for (int c = 0; c < kD; ++c) v[c] = 0.0f;
       }
       const float inv =
-          (have_o && row_ok && l_run > 0.0f) ? 1.0f / (l_run * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
+          (have_o && row_ok && l_all > 0.0f) ? 1.0f / (l_all * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
 #pragma unroll
       for (int c = 0; c < kD; ++c) v[c] *= inv;
       wht128_regs(v);
@@ -661,48 +729,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       }
     }
   } else if (warp == kMmaWarp) {
-    // ================= MMA issue (one lane) =================
-    if (lane == 0 && nG > 0) {
-      const uint32_t idS = instr_desc(kRows, kGrp, 0);
+    // ===== MMA issue (one lane) =====
+    if (lane == 0 && nB > 0) {
+      const uint32_t idS = instr_desc(kRows, kBlk, 0);
       const uint32_t idO = instr_desc(kRows, kD, 1);
       bool alive = mbar_wait(bars + kBarQFull, 0, abort_flag);
       if (!alive) ++timeouts;
       tc_fence_after();
-      // W_jj V_jj into O: A = W hi / lo (tensor memory, 8 columns per 16
-      // tokens), B = V tile, MN-major: token groups of 8 at 128 bytes (LBO),
-      // coordinate chunks of 8 at 512 bytes (SBO).
+      // O += W_jj V_jj: A = W (tensor memory; tokens 16 ks .. 16 ks + 15 of
+      // the hi or lo half), B = V tile, MN-major: token groups of 8 at 128
+      // bytes (LBO), coordinate chunks of 8 at kChunkStride bytes (SBO).
       auto issue_pv = [&](int64_t jj) -> bool {
-        if (!mbar_wait(bars + kBarPFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag)) return false;
+        if (!mbar_wait(bars + kBarWFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag)) return false;
         tc_fence_after();
         const uint32_t vt = smem_u32(slot_base(static_cast<int>(jj % ns)) + kTileBytes);
-        const uint32_t wp = tbase + kColP + 32 * static_cast<uint32_t>(jj & 1);
+        const uint32_t wb = tbase + kColS + 128 * static_cast<uint32_t>(jj & 1);
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const uint64_t bd = smem_desc(vt + ks * 256, 128, 512);
-          mma_ts(tbase + kColO, wp + ks * 8, bd, idO, (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_ts(tbase + kColO, wp + 16 + ks * 8, bd, idO, 1u);
+        for (int ks = 0; ks < kBlk / 16; ++ks) {
+          const uint64_t bd = smem_desc(vt + ks * 256, 128, kChunkStride);
+          const uint32_t wc = wb + (ks < 4 ? 0u : 64u) + (ks & 3) * 8;
+          mma_ts(tbase + kColO, wc, bd, idO, (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tbase + kColO, wc + 32, bd, idO, 1u);
         }
         tc_commit(bars + kBarPvDone + (jj & 1));
         tc_commit(bars + kBarEmpty + static_cast<int>(jj % ns));
         return true;
       };
-      for (int64_t j = 0; j < nG && alive; ++j) {
+      for (int64_t j = 0; j < nB && alive; ++j) {
         const int rb = static_cast<int>(j % ns);
         alive = mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag);
+        // The score buffer j & 1 held W of block j - 2: wait until its P.V is done.
         if (alive && j >= 2)
-          alive = mbar_wait(bars + kBarSFree + (j & 1), static_cast<uint32_t>(((j - 2) >> 1) & 1), abort_flag);
+          alive = mbar_wait(bars + kBarPvDone + (j & 1), static_cast<uint32_t>(((j - 2) >> 1) & 1), abort_flag);
         if (!alive) {
           ++timeouts;
           break;
         }
         tc_fence_after();
         // S_j = q~ K_j^T: B = K tile, K-major: token groups of 8 at 128 bytes
-        // (SBO), coordinate chunks of 8 at 512 bytes (LBO).
+        // (SBO), coordinate chunks of 8 at kChunkStride bytes (LBO).
         const uint32_t kt = smem_u32(slot_base(rb));
-        const uint32_t sd = tbase + kColS + 32 * static_cast<uint32_t>(j & 1);
+        const uint32_t sd = tbase + kColS + 128 * static_cast<uint32_t>(j & 1);
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint64_t bd = smem_desc(kt + ks * 1024, 512, 128);
+          const uint64_t bd = smem_desc(kt + ks * 2 * kChunkStride, kChunkStride, 128);
           mma_ts(sd, tbase + kColQh + ks * 8, bd, idS, ks > 0 ? 1u : 0u);
           mma_ts(sd, tbase + kColQl + ks * 8, bd, idS, 1u);
         }
@@ -712,30 +782,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
           alive = false;
         }
       }
-      if (alive && !issue_pv(nG - 1)) ++timeouts;
+      if (alive && !issue_pv(nB - 1)) ++timeouts;
       // Drain: every MMA issued above has completed before tensor memory is freed.
       tc_commit(bars + kBarDrain);
-      if (!mbar_wait(bars + kBarDrain, 0, abort_flag)) {
-        // The abort path may skip the wait above; wait once more without
-        // looking at the flag, still bounded.
-        const uint32_t da = smem_u32(bars + kBarDrain);
-        for (uint32_t it = 0; it < kSpin; ++it) {
-          uint32_t done;
-          asm volatile(
-              "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], 0;\nselp.u32 %0, 1, 0, P;\n}\n"
-              : "=r"(done)
-              : "r"(da)
-              : "memory");
-          if (done) break;
-        }
+      const uint32_t da = smem_u32(bars + kBarDrain);
+      for (uint32_t it = 0; it < kSpin; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], 0;\nselp.u32 %0, 1, 0, P;\n}\n"
+            : "=r"(done)
+            : "r"(da)
+            : "memory");
+        if (done) break;
       }
     }
   } else if (warp == kLoadWarp) {
-    // ================= slot loader (one lane) =================
-    if (lane == 0 && nG > 0) {
-      const uint8_t *src = a.tiles + static_cast<size_t>(bh * gcap) * kSlotBytes;
+    // ===== slot loader (one lane) =====
+    if (lane == 0 && nB > 0) {
+      const uint8_t *src = a.tiles + static_cast<size_t>(bh * gslots) * kSlotBytes;
       int64_t issued = 0;
-      for (int64_t j = 0; j < nG; ++j) {
+      for (int64_t j = 0; j < nB; ++j) {
         const int sl = static_cast<int>(j % ns);
         if (j >= ns && !mbar_wait(bars + kBarEmpty + sl, static_cast<uint32_t>(((j / ns) - 1) & 1), abort_flag)) {
           ++timeouts;
@@ -803,7 +869,7 @@ int64_t prefill_grid(int B, int Hkv, int G, int n_q) {
 }
 
 size_t prefill_workspace_bytes(int B, int Hkv, int64_t T_cap) {
-  return static_cast<size_t>(B) * Hkv * static_cast<size_t>(T_cap / kGrp) * kSlotBytes;
+  return static_cast<size_t>(B) * Hkv * static_cast<size_t>((T_cap + kBlk - 1) / kBlk) * kSlotBytes;
 }
 
 bool prefill_supported(int ck, int cv) {
