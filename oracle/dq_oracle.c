@@ -537,6 +537,101 @@ int dqo_encode_vector(const dqo_stream *st, const int8_t *signs,
   return 0;
 }
 
+/* Rate-distortion fill (drift mode 1). [news] "So What": once entropy
+ * coding sits in the KV path, the rate-distortion toolbox of video coding
+ * carries over. Reading: a container's unused bytes are spent on accuracy,
+ * the mirror image of drift. A candidate is a symbol i whose nearest level j
+ * (least (u_i - y_j)^2 in fp32, ties to the lower level) is one level from
+ * its current symbol q[i] and at most one level from the quantiser's symbol
+ * q0[i], with dD = (u_i - y_j)^2 - (u_i - y_q)^2 < 0 and
+ * dR = cost[j] - cost[q] > 0 (fp32). Candidates are taken in order of
+ * key = dD / dR (fp32; ties to the lower i); each is kept if the re-encoded
+ * stream still fits `budget`, else undone. Returns the final length;
+ * *ups = candidates kept. */
+int dqo_rd_fill(const dqo_stream *st, const float *u, const uint8_t *q0,
+                uint8_t *q, int n, int budget, int *ups) {
+  int len = dqo_rans_encode(st, q, n, NULL, 0);
+  *ups = 0;
+  if (len > budget) return len;
+  int ci[DQO_D], cj[DQO_D];
+  float ck[DQO_D];
+  int nc = 0;
+  for (int i = 0; i < n && i < DQO_D; ++i) {
+    int j = 0;
+    float best = 0.0f;
+    for (int l = 0; l < st->n_levels; ++l) {
+      float d = u[i] - st->yf[l];
+      float e = d * d;
+      if (l == 0 || e < best) {
+        best = e;
+        j = l;
+      }
+    }
+    int s = q[i];
+    if (j == s || abs(j - s) != 1 || abs(j - (int)q0[i]) > 1) continue;
+    float dj = u[i] - st->yf[j];
+    float ds = u[i] - st->yf[s];
+    float dd = dj * dj - ds * ds;
+    float dr = st->cost[j] - st->cost[s];
+    if (!(dd < 0.0f) || !(dr > 0.0f)) continue;
+    float key = dd / dr;
+    /* insertion in (key, i) order */
+    int k = nc++;
+    while (k > 0 && (ck[k - 1] > key)) {
+      ck[k] = ck[k - 1];
+      ci[k] = ci[k - 1];
+      cj[k] = cj[k - 1];
+      --k;
+    }
+    ck[k] = key;
+    ci[k] = i;
+    cj[k] = j;
+  }
+  for (int k = 0; k < nc; ++k) {
+    uint8_t old = q[ci[k]];
+    q[ci[k]] = (uint8_t)cj[k];
+    int l2 = dqo_rans_encode(st, q, n, NULL, 0);
+    if (l2 > budget) {
+      q[ci[k]] = old;
+    } else {
+      len = l2;
+      *ups += 1;
+    }
+  }
+  return len;
+}
+
+/* E1-E7 with the drift mode: 0 = drift only (dqo_encode_vector), 1 = drift
+ * then the rate-distortion fill (skipped after a fallback). */
+int dqo_encode_vector_mode(const dqo_stream *st, const int8_t *signs,
+                           const float *x, uint8_t *container, uint8_t *q_out,
+                           dqo_stats *stats, int drift_mode) {
+  if (drift_mode == 0) return dqo_encode_vector(st, signs, x, container, q_out, stats);
+  float u[DQO_D];
+  uint16_t nh = 0;
+  int nf = dqo_rotate_normalize(x, signs, u, &nh);
+  uint8_t q0[DQO_D], q[DQO_D];
+  dqo_quantize(st, u, DQO_D, q0);
+  memcpy(q, q0, DQO_D);
+  int moves = 0, fb = 0, ups = 0;
+  int len = dqo_drift_fit(st, u, q, DQO_D, st->payload_bytes, &moves, NULL, &fb);
+  if (!fb && len <= st->payload_bytes) len = dqo_rd_fill(st, u, q0, q, DQO_D, st->payload_bytes, &ups);
+  memset(container, 0, (size_t)st->container_bytes);
+  container[0] = (uint8_t)(nh & 0xFFu);
+  container[1] = (uint8_t)(nh >> 8);
+  if (stats) {
+    stats->nonfinite_inputs += (uint64_t)nf;
+    stats->syms_drifted += (uint64_t)moves;
+    stats->cont_drifted += (moves > 0) ? 1u : 0u;
+    stats->overflow_fallbacks += (uint64_t)fb;
+    stats->syms_filled += (uint64_t)ups;
+  }
+  if (q_out) memcpy(q_out, q, DQO_D);
+  if (len < 0 || len > st->payload_bytes) return -1;
+  dqo_rans_encode(st, q, DQO_D, container + 2, st->payload_bytes);
+  return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* Decode                                                             */
 /* ------------------------------------------------------------------ */
@@ -602,6 +697,20 @@ int dqo_encode_batch(const dqo_stream *st, const int8_t *signs_per_head,
     int rc = dqo_encode_vector(st, sg, x + v * DQO_D,
                                containers + v * st->container_bytes,
                                syms ? syms + v * DQO_D : NULL, stats);
+    if (rc != 0) bad += 1;
+  }
+  return bad;
+}
+
+int dqo_encode_batch_mode(const dqo_stream *st, const int8_t *signs_per_head,
+                          const float *x, const int32_t *head_of, int64_t n_vec,
+                          uint8_t *containers, uint8_t *syms, dqo_stats *stats,
+                          int drift_mode) {
+  int bad = 0;
+  for (int64_t v = 0; v < n_vec; ++v) {
+    const int8_t *sg = signs_per_head + (int64_t)head_of[v] * DQO_D;
+    int rc = dqo_encode_vector_mode(st, sg, x + v * DQO_D, containers + v * st->container_bytes,
+                                    syms ? syms + v * DQO_D : NULL, stats, drift_mode);
     if (rc != 0) bad += 1;
   }
   return bad;

@@ -69,6 +69,7 @@ typedef struct {
   uint64_t cont_drifted;       /* containers with >= 1 move          */
   uint64_t overflow_fallbacks; /* containers that took the fallback  */
   uint64_t nonfinite_inputs;   /* vectors treated as zero            */
+  uint64_t syms_filled;        /* symbols moved up by the RD fill    */
 } dqo_stats;
 
 /* ---- tables ---------------------------------------------------------- */
@@ -102,6 +103,11 @@ int dqo_drift_fit(const dqo_stream *st, const float *u, uint8_t *q, int n,
 int dqo_encode_vector(const dqo_stream *st, const int8_t *signs,
                       const float *x, uint8_t *container, uint8_t *q_out,
                       dqo_stats *stats);
+int dqo_rd_fill(const dqo_stream *st, const float *u, const uint8_t *q0,
+                uint8_t *q, int n, int budget, int *ups);
+int dqo_encode_vector_mode(const dqo_stream *st, const int8_t *signs,
+                           const float *x, uint8_t *container, uint8_t *q_out,
+                           dqo_stats *stats, int drift_mode);
 
 /* ---- decode ---------------------------------------------------------- */
 int dqo_rans_decode(const dqo_stream *st, const uint8_t *buf, int len,
@@ -113,6 +119,10 @@ int dqo_decode_container(const dqo_stream *st, const uint8_t *container,
 int dqo_encode_batch(const dqo_stream *st, const int8_t *signs_per_head,
                      const float *x, const int32_t *head_of, int64_t n_vec,
                      uint8_t *containers, uint8_t *syms, dqo_stats *stats);
+int dqo_encode_batch_mode(const dqo_stream *st, const int8_t *signs_per_head,
+                          const float *x, const int32_t *head_of, int64_t n_vec,
+                          uint8_t *containers, uint8_t *syms, dqo_stats *stats,
+                          int drift_mode);
 int64_t dqo_decode_batch(const dqo_stream *st, const uint8_t *containers,
                          int64_t n_vec, uint8_t *syms, uint16_t *norm16,
                          int32_t *status);

@@ -54,6 +54,7 @@ class _Stats(C.Structure):
         ("cont_drifted", C.c_uint64),
         ("overflow_fallbacks", C.c_uint64),
         ("nonfinite_inputs", C.c_uint64),
+        ("syms_filled", C.c_uint64),
     ]
 
 
@@ -97,6 +98,9 @@ def load():
         lib.dqo_encode_batch.argtypes = [P(_Stream), vp, vp, vp, C.c_int64, vp,
                                          vp, P(_Stats)]
         lib.dqo_decode_batch.argtypes = [P(_Stream), vp, C.c_int64, vp, vp, vp]
+        lib.dqo_encode_batch_mode.argtypes = [P(_Stream), vp, vp, vp, C.c_int64, vp,
+                                              vp, P(_Stats), C.c_int]
+        lib.dqo_rd_fill.argtypes = [P(_Stream), vp, vp, vp, C.c_int, C.c_int, P(C.c_int)]
         lib.dqo_decode_batch.restype = C.c_int64
         _lib = lib
     return _lib
@@ -113,12 +117,14 @@ class Stats:
     cont_drifted: int = 0
     overflow_fallbacks: int = 0
     nonfinite_inputs: int = 0
+    syms_filled: int = 0
 
     def add(self, s: _Stats):
         self.syms_drifted += int(s.syms_drifted)
         self.cont_drifted += int(s.cont_drifted)
         self.overflow_fallbacks += int(s.overflow_fallbacks)
         self.nonfinite_inputs += int(s.nonfinite_inputs)
+        self.syms_filled += int(s.syms_filled)
 
 
 class Stream:
@@ -263,9 +269,21 @@ def drift_fit(st: Stream, u: np.ndarray, q: np.ndarray, budget: int):
     return ln, q, moved.astype(bool), int(moves.value), bool(fb.value)
 
 
+def rd_fill(st: Stream, u: np.ndarray, q0: np.ndarray, q: np.ndarray, budget: int):
+    """Rate-distortion fill of one symbol string (drift mode 1): returns
+    (length, filled symbols, number of symbols moved up)."""
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    q0 = np.ascontiguousarray(q0, dtype=np.uint8)
+    q = np.ascontiguousarray(q, dtype=np.uint8).copy()
+    ups = C.c_int(0)
+    ln = load().dqo_rd_fill(st.ref, _ptr(u), _ptr(q0), _ptr(q), q.shape[0], budget, C.byref(ups))
+    return ln, q, int(ups.value)
+
+
 def encode_vectors(st: Stream, sg_per_head: np.ndarray, x: np.ndarray,
-                   head_of: np.ndarray):
+                   head_of: np.ndarray, drift_mode: int = 0):
     """Encode N vectors x[N,128] (float32) with sign rows sg_per_head[head_of[v]].
+    drift_mode 0: drift only; 1: drift, then the rate-distortion fill.
 
     Returns (containers [N,C] uint8, symbols [N,128] uint8, Stats, n_bad)."""
     x = np.ascontiguousarray(x, dtype=np.float32)
@@ -275,8 +293,8 @@ def encode_vectors(st: Stream, sg_per_head: np.ndarray, x: np.ndarray,
     cont = np.zeros((n, st.container_bytes), dtype=np.uint8)
     syms = np.zeros((n, D), dtype=np.uint8)
     s = _Stats()
-    bad = load().dqo_encode_batch(st.ref, _ptr(sg), _ptr(x), _ptr(ho), n,
-                                  _ptr(cont), _ptr(syms), C.byref(s))
+    bad = load().dqo_encode_batch_mode(st.ref, _ptr(sg), _ptr(x), _ptr(ho), n,
+                                       _ptr(cont), _ptr(syms), C.byref(s), int(drift_mode))
     stats = Stats()
     stats.add(s)
     return cont, syms, stats, int(bad)
@@ -299,7 +317,8 @@ class Tables:
     def __init__(self, n_kv_heads: int, k_levels: int = 8, v_levels: int = 6,
                  k_container_bytes: int = 36, v_container_bytes: int = 36,
                  sign_seed: int = 0, k_rate_offset: float = 0.0,
-                 v_rate_offset: float = 0.0):
+                 v_rate_offset: float = 0.0, drift_mode: int = 0):
+        self.drift_mode = drift_mode
         self.k = Stream(k_levels, k_container_bytes, k_rate_offset)
         self.v = Stream(v_levels, v_container_bytes, v_rate_offset)
         self.n_kv_heads = n_kv_heads
@@ -312,8 +331,8 @@ def encode_cache(tab: Tables, K: np.ndarray, V: np.ndarray):
     B, H, T, d = K.shape
     assert d == D and V.shape == K.shape and H == tab.n_kv_heads
     head_of = np.broadcast_to(np.arange(H, dtype=np.int32)[None, :, None], (B, H, T)).reshape(-1)
-    kc, ks, kst, kbad = encode_vectors(tab.k, tab.signs, K.reshape(-1, D), head_of)
-    vc, vs, vst, vbad = encode_vectors(tab.v, tab.signs, V.reshape(-1, D), head_of)
+    kc, ks, kst, kbad = encode_vectors(tab.k, tab.signs, K.reshape(-1, D), head_of, tab.drift_mode)
+    vc, vs, vst, vbad = encode_vectors(tab.v, tab.signs, V.reshape(-1, D), head_of, tab.drift_mode)
     assert kbad == 0 and vbad == 0
     return (kc.reshape(B, H, T, -1), vc.reshape(B, H, T, -1),
             ks.reshape(B, H, T, D), vs.reshape(B, H, T, D), kst, vst)
