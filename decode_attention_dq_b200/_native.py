@@ -19,7 +19,8 @@ DQ_F32, DQ_BF16 = 0, 1
 DQ_STREAM_K, DQ_STREAM_V = 0, 1
 STATS_FIELDS = ("k_syms_drifted", "v_syms_drifted", "k_cont_drifted", "v_cont_drifted",
                 "overflow_fallbacks", "integrity_errors", "nonfinite_inputs",
-                "dropped_writes", "clamped_lengths", "bad_pages", "wait_timeouts")
+                "dropped_writes", "clamped_lengths", "bad_pages", "wait_timeouts",
+                "k_syms_filled", "v_syms_filled")
 EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_stream_table",
             "dq_get_stream_design", "dq_get_signs", "dq_append_kv", "dq_decode_workspace_bytes",
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",
@@ -33,7 +34,7 @@ class DqConfig(C.Structure):
         ("head_dim", C.c_int32), ("k_levels", C.c_int32), ("v_levels", C.c_int32),
         ("prob_bits", C.c_int32), ("k_container_bytes", C.c_int32),
         ("v_container_bytes", C.c_int32), ("k_bits_per_value", C.c_float),
-        ("v_bits_per_value", C.c_float), ("n_kv_heads", C.c_int32), ("reserved", C.c_int32),
+        ("v_bits_per_value", C.c_float), ("n_kv_heads", C.c_int32), ("drift_mode", C.c_int32),
         ("sign_seed", C.c_uint64), ("k_rate_offset", C.c_float), ("v_rate_offset", C.c_float),
     ]
 

@@ -250,7 +250,7 @@ int dq_build_tables(const dq_config *cfg, dq_tables **out) {
   if (!cfg || !out) return DQ_ERR_NULL;
   *out = nullptr;
   if (cfg->head_dim != dqi::kD || cfg->prob_bits != dqi::kProbBits || cfg->n_kv_heads < 1 ||
-      cfg->n_kv_heads > 4096 || cfg->reserved != 0)
+      cfg->n_kv_heads > 4096 || (cfg->drift_mode != 0 && cfg->drift_mode != 1))
     return DQ_ERR_CONFIG;
   dq_tables *t = nullptr;
   try {
@@ -390,6 +390,7 @@ static int append_core(const dq_tables *t, const void *k, const void *v, int dty
     a.cv = t->v.container_bytes;
     a.nk = t->k.n_levels;
     a.nv = t->v.n_levels;
+    a.drift_mode = t->cfg.drift_mode;
     a.two_k = has_small_freq(t->k);
     a.two_v = has_small_freq(t->v);
     a.stats = d_stats;

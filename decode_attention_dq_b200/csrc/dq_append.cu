@@ -368,9 +368,10 @@ struct DriftCount {
 
 // E6 for one over-long container, by the whole warp. On entry q[] holds the
 // symbols and u[k] this lane's coordinates lane + 32 k; rank[] and tgt[] are
-// scratch, stack the warp's push stacks.
+// scratch, stack the warp's push stacks. Returns the number of moves applied
+// (the ranked moves 0 .. n - 1, in rank[] / tgt[]), or -1 after a fallback.
 template <bool kTwo>
-__device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
+__device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
                                           uint8_t *stack, const uint8_t *q, uint8_t *rank, uint8_t *tgt, int64_t vd,
                                           uint16_t n16v, const float (&u)[4], int lane, int first_batch,
                                           DriftCount &dc) {
@@ -460,10 +461,103 @@ __device__ __forceinline__ void drift_one(const AppendArgs &a, const StreamCtx &
     }
     applied = ranked;
     ++dc.fallbacks;
+    dc.moves += static_cast<unsigned>(applied);
+    dc.containers += applied > 0 ? 1u : 0u;
+    __syncwarp();
+    return -1;
   }
   dc.moves += static_cast<unsigned>(applied);
   dc.containers += applied > 0 ? 1u : 0u;
   __syncwarp();
+  return applied;
+}
+
+// Rate-distortion fill (drift mode 1) of one container that fits, by the
+// whole warp: qd[] holds the symbols after drift, q0[] the quantiser's, u[k]
+// this lane's coordinates lane + 32 k. A candidate is a symbol whose nearest
+// level j (least (u - y_j)^2 in fp32, ties to the lower level) is one level
+// from qd and at most one from q0, with dD = (u - y_j)^2 - (u - y_qd)^2 < 0 and
+// dR = cost_j - cost_qd > 0; candidates go in order of dD / dR (fp32, ties to
+// the lower index), each kept if lane 0's re-encode still fits. Stores the
+// container; returns the number of symbols moved.
+template <bool kTwo>
+__device__ __forceinline__ int rd_fill(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
+                                       uint8_t *stack, const uint8_t *q0, uint8_t *qd, int64_t v, uint16_t n16,
+                                       const float (&u)[4], int lane) {
+  float key[4];
+  uint8_t jn[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = lane + 32 * k;
+    int j = 0;
+    float best = 0.0f;
+    for (int l = 0; l < c.nl; ++l) {
+      const float d = __fsub_rn(u[k], T.lev[l]);
+      const float e = __fmul_rn(d, d);
+      if (l == 0 || e < best) {
+        best = e;
+        j = l;
+      }
+    }
+    const int s = qd[i];
+    jn[k] = static_cast<uint8_t>(j);
+    key[k] = INFINITY;
+    if (j != s && abs(j - s) == 1 && abs(j - static_cast<int>(q0[i])) <= 1) {
+      const float dj = __fsub_rn(u[k], T.lev[j]);
+      const float ds = __fsub_rn(u[k], T.lev[s]);
+      const float dd = __fsub_rn(__fmul_rn(dj, dj), __fmul_rn(ds, ds));
+      const float dr = __fsub_rn(T.cost[j], T.cost[s]);
+      if (dd < 0.0f && dr > 0.0f) key[k] = __fdiv_rn(dd, dr);
+    }
+  }
+  uint8_t *stk = stack;  // lane 0's push stack
+  int ups = 0;
+  while (true) {
+    float bk = key[0];
+    int bi = lane;
+#pragma unroll
+    for (int k = 1; k < 4; ++k)
+      if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const float ok = __shfl_xor_sync(kFull, bk, off);
+      const int oi = __shfl_xor_sync(kFull, bi, off);
+      if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
+    }
+    if (bk == INFINITY) break;
+    uint8_t old = 0;
+    if ((bi & 31) == lane) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (bi == lane + 32 * k) {
+          key[k] = INFINITY;
+          old = qd[bi];
+          qd[bi] = jn[k];
+        }
+    }
+    __syncwarp();
+    int len = 0;
+    if (lane == 0) {
+      uint32_t x = 0;
+      len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(qd[i]); }, T.es, stk, &x);
+    }
+    len = __shfl_sync(kFull, len, 0);
+    if (len > c.P) {
+      if ((bi & 31) == lane) qd[bi] = old;
+    } else {
+      ++ups;
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    uint32_t x = 0;
+    const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(qd[i]); }, T.es, stk, &x);
+    bool dr = false;
+    uint8_t *dst = c.dst_of(a, v, &dr);
+    if (dst && len <= c.P) store_container(dst, c.C, n16, x, stk, len);
+  }
+  __syncwarp();
+  return ups;
 }
 
 __device__ __forceinline__ void add_stats(const AppendArgs &a, bool is_v, const DriftCount &dc, unsigned nf,
@@ -566,12 +660,26 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   bool dropped = false, bad_page = false;
   uint8_t *dst = c.dst_of(a, v, &dropped, &bad_page);
   DriftCount dc;
+  int applied = 0;
   if (len <= c.P) {
     if (lane == 0 && dst) store_container(dst, c.C, n16, x, stk, len);
   } else {
     __syncwarp();
     // One pass of 32 in most cases (latency of a small append).
-    drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 32, dc);
+    applied = drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 32, dc);
+  }
+  if (a.drift_mode == 1 && applied >= 0) {
+    // The symbols after drift (the first `applied` ranked moves) go to tgt[].
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = lane + 32 * k;
+      const uint32_t r = (len <= c.P) ? kNoRank : W.rank[i];
+      W.tgt[i] = (r != kNoRank && static_cast<int>(r) < applied) ? W.tgt[i] : W.q[i];
+    }
+    __syncwarp();
+    const int ups = rd_fill<kTwo>(a, c, T, W.stack, W.q, W.tgt, v, n16, u, lane);
+    if (lane == 0 && ups && a.stats)
+      atomicAdd(is_v ? &a.stats->v_syms_filled : &a.stats->k_syms_filled, static_cast<unsigned long long>(ups));
   }
   if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u, bad_page ? 1u : 0u);
 }
@@ -795,7 +903,8 @@ int launch_append(const AppendArgs &a, void *stream) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // Lane per vector once every SM gets a few full CTAs of 128 vectors per
   // stream; below that, a warp per vector spreads the work wider.
-  const bool lanes = nvec >= static_cast<int64_t>(sms) * kAW * 32 * 2;
+  // Drift mode 1 (rate-distortion fill) runs in the warp-per-vector kernel.
+  const bool lanes = a.drift_mode == 0 && nvec >= static_cast<int64_t>(sms) * kAW * 32 * 2;
   AppendArgs b = a;
   // The drift list holds 32-bit vector indices, one slot per vector.
   if (!lanes || b.list_cap < nvec || nvec > 0xFFFFFFFFll) b.drift_list = nullptr;

@@ -82,6 +82,7 @@ struct AppendArgs {
   int ck, cv;       // container bytes
   int nk, nv;       // levels
   bool two_k, two_v;  // the stream's table has a symbol with f < 16 (two pushes per step)
+  int drift_mode;     // 0: drift only; 1: drift, then the rate-distortion fill
   dq_stats *stats;
   // Optional drift list (workspace): over-long containers of the
   // lane-per-vector kernel are listed here ([2][list_cap] vector indices, K

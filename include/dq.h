@@ -83,7 +83,8 @@ typedef struct {
   float k_bits_per_value;    /* default 2.26                                 */
   float v_bits_per_value;    /* default 2.26                                 */
   int32_t n_kv_heads;        /* >= 1; one rotation-sign vector per KV head   */
-  int32_t reserved;          /* must be 0                                    */
+  int32_t drift_mode;        /* 0: drift only (default); 1: drift, then the  */
+                             /* rate-distortion fill (see dq_append_kv)      */
   uint64_t sign_seed;        /* rotation signs: splitmix64 from this seed    */
   float k_rate_offset;       /* added to the target rate, bits/value (0)     */
   float v_rate_offset;       /* added to the target rate, bits/value (0)     */
@@ -103,6 +104,8 @@ typedef struct {
   unsigned long long clamped_lengths;    /* seq_len > T_max or > T_cap       */
   unsigned long long bad_pages;          /* page-table entries out of range  */
   unsigned long long wait_timeouts;      /* bounded in-kernel waits given up */
+  unsigned long long k_syms_filled;      /* K symbols moved up by the fill   */
+  unsigned long long v_syms_filled;      /* V symbols moved up by the fill   */
 } dq_stats;
 
 typedef struct dq_tables dq_tables; /* opaque, library-owned */
@@ -169,7 +172,15 @@ int dq_get_signs(const dq_tables *t, int8_t *signs);
  *   stream      cudaStream_t
  * Hkv must equal the tables' n_kv_heads. Containers are bit-identical to the
  * reference definition (fp32 rotation/normalisation in a fixed order, greedy
- * drift, zero padding). */
+ * drift, zero padding).
+ * With drift_mode 1 in the tables' configuration, a rate-distortion fill
+ * follows drift ([news] "So What": the rate-distortion toolbox of video
+ * coding carries over): a container's unused bytes are spent on accuracy by
+ * moving symbols one level up to their nearest level (at most one level from
+ * the quantiser's symbol), best error reduction per bit first, each kept
+ * only if the exact coded length still fits (none after a fallback). The
+ * decoder is unchanged; encoding is several times slower (every append then
+ * runs a warp per vector). */
 int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype,
                  int B, int Hkv, int n_new, const int32_t *d_start_pos,
                  uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
