@@ -13,7 +13,10 @@ roofline fraction are reported beside it.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dq|reference]
                   [--workload NAME] [--paged] [--layers L] [--graph] [--prefill N_Q]
---paged keeps the caches in page pools behind a shuffled page table; --layers
+                  [--drift-mode 0|1]
+--drift-mode 1 encodes with the rate-distortion fill after drift (the encode
+report then shows its cost); --paged keeps the caches in page pools behind a
+shuffled page table; --layers
 runs an L-layer attention-only decode loop (one cache per layer); --graph also
 times the step captured once as a CUDA graph and replayed. --prefill N_Q
 switches to the chunked-prefill step (append an N_Q-token chunk to every
@@ -201,7 +204,8 @@ def run_dq(args):
         import torch.distributed as dist
     w = replica_workload(synth.WORKLOADS[args.workload], rank)
     dev = torch.device("cuda", torch.cuda.current_device())
-    tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
+    tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits,
+                             drift_mode=args.drift_mode)
     ck, cv = tab.k.container_bytes, tab.v.container_bytes
     T = w.T
     T_cap = (T + 31) // 32 * 32
@@ -384,6 +388,7 @@ def run_dq(args):
                        "k_container_bytes": ck, "v_container_bytes": cv,
                        "l2": "inputs larger than L2 (%.0f MB of containers read per step)" % (comp_bytes / 1e6),
                        "cache": "paged: 32-token pages in a shuffled order" if args.paged else "contiguous",
+                       "drift_mode": args.drift_mode,
                        "layers": L,
                        "parallelism": "replicas x%d" % ws},
             "hbm_gbs": hbm_gbs,
@@ -400,7 +405,9 @@ def run_dq(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": LAUNCHES_PER_STEP * L * args.steps,
             "clocks": clk,
-            "drift": {"prefill_k_syms_pct": 100.0 * pstats["k_syms_drifted"] / (token_heads * 128),
+            "drift": {"prefill_k_syms_filled_pct": 100.0 * pstats["k_syms_filled"] / (token_heads * 128),
+                      "prefill_v_syms_filled_pct": 100.0 * pstats["v_syms_filled"] / (token_heads * 128),
+                      "prefill_k_syms_pct": 100.0 * pstats["k_syms_drifted"] / (token_heads * 128),
                       "prefill_v_syms_pct": 100.0 * pstats["v_syms_drifted"] / (token_heads * 128),
                       "prefill_k_cont_pct": 100.0 * pstats["k_cont_drifted"] / token_heads,
                       "prefill_v_cont_pct": 100.0 * pstats["v_cont_drifted"] / token_heads,
@@ -837,6 +844,8 @@ def main():
     ap.add_argument("--paged", action="store_true", help="page pools and a shuffled page table")
     ap.add_argument("--layers", type=int, default=1, help="layers of the decode loop (one cache each)")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as a CUDA graph")
+    ap.add_argument("--drift-mode", type=int, default=0, choices=[0, 1],
+                    help="0: drift only (default); 1: drift, then the rate-distortion fill")
     ap.add_argument("--prefill", type=int, default=0, metavar="N_Q",
                     help="chunked-prefill mode: append an N_Q-token chunk and attend its queries causally")
     args = ap.parse_args()

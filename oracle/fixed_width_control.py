@@ -8,7 +8,8 @@ and can afford finer levels in the same bytes ("Drift: Bending Variable Back
 to Fixed" gives 8 levels for K and 6 for V at 2.26 bits per value).
 
 This module measures that claim on the synthetic workloads with the oracle
-only (CPU, fp64 where it matters): D-Quant containers (rANS + drift) against a
+only (CPU, fp64 where it matters): D-Quant containers (rANS + drift, and with
+the rate-distortion fill of drift mode 1) against a
 fixed-width control that quantises the same rotated, normalised coordinates
 with the Gaussian Lloyd-Max quantiser of 2^b levels at b bits per value (b = 2:
 4 levels, 32 bytes of codes + the 2-byte fp16 norm = 34 bytes, within the
@@ -68,8 +69,9 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
 
 
 def measure(workload: str = "qwen3_8b_b16_t8k", rows: int = 64, tokens: int = 512,
-            budgets=(1.96, 2.26, 3.0), fixed_bits=(2,)):
-    """Rows of results: one per (stream, coder, budget)."""
+            budgets=(1.96, 2.26, 3.0), fixed_bits=(2,), drift_modes=(0, 1)):
+    """Rows of results: one per (stream, coder, budget); D-Quant once per
+    drift mode (0: drift only; 1: drift, then the rate-distortion fill)."""
     from decode_attention_dq_b200 import synth
 
     w = synth.WORKLOADS[workload]
@@ -95,10 +97,10 @@ def measure(workload: str = "qwen3_8b_b16_t8k", rows: int = 64, tokens: int = 51
     results = []
     rotated = {s: [rotate_all(data[s][r], sg_all[picks[r][1]]) for r in range(rows)] for s in ("k", "v")}
 
-    # D-Quant at each budget (same budget for K and V).
-    for bits in budgets:
+    # D-Quant at each budget (same budget for K and V) and drift mode.
+    for bits, mode in [(b_, m_) for b_ in budgets for m_ in drift_modes]:
         C = o.container_bytes(bits)
-        tab = o.Tables(w.Hkv, k_container_bytes=C, v_container_bytes=C)
+        tab = o.Tables(w.Hkv, k_container_bytes=C, v_container_bytes=C, drift_mode=mode)
         recon = {}
         for s in ("k", "v"):
             st = tab.k if s == "k" else tab.v
@@ -107,7 +109,8 @@ def measure(workload: str = "qwen3_8b_b16_t8k", rows: int = 64, tokens: int = 51
             for r in range(rows):
                 h = picks[r][1]
                 x = data[s][r]
-                cont, syms, stt, bad = o.encode_vectors(st, tab.signs, x, np.full(x.shape[0], h, np.int32))
+                cont, syms, stt, bad = o.encode_vectors(st, tab.signs, x, np.full(x.shape[0], h, np.int32),
+                                                        drift_mode=mode)
                 assert bad == 0
                 u, _ = rotated[s][r]
                 y_hat = st.yf.astype(np.float64)[syms.astype(np.int64)]
@@ -119,7 +122,8 @@ def measure(workload: str = "qwen3_8b_b16_t8k", rows: int = 64, tokens: int = 51
                 rel_x += float(np.sum((xh - x) ** 2)) / float(np.sum(x.astype(np.float64) ** 2))
                 moved += stt.syms_drifted
             n = rows * tokens
-            results.append(dict(stream=s.upper(), coder="D-Quant %d levels (rANS + drift)" % st.n,
+            results.append(dict(stream=s.upper(),
+                                coder="D-Quant %d levels (rANS + drift%s)" % (st.n, " + RD fill" if mode else ""),
                                 bits=bits, bytes=C, mse_u=mse_u / (n * o.D), rel_x=rel_x / rows,
                                 drift=moved / (n * o.D)))
         err = stats_for(recon)
