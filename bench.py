@@ -363,6 +363,35 @@ def run_dq(args):
     barrier()
     e2e_ms = max_over_ranks([f0.elapsed_time(f1)], dist, dev)[0]
     e2e_value = whole_job_rate(kv_tokens_step, ws, e2e_ms / args.steps)
+
+    # ---- chunked prefill over the same cache: the last n_q positions as a
+    # chunk of queries (dq_prefill_attention), device-resident inputs ----
+    prefill = None
+    if args.prefill_chunk > 0 and page_table is None and L == 1 and T > args.prefill_chunk:
+        n_q = args.prefill_chunk
+        gq = torch.Generator(device=dev).manual_seed(w.seed)
+        qc = torch.randn((w.B, n_q, w.Hq, 128), generator=gq, device=dev).to(w.torch_dtype)
+        outc = torch.empty((w.B, n_q, w.Hq, 128), dtype=torch.float32, device=dev)
+        qs0 = torch.full((w.B,), T - n_q, dtype=torch.int32, device=dev)
+        pws = torch.empty(dq.dq_prefill_workspace_bytes(tab, w.B, w.Hkv, T_cap), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            dq.dq_prefill_attention(tab, qc, kc, vc, qs0, outc, workspace=pws, stats=stats)
+        torch.cuda.synchronize()
+        barrier()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        p0.record(stream)
+        for _ in range(reps):
+            dq.dq_prefill_attention(tab, qc, kc, vc, qs0, outc, workspace=pws, stats=stats)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        pms = max_over_ranks([p0.elapsed_time(p1) / reps], dist, dev)[0]
+        del pws
+        prefill = {"chunk": n_q, "q_start": T - n_q, "ms": pms,
+                   "query_tokens_per_s": whole_job_rate(w.B * n_q, ws, pms),
+                   "useful_flops": chunk_pairs(w.B, w.Hq, T - n_q, n_q) * FLOPS_PER_PAIR,
+                   "launches": 2 * reps}
     h2d = (host_k[0].numel() + host_v[0].numel() + host_q[0].numel()) * host_k[0].element_size()
     d2h = out_host.numel() * out_host.element_size()
     st = dq.stats_dict(stats)
@@ -415,6 +444,13 @@ def run_dq(args):
             "integrity_errors": st["integrity_errors"],
             "prefill_s": prefill_s,
             "encode": encode_report(enc_ms, enc_vectors, w, ck, cv, alu_peak, peaks),
+            "chunked_prefill": None if prefill is None else dict(
+                prefill, what="dq_prefill_attention of the last %d positions of every sequence as a chunk of "
+                              "queries over the %d-token compressed cache (random queries)" % (prefill["chunk"], T),
+                tflops=prefill["useful_flops"] / (prefill["ms"] * 1e-3) / 1e12,
+                roofline={"bound": "tensor", "peak": float(peaks.get("bf16_tflops", 1590.0)), "unit": "TFLOP/s",
+                          "frac": prefill["useful_flops"] / (prefill["ms"] * 1e-3) / 1e12
+                          / float(peaks.get("bf16_tflops", 1590.0))}),
             "serving": {"what": "attention-only decode loop over %d layer(s): append 1 token + decode "
                                 "attention per layer, %d sequences of %d tokens" % (L, w.B, T),
                         "tokens_per_s": whole_job_rate(w.B, ws, ms_per_step),
@@ -540,6 +576,29 @@ FLOPS_PER_PAIR = 4 * 128
 # Kernel launches of one prefill step: dq_append_kv of the chunk (encode +
 # drift kernels) and dq_prefill_attention (tile decode + attention kernels).
 PREFILL_LAUNCHES_PER_STEP = 4
+
+
+# DRAM traffic of prefill_kernel (the dominant kernel of the prefill step)
+# from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, one
+# pass) of `bench.py --prefill 512 --workload qwen3_8b_b16_t8k`: the decoded
+# tiles read once (545 MB) plus the queries, and the fp32 output. Reported
+# only for that workload and container size while the kernel source matches.
+PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "511adba83ee0a406",
+                   "workload": "qwen3_8b_b16_t8k", "chunk": 512, "ck": 36, "cv": 36,
+                   "bytes": 615.08e6 + 117.36e6}
+
+
+def prefill_traffic(workload, n_q, ck, cv):
+    import hashlib
+    t = PREFILL_TRAFFIC
+    try:
+        with open(os.path.join(ROOT, t["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if sha != t["sha256_16"] or (workload, n_q, ck, cv) != (t["workload"], t["chunk"], t["ck"], t["cv"]):
+        return None
+    return t["bytes"]
 
 
 def chunk_pairs(B, Hq, q_start, n_q):
@@ -668,7 +727,10 @@ def run_prefill(args):
                        "parallelism": "replicas x%d" % ws},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "frac_of_sustained": achieved / peak_sus,
-                         "traffic": None,
+                         "traffic": prefill_traffic(w.name, n_q, ck, cv),
+                         "traffic_note": "prefill_kernel DRAM bytes per launch from one ncu capture of this "
+                                         "workload; algorithmic bytes: containers once + q + out",
+                         "algorithmic_bytes": comp_bytes + io_bytes,
                          "useful_flops": flops, "flops_convention": "4 x 128 per (query row, visible key)",
                          "kernel": "prefill_tiles_kernel + prefill_kernel (dq_prefill_attention)",
                          "kernel_ms": attn_ms,
@@ -844,6 +906,8 @@ def main():
     ap.add_argument("--paged", action="store_true", help="page pools and a shuffled page table")
     ap.add_argument("--layers", type=int, default=1, help="layers of the decode loop (one cache each)")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as a CUDA graph")
+    ap.add_argument("--prefill-chunk", type=int, default=512, metavar="N_Q",
+                    help="also time chunked prefill of the last N_Q positions over the decode cache (0: off)")
     ap.add_argument("--drift-mode", type=int, default=0, choices=[0, 1],
                     help="0: drift only (default); 1: drift, then the rate-distortion fill")
     ap.add_argument("--prefill", type=int, default=0, metavar="N_Q",
