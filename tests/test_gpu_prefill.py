@@ -5,8 +5,9 @@ Caches are filled through dq_append_kv (containers bit-identical to the
 oracle's, checked here too). Cases span several 128-row query blocks with a
 ragged last block, several 32-token groups with a ragged causal diagonal,
 G = 1, 2, 4, 8, fp32 and bf16 operands, rows whose positions fall outside the
-cache, a single-token chunk (which is decode attention), paged pools and a
-full-size chunk of 512 tokens at the end of an 8K context (sampled (b, h)
+cache, a single-token chunk (which is decode attention), paged pools,
+31- and 48-byte containers, a full-size chunk of 512 tokens at the end of an
+8K context and one of 256 tokens at the end of a 64K context (sampled (b, h)
 rows). The bar is max |gpu - oracle| <= 2e-3 * RMS(oracle).
 """
 import numpy as np
@@ -161,5 +162,49 @@ def test_full_size_chunk_at_end_of_8k_context_sampled():
     for b, h in rows:
         cm.assert_attention_close(got[b, :, h * G:(h + 1) * G], ref[b, :, h * G:(h + 1) * G],
                                   what="8K chunk row (%d,%d)" % (b, h))
+    s = dq.stats_dict(stats)
+    assert s["wait_timeouts"] == 0 and s["integrity_errors"] == 0
+
+
+@pytest.mark.parametrize("bits", [1.96, 3.0])
+def test_prefill_other_budgets(bits):
+    # 31- and 48-byte containers (other decode tables, the two-byte K step at
+    # 1.96 bits)
+    B, Hkv, G, T = 2, 2, 4, 300
+    w = synth.scaled(synth.WORKLOADS["qwen3_8b_b16_t8k"], B=B, Hkv=Hkv, Hq=Hkv * G, T=T)
+    K, V, _ = cm.inputs(w)
+    lib = cm.lib_tables(Hkv, k_bits=bits, v_bits=bits)
+    ref_t = cm.oracle_tables(Hkv, k_bits=bits, v_bits=bits)
+    kc, vc = cm.gpu_append_all(lib, K, V, torch.bfloat16)
+    rk, rv, _, _, _, _ = o.encode_cache(ref_t, K, V)
+    n_q = 90
+    q_start = [T - n_q, 17]
+    q = synth.q_chunk(w, n_q)
+    stats = dq.new_stats()
+    got = _prefill(lib, q, kc, vc, q_start, stats=stats)
+    ref = o.attention_prefill_fp64(ref_t, q, _pad(rk, kc.shape[2]), _pad(rv, vc.shape[2]), q_start)
+    cm.assert_attention_close(got, ref, what="prefill %.2f bits" % bits)
+    s = dq.stats_dict(stats)
+    assert s["wait_timeouts"] == 0 and s["integrity_errors"] == 0
+
+
+def test_long_context_chunk_sampled():
+    # The last 256 tokens of a 65536-token context (one (b, h) row checked).
+    w = synth.WORKLOADS["long_b4_t64k"]
+    lib = cm.lib_tables(w.Hkv)
+    ref_t = cm.oracle_tables(w.Hkv)
+    kc = dq.new_cache(w.B, w.Hkv, w.T, 36)
+    vc = dq.new_cache(w.B, w.Hkv, w.T, 36)
+    synth.prefill_cache(lib, w, kc, vc, w.T)
+    n_q = 256
+    q_start = [w.T - n_q] * w.B
+    q = synth.q_chunk(w, n_q)
+    stats = dq.new_stats()
+    got = _prefill(lib, q, kc, vc, q_start, out_dtype=torch.bfloat16, stats=stats)
+    G = w.Hq // w.Hkv
+    b, h = 2, 5
+    ref = o.attention_prefill_fp64(ref_t, q, cm.flat(kc), cm.flat(vc), q_start, rows=[(b, h)])
+    cm.assert_attention_close(got[b, :, h * G:(h + 1) * G], ref[b, :, h * G:(h + 1) * G], extra_rel=2.0 ** -8,
+                              what="64K chunk row (%d,%d)" % (b, h))
     s = dq.stats_dict(stats)
     assert s["wait_timeouts"] == 0 and s["integrity_errors"] == 0
