@@ -583,9 +583,9 @@ PREFILL_LAUNCHES_PER_STEP = 4
 # pass) of `bench.py --prefill 512 --workload qwen3_8b_b16_t8k`: the decoded
 # tiles read once (545 MB) plus the queries, and the fp32 output. Reported
 # only for that workload and container size while the kernel source matches.
-PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "511adba83ee0a406",
+PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "89b08ba04686d927",
                    "workload": "qwen3_8b_b16_t8k", "chunk": 512, "ck": 36, "cv": 36,
-                   "bytes": 615.08e6 + 117.36e6}
+                   "bytes": 617.62e6 + 119.89e6}
 
 
 def prefill_traffic(workload, n_q, ck, cv):

@@ -537,8 +537,14 @@ static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const ui
       return DQ_ERR_ALIGN;
     if (!std::isfinite(sm_scale)) return DQ_ERR_SHAPE;
     if (!dqi::prefill_supported(t->k.container_bytes, t->v.container_bytes)) return DQ_ERR_SHAPE;
-    if (dqi::prefill_grid(B, Hkv, G, n_q) > 0x7FFFFFFF) return DQ_ERR_SHAPE;
-    if (ws_bytes < dqi::prefill_workspace_bytes(B, Hkv, T_cap)) return DQ_ERR_WORKSPACE;
+    // The workspace holds the decoded tiles of a wave of (b, KV head) rows:
+    // at least one row; a smaller workspace than the whole batch's runs the
+    // call in several waves.
+    const int64_t rows = static_cast<int64_t>(B) * Hkv;
+    const size_t row_bytes = dqi::prefill_workspace_bytes(1, 1, T_cap);
+    if (T_cap > 0 && ws_bytes < row_bytes) return DQ_ERR_WORKSPACE;
+    const int64_t per_wave = row_bytes ? std::min<int64_t>(rows, static_cast<int64_t>(ws_bytes / row_bytes)) : rows;
+    if (per_wave > 0 && dqi::prefill_grid(per_wave, G, n_q) > 0x7FFFFFFF) return DQ_ERR_SHAPE;
     int rc = check_device(t);
     if (rc != DQ_OK) return rc;
     if (B == 0 || n_q == 0 || T_cap == 0) {
@@ -572,14 +578,19 @@ static int prefill_core(const dq_tables *t, const void *q, int q_dtype, const ui
     a.two_v = has_small_freq(t->v);
     a.tiles = static_cast<uint8_t *>(d_workspace);
     a.nslots = dqi::prefill_ring_slots();
-    const int64_t rows = static_cast<int64_t>(B) * Hkv * (T_cap / 32);
-    a.tile_grid = static_cast<int>(std::min<int64_t>(t->sm_count, (rows + 19) / 20));
     a.stats = d_stats;
     a.page_table = page_table;
     a.max_pages = max_pages;
     a.num_pages = num_pages;
-    int e = dqi::launch_prefill_attention(a, stream);
-    return e == 0 ? DQ_OK : cuda_fail(static_cast<cudaError_t>(e));
+    for (int64_t bh0 = 0; bh0 < rows; bh0 += per_wave) {
+      a.bh0 = bh0;
+      a.nbh = std::min<int64_t>(per_wave, rows - bh0);
+      const int64_t groups = a.nbh * (T_cap / 32);
+      a.tile_grid = static_cast<int>(std::min<int64_t>(t->sm_count, (groups + 19) / 20));
+      int e = dqi::launch_prefill_attention(a, stream);
+      if (e != 0) return cuda_fail(static_cast<cudaError_t>(e));
+    }
+    return DQ_OK;
   } catch (...) {
     return DQ_ERR_CUDA;
   }

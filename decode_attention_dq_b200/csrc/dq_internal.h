@@ -144,7 +144,8 @@ struct PrefillArgs {
   int out_dtype;
   int ck, cv;
   bool two_k, two_v;
-  uint8_t *tiles;      // workspace: decoded slots [B][Hkv][T_cap / 32]
+  uint8_t *tiles;      // workspace: decoded slots of rows bh0 .. bh0 + nbh - 1, [nbh][ceil(T_cap / 128)]
+  int64_t bh0, nbh;    // the wave of (b, KV head) rows (flat index b Hkv + h) this launch handles
   int nslots;          // ring depth of the attention kernel (prefill_ring_slots)
   int tile_grid;       // CTAs of the tile kernel
   dq_stats *stats;
@@ -153,8 +154,8 @@ struct PrefillArgs {
 };
 int launch_prefill_attention(const PrefillArgs &a, void *stream);
 int prefill_ring_slots();
-// CTAs of the attention kernel: B * Hkv * ceil(n_q / (128 / G)).
-int64_t prefill_grid(int B, int Hkv, int G, int n_q);
+// CTAs of the attention kernel for nbh rows: nbh * ceil(n_q / (128 / G)).
+int64_t prefill_grid(int64_t nbh, int G, int n_q);
 // Bytes of decoded slots for B x Hkv rows of T_cap tokens.
 size_t prefill_workspace_bytes(int B, int Hkv, int64_t T_cap);
 bool prefill_supported(int ck, int cv);

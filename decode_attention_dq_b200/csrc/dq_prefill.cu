@@ -339,16 +339,16 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   const int ck = a.ck, cv = a.cv;
   const int64_t gslots = (a.T_cap + kBlk - 1) / kBlk;  // slots per (b, h)
   constexpr int kQuarters = kBlk / kGrp;
-  // Work unit u = ((b Hkv + h) gslots + slot) * 4 + quarter: one 32-token
-  // group of one slot.
-  const int64_t total = static_cast<int64_t>(a.B) * a.Hkv * gslots * kQuarters;
+  // Work unit u = ((row - bh0) gslots + slot) * 4 + quarter, row = b Hkv + h
+  // of this wave: one 32-token group of one slot.
+  const int64_t total = a.nbh * gslots * kQuarters;  // this wave's units
   const int64_t W = static_cast<int64_t>(gridDim.x) * kTileWarps;
   uint8_t *stg = smem + L.stage + static_cast<size_t>(warp) * L.stage_bytes;
   auto kslot = [&](int s) { return stg + s * L.kslot; };
   auto vslot = [&](int s) { return stg + 2 * L.kslot + s * L.vslot; };
   unsigned bad = 0, bad_pages = 0;
   auto last_of = [&](int64_t u) -> int64_t {
-    return last_position(a.q_start[(u / (gslots * kQuarters)) / a.Hkv], a.n_q, a.T_cap);
+    return last_position(a.q_start[(a.bh0 + u / (gslots * kQuarters)) / a.Hkv], a.n_q, a.T_cap);
   };
   // Next unit >= u (in steps of W) inside a slot the chunk attends to.
   auto next_valid = [&](int64_t u) -> int64_t {
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   };
   // Cache block (32 tokens) of group j of the unit's (b, h).
   auto block_of = [&](int64_t u, int64_t j) -> int64_t {
-    const int64_t bh = u / (gslots * kQuarters);
+    const int64_t bh = a.bh0 + u / (gslots * kQuarters);
     if (a.page_table) {
       int64_t pg = a.page_table[(bh / a.Hkv) * a.max_pages + j];
       if (pg < 0 || pg >= a.num_pages) {
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   const int G = a.G, Mt = kRows / G;
   const int nqb = (a.n_q + Mt - 1) / Mt;
   const int64_t bid = blockIdx.x;
-  const int64_t bh = bid / nqb;
+  const int64_t bh = a.bh0 + bid / nqb;
   const int qb = nqb - 1 - static_cast<int>(bid % nqb);
   const int b = static_cast<int>(bh / a.Hkv), h = static_cast<int>(bh % a.Hkv);
   const int64_t qs = a.q_start[b];
@@ -799,7 +799,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   } else if (warp == kLoadWarp) {
     // ===== slot loader (one lane) =====
     if (lane == 0 && nB > 0) {
-      const uint8_t *src = a.tiles + static_cast<size_t>(bh * gslots) * kSlotBytes;
+      const uint8_t *src = a.tiles + static_cast<size_t>((bh - a.bh0) * gslots) * kSlotBytes;
       int64_t issued = 0;
       for (int64_t j = 0; j < nB; ++j) {
         const int sl = static_cast<int>(j % ns);
@@ -863,9 +863,9 @@ int prefill_ring_slots() {
   return ns;
 }
 
-int64_t prefill_grid(int B, int Hkv, int G, int n_q) {
+int64_t prefill_grid(int64_t nbh, int G, int n_q) {
   const int Mt = kRows / G;
-  return static_cast<int64_t>(B) * Hkv * ((n_q + Mt - 1) / Mt);
+  return nbh * ((n_q + Mt - 1) / Mt);
 }
 
 size_t prefill_workspace_bytes(int B, int Hkv, int64_t T_cap) {
@@ -881,7 +881,7 @@ int launch_prefill_attention(const PrefillArgs &a, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (a.nslots < 2 || a.nslots > kMaxSlots || a.tile_grid < 1 || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8))
     return static_cast<int>(cudaErrorInvalidValue);
-  const int64_t grid = prefill_grid(a.B, a.Hkv, a.G, a.n_q);
+  const int64_t grid = prefill_grid(a.nbh, a.G, a.n_q);
   if (grid < 1 || grid > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidValue);
   int e;
   if (a.two_k && a.two_v) e = launch_tiles_t<true, true>(a, st);

@@ -208,3 +208,28 @@ def test_long_context_chunk_sampled():
                               what="64K chunk row (%d,%d)" % (b, h))
     s = dq.stats_dict(stats)
     assert s["wait_timeouts"] == 0 and s["integrity_errors"] == 0
+
+
+def test_small_workspace_runs_in_waves_identically():
+    # A workspace with room for 3 (b, KV head) rows: 2 x 4 rows run in 3
+    # waves and give the same bits as one wave; below one row is refused.
+    B, Hkv, G, T = 2, 4, 4, 300
+    w, lib, ref_t, kc, vc, rk, rv = _setup(B, Hkv, G, T)
+    T_cap = kc.shape[2]
+    n_q = 64
+    q_start = [T - n_q, 40]
+    qt = torch.from_numpy(synth.q_chunk(w, n_q)).cuda()
+    qs = torch.tensor(q_start, dtype=torch.int32, device="cuda")
+    full = torch.empty(dq.dq_prefill_workspace_bytes(lib, B, Hkv, T_cap), dtype=torch.uint8, device="cuda")
+    row = dq.dq_prefill_workspace_bytes(lib, 1, 1, T_cap)
+    small = torch.empty(3 * row + 100, dtype=torch.uint8, device="cuda")
+    out_a = torch.empty_like(qt)
+    out_b = torch.empty_like(qt)
+    stats = dq.new_stats()
+    dq.dq_prefill_attention(lib, qt, kc, vc, qs, out_a, workspace=full)
+    dq.dq_prefill_attention(lib, qt, kc, vc, qs, out_b, workspace=small, stats=stats)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, out_b)
+    assert dq.stats_dict(stats)["wait_timeouts"] == 0
+    with pytest.raises(dq.DqError):
+        dq.dq_prefill_attention(lib, qt, kc, vc, qs, out_b, workspace=small[:row - 16])
