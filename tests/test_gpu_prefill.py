@@ -95,19 +95,22 @@ def test_single_token_chunk_is_decode_attention():
 
 
 def test_rows_outside_the_cache_are_zero_and_counted():
-    B, Hkv, G, T = 3, 1, 2, 96
+    B, Hkv, G, T = 5, 1, 2, 96
     w, lib, ref_t, kc, vc, rk, rv = _setup(B, Hkv, G, T)
     T_cap = kc.shape[2]
     n_q = 10
-    q_start = [-4, T_cap - 3, 40]  # 4 rows below 0; 7 rows at or past T_cap
+    # 4 rows below 0; 7 rows at or past T_cap; all valid; all past the cache;
+    # all below 0 (whole query blocks with nothing to attend)
+    q_start = [-4, T_cap - 3, 40, T_cap + 5, -1000]
     q = synth.q_chunk(w, n_q)
     stats = dq.new_stats()
     got = _prefill(lib, q, kc, vc, q_start, stats=stats)
     ref = o.attention_prefill_fp64(ref_t, q, _pad(rk, T_cap), _pad(rv, T_cap), q_start)
     assert np.all(got[0, :4] == 0.0) and np.all(got[1, 3:] == 0.0)
+    assert np.all(got[3] == 0.0) and np.all(got[4] == 0.0)
     cm.assert_attention_close(got, ref, what="prefill out-of-range rows")
     s = dq.stats_dict(stats)
-    assert s["clamped_lengths"] == (4 + 7) * G and s["wait_timeouts"] == 0
+    assert s["clamped_lengths"] == (4 + 7 + 10 + 10) * G and s["wait_timeouts"] == 0
 
 
 def test_paged_prefill_equals_contiguous():
