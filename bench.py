@@ -367,22 +367,29 @@ def run_dq(args):
     # ---- chunked prefill over the same cache: the last n_q positions as a
     # chunk of queries (dq_prefill_attention), device-resident inputs ----
     prefill = None
-    if args.prefill_chunk > 0 and page_table is None and L == 1 and T > args.prefill_chunk:
+    if args.prefill_chunk > 0 and L == 1 and T > args.prefill_chunk:
         n_q = args.prefill_chunk
         gq = torch.Generator(device=dev).manual_seed(w.seed)
         qc = torch.randn((w.B, n_q, w.Hq, 128), generator=gq, device=dev).to(w.torch_dtype)
         outc = torch.empty((w.B, n_q, w.Hq, 128), dtype=torch.float32, device=dev)
         qs0 = torch.full((w.B,), T - n_q, dtype=torch.int32, device=dev)
         pws = torch.empty(dq.dq_prefill_workspace_bytes(tab, w.B, w.Hkv, T_cap), dtype=torch.uint8, device=dev)
+
+        def prefill_call():
+            if page_table is None:
+                dq.dq_prefill_attention(tab, qc, kc, vc, qs0, outc, workspace=pws, stats=stats)
+            else:
+                dq.dq_prefill_attention_paged(tab, qc, kc, vc, page_table, qs0, outc, workspace=pws, stats=stats)
+
         for _ in range(3):
-            dq.dq_prefill_attention(tab, qc, kc, vc, qs0, outc, workspace=pws, stats=stats)
+            prefill_call()
         torch.cuda.synchronize()
         barrier()
         p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 5
         p0.record(stream)
         for _ in range(reps):
-            dq.dq_prefill_attention(tab, qc, kc, vc, qs0, outc, workspace=pws, stats=stats)
+            prefill_call()
         p1.record(stream)
         torch.cuda.synchronize()
         barrier()
