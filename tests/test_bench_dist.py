@@ -67,3 +67,17 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     args = type("A", (), {"workload": "tiny_b1_t256", "steps": 1, "warmup": 0})()
     assert bench.run_reference(args) is None
+
+
+def test_prefill_pair_count_and_traffic_gate():
+    # Useful tensor work of a causal chunk: query token i at position
+    # q_start + i sees q_start + i + 1 keys, for every sequence and head.
+    import bench
+    for B, Hq, q_start, n_q in [(1, 1, 0, 1), (2, 4, 10, 7), (16, 32, 7680, 512)]:
+        brute = B * Hq * sum(q_start + i + 1 for i in range(n_q))
+        assert bench.chunk_pairs(B, Hq, q_start, n_q) == brute
+    # DRAM traffic is only reported for the captured workload and source
+    assert bench.prefill_traffic("serve_b32_t8k", 128, 36, 36) is None
+    assert bench.prefill_traffic("qwen3_8b_b16_t8k", 512, 31, 31) is None
+    t = bench.prefill_traffic("qwen3_8b_b16_t8k", 512, 36, 36)
+    assert t is None or abs(t - 737.51e6) < 1e3
