@@ -756,20 +756,30 @@ def run_prefill(args):
     return result
 
 
-def oracle_prefill_row(w, tabs, bh, n_q, ctx):
+def prefill_row_inputs(w, bh, n_q):
+    """The chunk's K, V and queries for one (sequence, KV head) row (host
+    generation, done outside the timed region)."""
+    import numpy as np
+
+    from decode_attention_dq_b200 import synth
+    b, h = bh
+    G = w.Hq // w.Hkv
+    q = np.zeros((1, n_q, w.Hq, 128))
+    q[0, :, h * G:(h + 1) * G] = np.stack([synth.q_rows(w, b, i)[h * G:(h + 1) * G] for i in range(n_q)])
+    return synth.kv_row(w, "k", b, h, n=n_q, step=1), synth.kv_row(w, "v", b, h, n=n_q, step=1), q
+
+
+def oracle_prefill_row(w, tabs, bh, n_q, ctx, inputs):
     """The oracle's prefill step for one (sequence, KV head) row: encode the
     chunk's K and V, then fp64 causal attention of the chunk's queries (the G
     heads of this KV head) over context + chunk."""
     import numpy as np
 
-    from decode_attention_dq_b200 import synth
     from oracle import oracle as o
     b, h = bh
     kc, vc = ctx
+    k_new, v_new, q = inputs
     T = kc.shape[0]
-    G = w.Hq // w.Hkv
-    k_new = synth.kv_row(w, "k", b, h, n=n_q, step=1)
-    v_new = synth.kv_row(w, "v", b, h, n=n_q, step=1)
     hh = np.full(n_q, h, np.int32)
     kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, hh)
     vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, hh)
@@ -779,13 +789,12 @@ def oracle_prefill_row(w, tabs, bh, n_q, ctx):
     vfull[0, h, :T - n_q] = vc[:T - n_q]
     kfull[0, h, T - n_q:] = kk
     vfull[0, h, T - n_q:] = vv
-    q = np.zeros((1, n_q, w.Hq, 128))
-    q[0, :, h * G:(h + 1) * G] = np.stack([synth.q_rows(w, b, i)[h * G:(h + 1) * G] for i in range(n_q)])
     o.attention_prefill_fp64(tabs, q, kfull, vfull, [T - n_q], rows=[(0, h)])
 
 
-def prefill_contexts(w, tabs, n_rows, seconds):
-    """Oracle containers of the context of sampled rows (setup, untimed)."""
+def prefill_contexts(w, tabs, n_rows, seconds, n_q=0):
+    """Oracle containers of the context of sampled rows and, with n_q, the
+    rows' chunk inputs (setup, untimed): [((b, h), (kc, vc), inputs)]."""
     import numpy as np
 
     from decode_attention_dq_b200 import synth
@@ -798,7 +807,7 @@ def prefill_contexts(w, tabs, n_rows, seconds):
         V = synth.kv_row(w, "v", b, h)
         kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
         vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
-        out.append(((b, h), (kc, vc)))
+        out.append(((b, h), (kc, vc), prefill_row_inputs(w, (b, h), n_q) if n_q else None))
         if time.time() - t0 > seconds:
             break
     return out
@@ -812,19 +821,29 @@ def prefill_cpu_baseline(w, n_q, seconds=12.0):
     from oracle import oracle as o
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
                     v_container_bytes=o.container_bytes(w.v_bits))
+    from concurrent.futures import ThreadPoolExecutor
+    ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
     with threadpool_limits(limits=1):
-        ctx = prefill_contexts(w, tabs, 16, seconds / 2)
+        ctx = prefill_contexts(w, tabs, 16, seconds / 2, n_q)
         done = 0
         t0 = time.time()
-        for bh, cc in ctx:
-            oracle_prefill_row(w, tabs, bh, n_q, cc)
+        for bh, cc, inp in ctx:
+            oracle_prefill_row(w, tabs, bh, n_q, cc, inp)
             done += 1
             if time.time() - t0 > seconds / 2:
                 break
         dt = time.time() - t0
+        # All cores: a thread per row (the oracle's C calls and numpy release the GIL).
+        rows = ctx[:max(done, min(len(ctx), ncores))]
+        t1 = time.time()
+        with ThreadPoolExecutor(ncores) as ex:
+            list(ex.map(lambda p: oracle_prefill_row(w, tabs, p[0], n_q, p[1], p[2]), rows))
+        dt_all = time.time() - t1
     return {"value": done * n_q / w.Hkv / dt, "unit": PREFILL_UNIT, "cores": 1, "kind": "oracle",
             "sample": "%d (sequence, KV head) rows of %s: encode a %d-token chunk + fp64 causal attention of "
-                      "its queries over %d tokens, one thread, %.1f s" % (done, w.name, n_q, w.T, dt)}
+                      "its queries over %d tokens, one thread, %.1f s" % (done, w.name, n_q, w.T, dt),
+            "all_cores": {"value": len(rows) * n_q / w.Hkv / dt_all, "unit": PREFILL_UNIT, "cores": ncores,
+                          "sample": "%d rows, one thread per row, %.1f s" % (len(rows), dt_all)}}
 
 
 def run_reference_prefill(args, w):
@@ -837,12 +856,12 @@ def run_reference_prefill(args, w):
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
                     v_container_bytes=o.container_bytes(w.v_bits))
     with threadpool_limits(limits=1):
-        ctx = prefill_contexts(w, tabs, args.warmup + args.steps, 1e9)
+        ctx = prefill_contexts(w, tabs, args.warmup + args.steps, 1e9, n_q)
         for i in range(args.warmup):
-            oracle_prefill_row(w, tabs, ctx[i][0], n_q, ctx[i][1])
+            oracle_prefill_row(w, tabs, ctx[i][0], n_q, ctx[i][1], ctx[i][2])
         t0 = time.time()
         for i in range(args.warmup, args.warmup + args.steps):
-            oracle_prefill_row(w, tabs, ctx[i][0], n_q, ctx[i][1])
+            oracle_prefill_row(w, tabs, ctx[i][0], n_q, ctx[i][1], ctx[i][2])
         dt = time.time() - t0
     value = args.steps * n_q / w.Hkv / dt
     sample = ("per step: one (sequence, KV head) row of %s, encode a %d-token chunk + fp64 causal attention "
