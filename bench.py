@@ -57,13 +57,13 @@ ENCODE_OPS_PER_VECTOR = 2560
 LAUNCHES_PER_STEP = 4
 # DRAM traffic of decode_split_kernel from one ncu capture (dram__bytes_read
 # + dram__bytes_write) of the 32-sequence, 8192-token workload with 36-byte
-# containers: 151.44 MB + 6.80 MB per launch over 32*8*8192 token-heads. It
+# containers: 151.37 MB + 3.62 MB per launch over 32*8*8192 token-heads. It
 # scales with the token-heads a launch processes (reads are the containers,
 # writes the partial states). It belongs to one version of the kernel source:
 # for any other, or other container sizes, traffic is reported as null.
 DECODE_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_decode.cu",
-                  "sha256_16": "6d0be282ac859e1f", "ck": 36, "cv": 36,
-                  "bytes_per_token_head": (151.442944e6 + 6.804992e6) / (32 * 8 * 8192)}
+                  "sha256_16": "36f00627cfa3f944", "ck": 36, "cv": 36,
+                  "bytes_per_token_head": (151.368192e6 + 3.621888e6) / (32 * 8 * 8192)}
 
 
 def decode_traffic(token_heads, ck, cv):
@@ -590,9 +590,9 @@ PREFILL_LAUNCHES_PER_STEP = 4
 # pass) of `bench.py --prefill 512 --workload qwen3_8b_b16_t8k`: the decoded
 # tiles read once (545 MB) plus the queries, and the fp32 output. Reported
 # only for that workload and container size while the kernel source matches.
-PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "89b08ba04686d927",
+PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "a915fc4568df19d4",
                    "workload": "qwen3_8b_b16_t8k", "chunk": 512, "ck": 36, "cv": 36,
-                   "bytes": 617.62e6 + 119.89e6}
+                   "bytes": 616.17e6 + 118.29e6}
 
 
 def prefill_traffic(workload, n_q, ck, cv):

@@ -286,7 +286,7 @@ __device__ __forceinline__ RansLane rans_open(const uint8_t *smem, uint32_t off)
 }
 
 // One decode step (table entry: bits 0..10 slot - c_s, 11..13 s, 20..31 f_s):
-// x = f (x >> 12) + slot - c_s, then arithmetic byte renormalisation (one
+// x = f (x >> 12) + slot - c_s, then byte renormalisation by selects (one
 // byte, or two for tables with a symbol of f < 16). Returns 4 s.
 template <bool kTwo>
 __device__ __forceinline__ uint32_t rans_step(RansLane &r, const uint32_t *lut, const uint8_t *smem) {
@@ -294,15 +294,16 @@ __device__ __forceinline__ uint32_t rans_step(RansLane &r, const uint32_t *lut, 
   uint32_t x = (e >> 20) * (r.x >> kProbBits) + (e & 0x7FFu);
   const uint32_t b0 = smem[r.p];
   const uint32_t b1 = kTwo ? static_cast<uint32_t>(smem[r.p + kGrp]) : 0u;
-  const uint32_t n0 = __umulhi(x - kL, 2u);
-  x += n0 * (x * 255u + b0);
-  uint32_t adv = n0;
+  uint32_t p = r.p;
+  const bool lo0 = x < kL;
+  x = lo0 ? (x * 256u + b0) : x;
+  p = lo0 ? p + kGrp : p;
   if constexpr (kTwo) {
-    const uint32_t n1 = __umulhi(x - kL, 2u);
-    x += n1 * (x * 255u + b1);
-    adv += n1;
+    const bool lo1 = x < kL;
+    x = lo1 ? (x * 256u + b1) : x;
+    p = lo1 ? p + kGrp : p;
   }
-  r.p += adv * kGrp;
+  r.p = p;
   r.x = x;
   return (e >> 9) & 0x1Cu;
 }
