@@ -3,7 +3,8 @@
 The page fixes two hard properties ([news] "Drift: Bending Variable Back to
 Fixed"): a drifted symbol moves to a nearby lower-cost symbol, and no symbol
 moves by more than one reconstruction level; the result fits the container.
-The greedy ranking is this build's reading; it is pinned here against an
+The greedy ranking (least added squared error per bit saved, ties to the
+lowest index) is a reading where the page is silent; it is pinned here against an
 independent restatement that sorts every candidate move once and applies them
 in order (the same rule, written as a sort rather than a repeated arg-min),
 which checks the procedure and its tie order on small strings.
