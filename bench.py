@@ -205,7 +205,8 @@ def run_dq(args):
     w = replica_workload(synth.WORKLOADS[args.workload], rank)
     dev = torch.device("cuda", torch.cuda.current_device())
     tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits,
-                             drift_mode=args.drift_mode)
+                             drift_mode=args.drift_mode, k_rate_offset=args.k_rate_offset,
+                             v_rate_offset=args.v_rate_offset)
     ck, cv = tab.k.container_bytes, tab.v.container_bytes
     T = w.T
     T_cap = (T + 31) // 32 * 32
@@ -425,6 +426,7 @@ def run_dq(args):
                        "l2": "inputs larger than L2 (%.0f MB of containers read per step)" % (comp_bytes / 1e6),
                        "cache": "paged: 32-token pages in a shuffled order" if args.paged else "contiguous",
                        "drift_mode": args.drift_mode,
+                       "rate_offsets": [args.k_rate_offset, args.v_rate_offset],
                        "layers": L,
                        "parallelism": "replicas x%d" % ws},
             "hbm_gbs": hbm_gbs,
@@ -465,7 +467,8 @@ def run_dq(args):
                         "graph_tokens_per_s": None if graph_ms is None else whole_job_rate(w.B, ws, graph_ms)},
         }
         if ws == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(w, tab_seed=0, seconds=args.cpu_seconds)
+            result["cpu_baseline"] = cpu_baseline(w, tab_seed=0, seconds=args.cpu_seconds,
+                                                  rate_offsets=(args.k_rate_offset, args.v_rate_offset))
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -516,7 +519,7 @@ def oracle_sample_step(w, tabs, rows, cache_rows):
         o.attention_fp64(tabs, qb, kfull, vfull, [kc.shape[0]], rows=[(0, h)])
 
 
-def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512):
+def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0.0)):
     """The oracle, as it stands, on the host: a bounded sample of the step,
     once on one thread (BLAS limited to one thread too) and once on all host
     cores (a thread per (sequence, KV head) row; the oracle's C calls and
@@ -530,7 +533,8 @@ def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512):
     from oracle import oracle as o
 
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
-                    v_container_bytes=o.container_bytes(w.v_bits), sign_seed=tab_seed)
+                    v_container_bytes=o.container_bytes(w.v_bits), sign_seed=tab_seed,
+                    k_rate_offset=rate_offsets[0], v_rate_offset=rate_offsets[1])
     ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
     with threadpool_limits(limits=1):
         # Containers for sampled rows, encoded by the oracle (setup, untimed).
@@ -934,6 +938,10 @@ def main():
     ap.add_argument("--graph", action="store_true", help="also time the step captured as a CUDA graph")
     ap.add_argument("--prefill-chunk", type=int, default=512, metavar="N_Q",
                     help="also time chunked prefill of the last N_Q positions over the decode cache (0: off)")
+    ap.add_argument("--k-rate-offset", type=float, default=0.0,
+                    help="K table target rate above the container's nominal rate (bit/value)")
+    ap.add_argument("--v-rate-offset", type=float, default=0.0,
+                    help="V table target rate above the container's nominal rate (bit/value)")
     ap.add_argument("--drift-mode", type=int, default=0, choices=[0, 1],
                     help="0: drift only (default); 1: drift, then the rate-distortion fill")
     ap.add_argument("--prefill", type=int, default=0, metavar="N_Q",
