@@ -30,10 +30,10 @@
 //     arithmetic), ranks the candidate moves by repeated arg-min (least key
 //     first, ties to the lower index), and lane m encodes the string with the
 //     first m+1 moves applied; the smallest m that fits is the greedy result.
-//     The first pass tries 8 move counts (32 in the warp-per-vector
-//     kernel), later ones 32. The separate drift kernel ranks 8 moves for
-//     each of 4 containers and tries all 32 (container, count) pairs in one
-//     encode pass.
+//     The warp-per-vector kernel tries 32 move counts per pass. The separate
+//     drift kernel (lane-per-vector appends) keeps 8 containers per warp in
+//     flight and tries 4 move counts of each per encode pass, ranking 4 more
+//     moves of a container only when its window had no fit.
 #include "dq_device.cuh"
 
 namespace dqi {
@@ -254,11 +254,11 @@ __device__ __forceinline__ int encode_bf(SymFn sym, const EncSym *es, uint8_t *s
 
 // Phase-1 arithmetic for one vector spread over the warp (coordinate
 // lane + 32 k in u[k]): same operations, same order, so the same u, symbols
-// and norm as lane_prepare. Writes the symbols to q[]; returns the fp16 norm
-// and whether the vector was non-finite.
-__device__ __forceinline__ void warp_prepare(const AppendArgs &a, const void *src, int64_t v, int h,
-                                             const float (&t)[7], int lane, float (&u)[4], uint8_t *q,
-                                             uint16_t *n16_out, bool *nf_out) {
+// and norm as lane_prepare. Returns the symbols of this lane's coordinates in
+// qk[], the fp16 norm and whether the vector was non-finite.
+__device__ __forceinline__ void warp_prepare_regs(const AppendArgs &a, const void *src, int64_t v, int h,
+                                                  const float (&t)[7], int lane, float (&u)[4], uint32_t (&qk)[4],
+                                                  uint16_t *n16_out, bool *nf_out) {
   float z[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k)
@@ -282,10 +282,20 @@ __device__ __forceinline__ void warp_prepare(const AppendArgs &a, const void *sr
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     u[k] = nf ? 0.0f : __fmul_rn(z[k], sigma);
-    q[lane + 32 * k] = static_cast<uint8_t>(quantize7(u[k], t));
+    qk[k] = quantize7(u[k], t);
   }
   *n16_out = n16;
   *nf_out = nf;
+}
+
+// warp_prepare_regs with the symbols written to q[lane + 32 k].
+__device__ __forceinline__ void warp_prepare(const AppendArgs &a, const void *src, int64_t v, int h,
+                                             const float (&t)[7], int lane, float (&u)[4], uint8_t *q,
+                                             uint16_t *n16_out, bool *nf_out) {
+  uint32_t qk[4];
+  warp_prepare_regs(a, src, v, h, t, lane, u, qk, n16_out, nf_out);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) q[lane + 32 * k] = static_cast<uint8_t>(qk[k]);
 }
 
 // Where the vectors of one append call come from and go to (one stream).
@@ -325,9 +335,9 @@ struct StreamCtx {
   }
 };
 
-// Copies one stream's tables into shared memory (threads 0..7) and fills the
-// stream context. Callers synchronise before using T.
-__device__ __forceinline__ StreamCtx stream_setup(const AppendArgs &a, AppendTables &T, bool is_v) {
+// Copies one stream's tables into shared memory (the threads with filler
+// index 0..7) and fills the stream context. Callers synchronise before using T.
+__device__ __forceinline__ StreamCtx stream_setup(const AppendArgs &a, AppendTables &T, bool is_v, int filler) {
   const DevStream &tab = is_v ? a.tabs->v : a.tabs->k;
   StreamCtx c;
   c.nl = is_v ? a.nv : a.nk;
@@ -337,8 +347,8 @@ __device__ __forceinline__ StreamCtx stream_setup(const AppendArgs &a, AppendTab
   c.cache = is_v ? a.vcache : a.kcache;
   c.per_seq = static_cast<int64_t>(a.Hkv) * a.n_new;
   c.nvec = static_cast<int64_t>(a.B) * c.per_seq;
-  if (threadIdx.x < kMaxLevels) {
-    const int s = threadIdx.x;
+  if (filler < kMaxLevels) {
+    const int s = filler;
     T.lev[s] = tab.levels[s];
     T.thr[s] = (s < c.nl - 1) ? tab.thresholds[s] : INFINITY;
     T.cost[s] = tab.cost[s];
@@ -576,7 +586,7 @@ __device__ __forceinline__ void add_stats(const AppendArgs &a, bool is_v, const 
 template <bool kBF16, bool kTwo>
 __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, WarpArea &W, bool is_v) {
   const int lane = threadIdx.x & 31;
-  const StreamCtx c = stream_setup(a, T, is_v);
+  const StreamCtx c = stream_setup(a, T, is_v, static_cast<int>(threadIdx.x));
   __syncthreads();
   const int64_t v0 = (static_cast<int64_t>(blockIdx.x) * kAW + (threadIdx.x >> 5)) * 32;
   if (v0 >= c.nvec) return;
@@ -645,7 +655,7 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
 template <bool kTwo>
 __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, WarpArea &W, bool is_v) {
   const int lane = threadIdx.x & 31;
-  const StreamCtx c = stream_setup(a, T, is_v);
+  const StreamCtx c = stream_setup(a, T, is_v, static_cast<int>(threadIdx.x));
   __syncthreads();
   const int64_t v = static_cast<int64_t>(blockIdx.x) * kAW + (threadIdx.x >> 5);
   if (v >= c.nvec) return;
@@ -684,153 +694,195 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   if (lane == 0) add_stats(a, is_v, dc, nf ? 1u : 0u, dropped ? 1u : 0u, bad_page ? 1u : 0u);
 }
 
-// Drift kernel scratch: kBatch containers per warp are prepared and ranked,
-// then their first kFirst candidate move counts are tried in one encode
-// pass (lane 8 c + k tries container c with moves 0..k).
-constexpr int kBatch = 4;
-constexpr int kFirst = 8;
-static_assert(kBatch * kFirst == 32, "one trial per lane");
+// Drift kernel: each warp keeps kSlots listed containers in flight. One
+// encode pass tries kWin consecutive move counts of every one of them (lane
+// kWin c + j: container c with its ranked moves 0 .. win_c + j applied); the
+// first count that fits is the greedy result, the container is stored and
+// its slot takes the next list entry. A container with no fitting count in
+// its window ranks kWin more moves (the keys of the moves not yet ranked stay
+// in shared memory) and is tried again in the next pass; one whose candidates
+// run out tries the fallback string on the last lane of its window.
+constexpr int kSlots = 8;
+constexpr int kWin = 4;
+static_assert(kSlots * kWin == 32, "one trial per lane");
+constexpr int kDriftWarps = 4;  // warps per drift CTA
 
 struct DriftArea {
   uint8_t stack[kStackSlots * 32];
-  uint8_t q[kBatch][kD], rank[kBatch][kD], tgt[kBatch][kD];
-  int64_t vd[kBatch];
-  int32_t added[kBatch];
-  uint16_t n16[kBatch];
+  uint32_t sw[kD][kSlots];   // symbol i of slot c: q | tgt << 8 | rank << 16 (kNoRank: not ranked)
+  float key[kSlots][4][32];  // key of the move of symbol l + 32 k, +inf once ranked or without a candidate
+  int64_t vd[kSlots];
+  int32_t ranked[kSlots], win[kSlots];
+  uint16_t n16[kSlots];
+  AppendTables T;
 };
 
-// Ranks up to kFirst best moves of one container (u: this lane's coordinates,
-// q: symbols) into rank[] / tgt[] (repeated warp arg-min over (key, index),
-// as in drift_one). Returns how many were ranked.
-__device__ __forceinline__ int rank_first(const AppendTables &T, int nl, const float (&u)[4], const uint8_t *q,
-                                          uint8_t *rank, uint8_t *tgt, int lane) {
-  float key[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int i = lane + 32 * k;
-    int tj;
-    key[k] = best_move(T, nl, q[i], u[k], &tj);
-    rank[i] = kNoRank;
-    tgt[i] = static_cast<uint8_t>(tj);
-  }
-  __syncwarp();
-  int added = 0;
-  for (; added < kFirst; ++added) {
-    float bk = key[0];
-    int bi = lane;
-#pragma unroll
-    for (int k = 1; k < 4; ++k)
-      if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ok = __shfl_xor_sync(kFull, bk, off);
-      const int oi = __shfl_xor_sync(kFull, bi, off);
-      if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-    }
-    if (bk == INFINITY) break;  // no candidate left
-    if ((bi & 31) == lane) {
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (bi == lane + 32 * k) key[k] = INFINITY;
-      rank[bi] = static_cast<uint8_t>(added);
-    }
-  }
-  __syncwarp();
-  return added;
-}
-
-// E6 for the containers listed by the lane-per-vector kernel: each warp of
-// a persistent grid takes kBatch list entries at a time. A container whose
-// first kFirst moves are not enough goes through drift_one.
+// E6 for one stream's drift list: entries first, first + stride, ... .
 template <bool kTwo>
-__device__ __forceinline__ void drift_body(const AppendArgs &a, AppendTables &T, DriftArea &A, bool is_v) {
-  const int lane = threadIdx.x & 31;
-  const StreamCtx c = stream_setup(a, T, is_v);
-  __syncthreads();
+__device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, bool is_v, int lane, uint32_t first,
+                                             uint32_t stride, DriftCount &dc) {
+  __syncwarp();
+  const StreamCtx c = stream_setup(a, A.T, is_v, lane);
+  if (lane < kSlots) {
+    A.ranked[lane] = 0;
+    A.win[lane] = 0;
+  }
+  __syncwarp();
   const uint32_t n = a.drift_count[is_v ? 1 : 0];
   const uint32_t *list = a.drift_list + (is_v ? a.list_cap : 0);
-  const uint32_t stride = gridDim.x * kAW * kBatch;
   uint8_t *stk = A.stack + lane;
-  DriftCount dc;
-  for (uint32_t base = (blockIdx.x * kAW + (threadIdx.x >> 5)) * kBatch; base < n; base += stride) {
-    const int nb = (n - base) < static_cast<uint32_t>(kBatch) ? static_cast<int>(n - base) : kBatch;
-    // Loops over the batch stay rolled: the kernel's code has to fit the
-    // instruction caches shared by its warps.
+  const int cs = lane / kWin, jw = lane % kWin;
+  const uint32_t hlf = static_cast<uint32_t>(c.nl / 2);
+  uint64_t cursor = first;
+  uint32_t live = 0, exh = 0;  // warp-uniform slot masks: holds a container; candidates ran out
+  for (;;) {
+    // Free slots take the next list entries: symbols, move targets and keys.
 #pragma unroll 1
-    for (int cb = 0; cb < nb; ++cb) {
-      const int64_t v = list[base + cb];
+    for (int s = 0; s < kSlots && cursor < n; ++s) {
+      if ((live >> s) & 1u) continue;
+      const int64_t v = list[cursor];
+      cursor += stride;
       float u[4];
+      uint32_t qk[4];
       uint16_t n16v;
       bool nf;
-      warp_prepare(a, c.src, v, c.head_of(a, v), c.t, lane, u, A.q[cb], &n16v, &nf);
-      __syncwarp();
-      const int ad = rank_first(T, c.nl, u, A.q[cb], A.rank[cb], A.tgt[cb], lane);
+      warp_prepare_regs(a, c.src, v, c.head_of(a, v), c.t, lane, u, qk, &n16v, &nf);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        int tj;
+        A.key[s][k][lane] = best_move(A.T, c.nl, static_cast<int>(qk[k]), u[k], &tj);
+        A.sw[lane + 32 * k][s] = qk[k] | (static_cast<uint32_t>(tj) << 8) | (static_cast<uint32_t>(kNoRank) << 16);
+      }
       if (lane == 0) {
-        A.vd[cb] = v;
-        A.n16[cb] = n16v;
-        A.added[cb] = ad;
+        A.vd[s] = v;
+        A.n16[s] = n16v;
+        A.ranked[s] = 0;
+        A.win[s] = 0;
       }
+      live |= 1u << s;
+      exh &= ~(1u << s);
+    }
+    if (!live) break;
+    __syncwarp();
+    // Every live slot with candidates left ranks its moves up to win + kWin
+    // by repeated arg-min over (key, index).
+#pragma unroll 1
+    for (int s = 0; s < kSlots; ++s) {
+      if (!(((live & ~exh) >> s) & 1u)) continue;
+      int r = A.ranked[s];
+      const int target = A.win[s] + kWin;
+      if (r >= target) continue;
+      float key[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) key[k] = A.key[s][k][lane];
+      for (; r < target; ++r) {
+        float bk = key[0];
+        int bi = lane;
+#pragma unroll
+        for (int k = 1; k < 4; ++k)
+          if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+          const float ok = __shfl_xor_sync(kFull, bk, off);
+          const int oi = __shfl_xor_sync(kFull, bi, off);
+          if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
+        }
+        if (bk == INFINITY) {
+          exh |= 1u << s;
+          break;
+        }
+        if ((bi & 31) == lane) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            if (bi == lane + 32 * k) key[k] = INFINITY;
+          A.sw[bi][s] = (A.sw[bi][s] & 0xFFFFu) | (static_cast<uint32_t>(r) << 16);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) A.key[s][k][lane] = key[k];
+      if (lane == 0) A.ranked[s] = r;
     }
     __syncwarp();
-    // Lane 8 cb + k encodes container cb with its moves 0..k applied.
-    const int cm = (lane / kFirst) < nb ? lane / kFirst : 0, km = lane % kFirst;
-    const uint8_t *q = A.q[cm], *rk = A.rank[cm], *tg = A.tgt[cm];
+    // One encode pass. An exhausted slot has ranked < win + kWin, so the last
+    // lane of its window is free for the fallback string (all ranked moves,
+    // then every symbol to the innermost level of its side).
+    const bool mine = (live >> cs) & 1u;
+    // A lane whose slot is empty encodes a live slot's string (its words
+    // were all written at refill, every symbol below nl); its result is
+    // not used.
+    const uint32_t *swc = &A.sw[0][mine ? cs : __ffs(live) - 1];
+    const int win = A.win[cs], ranked = A.ranked[cs];
+    const int km = win + jw;
+    const bool trial = mine && km < ranked;
+    const bool fb = mine && ((exh >> cs) & 1u) && jw == kWin - 1;
     uint32_t x = 0;
-    const int len = encode_bf<kTwo, false>(
-        [&](int i) {
-          const uint32_t r = rk[i];
-          return (r != kNoRank && static_cast<int>(r) <= km) ? static_cast<uint32_t>(tg[i]) : static_cast<uint32_t>(q[i]);
-        },
-        T.es, stk, &x);
-    const unsigned fit =
-        __ballot_sync(kFull, lane / kFirst < nb && km < A.added[cm] && len <= c.P);
-    // The first fitting lane of each container stores it.
-    {
-      const int cb = lane / kFirst;
-      const unsigned fc = (fit >> (kFirst * cb)) & ((1u << kFirst) - 1u);
-      if (cb < nb && fc && km == __ffs(fc) - 1) {
-        bool dr = false;
-        uint8_t *dst = c.dst_of(a, A.vd[cb], &dr);
-        if (dst) store_container(dst, c.C, A.n16[cb], x, stk, len);
-      }
+    int len;
+    if (__any_sync(kFull, fb)) {
+      const uint32_t kmx = fb ? 254u : static_cast<uint32_t>(km);
+      len = encode_bf<kTwo, false>(
+          [&](int i) {
+            const uint32_t w = swc[i * kSlots];
+            uint32_t sy = ((w >> 16) <= kmx) ? ((w >> 8) & 0xFFu) : (w & 0xFFu);
+            if (fb) sy = sy >= hlf ? hlf : hlf - 1u;
+            return sy;
+          },
+          A.T.es, stk, &x);
+    } else {
+      const uint32_t kmx = static_cast<uint32_t>(km);
+      len = encode_bf<kTwo, false>(
+          [&](int i) {
+            const uint32_t w = swc[i * kSlots];
+            return ((w >> 16) <= kmx) ? ((w >> 8) & 0xFFu) : (w & 0xFFu);
+          },
+          A.T.es, stk, &x);
     }
+    const bool ok = len <= c.P;
+    const unsigned fit = __ballot_sync(kFull, trial && ok);
+    const unsigned fc = (fit >> (kWin * cs)) & ((1u << kWin) - 1u);
+    const bool store = fc ? (jw == __ffs(fc) - 1) : (fb && ok);
+    if (store) {
+      bool dr = false;
+      uint8_t *dst = c.dst_of(a, A.vd[cs], &dr);
+      if (dst) store_container(dst, c.C, A.n16[cs], x, stk, len);
+    }
+    // Slot bookkeeping (warp-uniform).
 #pragma unroll 1
-    for (int cb = 0; cb < nb; ++cb) {
-      const unsigned fc = (fit >> (kFirst * cb)) & ((1u << kFirst) - 1u);
-      if (fc) {
-        dc.moves += static_cast<unsigned>(__ffs(fc));
+    for (int s = 0; s < kSlots; ++s) {
+      if (!((live >> s) & 1u)) continue;
+      const unsigned f = (fit >> (kWin * s)) & ((1u << kWin) - 1u);
+      if (f) {
+        dc.moves += static_cast<unsigned>(A.win[s] + __ffs(f));
         dc.containers += 1;
+        live &= ~(1u << s);
+      } else if ((exh >> s) & 1u) {
+        const int r = A.ranked[s];
+        dc.fallbacks += 1;
+        dc.moves += static_cast<unsigned>(r);
+        dc.containers += r > 0 ? 1u : 0u;
+        live &= ~(1u << s);
       }
     }
     __syncwarp();
-    // Containers that need more moves (or run out of candidates): the full
-    // greedy search, which ranks its moves again from the first.
-#pragma unroll 1
-    for (int cb = 0; cb < nb; ++cb) {
-      if ((fit >> (kFirst * cb)) & ((1u << kFirst) - 1u)) continue;
-      const int64_t v = A.vd[cb];
-      float u[4];
-      uint16_t n16v;
-      bool nf;
-      warp_prepare(a, c.src, v, c.head_of(a, v), c.t, lane, u, A.q[0], &n16v, &nf);
-      __syncwarp();
-      drift_one<kTwo>(a, c, T, A.stack, A.q[0], A.rank[0], A.tgt[0], v, n16v, u, lane, 32, dc);
-    }
+    if (lane < kSlots && ((live >> lane) & 1u)) A.win[lane] += kWin;
+    __syncwarp();
   }
-  if (lane == 0) add_stats(a, is_v, dc, 0u, 0u);
 }
 
+// Every warp walks its share of the K list, then of the V list, so the two
+// streams' lists (often of very different lengths) spread over all warps.
 template <bool kTwoK, bool kTwoV>
-__global__ void __launch_bounds__(kAW * 32) append_drift_kernel(const AppendArgs a) {
-  __shared__ AppendTables T;
-  __shared__ DriftArea A[kAW];
-  const bool is_v = blockIdx.y == 1;
+__global__ void __launch_bounds__(kDriftWarps * 32) append_drift_kernel(const AppendArgs a) {
+  __shared__ DriftArea A[kDriftWarps];
+  const int lane = threadIdx.x & 31;
   DriftArea &w = A[threadIdx.x >> 5];
-  if constexpr (kTwoK == kTwoV) {
-    drift_body<kTwoK>(a, T, w, is_v);
-  } else {
-    if (is_v) drift_body<kTwoV>(a, T, w, true);
-    else drift_body<kTwoK>(a, T, w, false);
+  const uint32_t first = blockIdx.x * kDriftWarps + (threadIdx.x >> 5);
+  const uint32_t stride = gridDim.x * kDriftWarps;
+  DriftCount dk, dv;
+  drift_stream<kTwoK>(a, w, false, lane, first, stride, dk);
+  drift_stream<kTwoV>(a, w, true, lane, first, stride, dv);
+  if (lane == 0) {
+    add_stats(a, false, dk, 0u, 0u);
+    add_stats(a, true, dv, 0u, 0u);
   }
 }
 
@@ -880,8 +932,16 @@ int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, int sms, cudaStrea
   append_lane_kernel<kBF16, kTwoK, kTwoV><<<grid, kAW * 32, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.drift_list) return static_cast<int>(e);
-  // Drift: a persistent grid of 4 CTAs per SM and stream walks the lists.
-  append_drift_kernel<kTwoK, kTwoV><<<dim3(static_cast<unsigned>(4 * sms), 2), kAW * 32, 0, st>>>(a);
+  // Drift: a persistent grid, as many CTAs as fit on the SMs at once.
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV>, kDriftWarps * 32, 0) !=
+            cudaSuccess || n < 1)
+      n = 1;
+    per_sm = n;
+  }
+  append_drift_kernel<kTwoK, kTwoV><<<static_cast<unsigned>(per_sm * sms), kDriftWarps * 32, 0, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 
