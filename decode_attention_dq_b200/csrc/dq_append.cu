@@ -14,13 +14,14 @@
 // __fmul_rn, __fdiv_rn, __fsqrt_rn) so no multiply-add is contracted: the
 // containers are bit-identical to the format's definition.
 //
-// Work split: one warp takes 32 consecutive vectors of one stream, one per lane.
-//   phase 1 (lane per vector, all in registers): E1 sign flip, E2 Walsh-
-//     Hadamard transform (the seven butterfly stages in order), E3 norm in
-//     the fixed tree (the 32 partial sums of four squares, then pairwise
+// Work split: one warp takes 32 consecutive vectors of one stream.
+//   phase 1 (four lanes per vector, 32 coordinates each in registers, four
+//     passes of 8 vectors): E1 sign flip, E2 Walsh-Hadamard transform (the
+//     seven butterfly stages in order, two of them between lanes), E3 norm
+//     in the fixed tree (the 32 partial sums of four squares, then pairwise
 //     over offsets 16, 8, 4, 2, 1), scale, fp16 norm, E4 quantisation by a
 //     three-step search over the sorted thresholds; symbols packed 4 per
-//     register.
+//     word in shared memory.
 //   phase 2 (lane per vector): E5 rANS encode last-to-first without branches
 //     (a renormalisation push is written every step and kept only when
 //     needed; the division by f is an exact multiply-shift); containers that
@@ -67,6 +68,8 @@ struct WarpArea {
   uint8_t stack[kStackSlots * 32];
   uint32_t syms[kD / 4][32];
   uint8_t q[kD], rank[kD], tgt[kD];
+  uint16_t n16[32];  // fp16 norm of the warp's vector l (lane-per-vector kernel)
+  uint8_t nf[32];    // vector l was non-finite
 };
 
 // Writes one container; byte k goes to dst[32 k] (the cache interleaves the
@@ -122,92 +125,6 @@ __device__ __forceinline__ uint32_t quantize7(float u, const float (&t)[7]) {
 // Sign word bit `b` moved to the float sign position.
 __device__ __forceinline__ uint32_t sign_bit(uint32_t word, int b) { return (word << (31 - b)) & 0x80000000u; }
 
-// Phase 1 for the vector of this lane: loads, signs, WHT, norm, scale and
-// quantisation, all in registers. Writes the packed symbols (byte i % 4 of
-// pk[i / 4] = symbol i), the fp16 norm and whether the vector was
-// non-finite (then it is encoded as the zero vector).
-template <bool kBF16>
-__device__ __forceinline__ void lane_prepare(const void *src, int64_t v, const uint32_t (&sw)[4],
-                                             const float (&t)[7], uint32_t (&pk)[32], uint16_t *n16_out,
-                                             bool *nf_out) {
-  float z[kD];
-  if constexpr (kBF16) {
-    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(src) + v * kD);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint4 w = __ldg(p + c);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 8 * c + 2 * e;
-        z[i] = __uint_as_float((ww[e] << 16) ^ sign_bit(sw[i >> 5], i & 31));
-        z[i + 1] = __uint_as_float((ww[e] & 0xFFFF0000u) ^ sign_bit(sw[(i + 1) >> 5], (i + 1) & 31));
-      }
-    }
-  } else {
-    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const float *>(src) + v * kD);
-#pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const uint4 w = __ldg(p + c);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * c + e;
-        z[i] = __uint_as_float(ww[e] ^ sign_bit(sw[i >> 5], i & 31));
-      }
-    }
-  }
-  // E2: stages h = 1, 2, ..., 64; (a, b) -> (a + b, a - b) on the pairs
-  // (j, j + h) with bit h of j clear.
-#pragma unroll
-  for (int st = 0; st < 7; ++st) {
-    const int h = 1 << st;
-#pragma unroll
-    for (int pr = 0; pr < kD / 2; ++pr) {
-      const int j = ((pr >> st) << (st + 1)) | (pr & (h - 1));
-      const float a0 = z[j], b0 = z[j + h];
-      z[j] = __fadd_rn(a0, b0);
-      z[j + h] = __fsub_rn(a0, b0);
-    }
-  }
-  // E3: p_l = (z_l^2 + z_{l+32}^2) + (z_{l+64}^2 + z_{l+96}^2), then the
-  // pairwise tree over offsets 16, 8, 4, 2, 1.
-  float p[32];
-#pragma unroll
-  for (int l = 0; l < 32; ++l)
-    p[l] = __fadd_rn(__fadd_rn(__fmul_rn(z[l], z[l]), __fmul_rn(z[l + 32], z[l + 32])),
-                     __fadd_rn(__fmul_rn(z[l + 64], z[l + 64]), __fmul_rn(z[l + 96], z[l + 96])));
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1)
-#pragma unroll
-    for (int l = 0; l < o; ++l) p[l] = __fadd_rn(p[l], p[l + o]);
-  const float ss = p[0];
-  bool nf = !isfinite(ss);
-  uint16_t n16 = 0;
-  float sigma = 0.0f;
-  if (!nf) {
-    const float r = __fsqrt_rn(ss);
-    sigma = (r == 0.0f) ? 0.0f : __fdiv_rn(kSqrtD, r);
-    if (!(r != 0.0f && isfinite(sigma))) sigma = 0.0f;
-    float nv = __fdiv_rn(r, kSqrtD);
-    if (nv > 65504.0f) nv = 65504.0f;
-    n16 = __half_as_ushort(__float2half_rn(nv));
-  }
-  // E4 (u = 0 for the zero and the non-finite vector).
-#pragma unroll
-  for (int w = 0; w < 32; ++w) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float u = nf ? 0.0f : __fmul_rn(z[4 * w + e], sigma);
-      word |= quantize7(u, t) << (8 * e);
-    }
-    pk[w] = word;
-  }
-  *n16_out = n16;
-  *nf_out = nf;
-}
-
 // E5 without branches: rANS-encode 128 symbols (sym(i) gives symbol i),
 // coded 127 -> 0 from x = 2^16. A renormalisation push writes the low byte of
 // x to the lane's stack every step and keeps it only when x >= 4096 f; pushes
@@ -254,7 +171,7 @@ __device__ __forceinline__ int encode_bf(SymFn sym, const EncSym *es, uint8_t *s
 
 // Phase-1 arithmetic for one vector spread over the warp (coordinate
 // lane + 32 k in u[k]): same operations, same order, so the same u, symbols
-// and norm as lane_prepare. Returns the symbols of this lane's coordinates in
+// and norm as quad_prepare. Returns the symbols of this lane's coordinates in
 // qk[], the fp16 norm and whether the vector was non-finite.
 __device__ __forceinline__ void warp_prepare_regs(const AppendArgs &a, const void *src, int64_t v, int h,
                                                   const float (&t)[7], int lane, float (&u)[4], uint32_t (&qk)[4],
@@ -369,6 +286,164 @@ __device__ __forceinline__ StreamCtx stream_setup(const AppendArgs &a, AppendTab
 #pragma unroll
   for (int j = 0; j < 7; ++j) c.t[j] = (j < c.nl - 1) ? tab.thresholds[j] : INFINITY;
   return c;
+}
+
+// Norm and scale from the sum of squares ss (E3): sigma = sqrt(128) / r with
+// r = sqrt(ss) (0 for the zero vector), the fp16 norm r / sqrt(128)
+// (clamped to the largest finite half), and whether the vector is
+// non-finite (then u = 0 and the norm is 0).
+__device__ __forceinline__ void norm_scale(float ss, float *sigma_out, uint16_t *n16_out, bool *nf_out) {
+  const bool nf = !isfinite(ss);
+  uint16_t n16 = 0;
+  float sigma = 0.0f;
+  if (!nf) {
+    const float r = __fsqrt_rn(ss);
+    sigma = (r == 0.0f) ? 0.0f : __fdiv_rn(kSqrtD, r);
+    if (!(r != 0.0f && isfinite(sigma))) sigma = 0.0f;
+    float nv = __fdiv_rn(r, kSqrtD);
+    if (nv > 65504.0f) nv = 65504.0f;
+    n16 = __half_as_ushort(__float2half_rn(nv));
+  }
+  *sigma_out = sigma;
+  *n16_out = n16;
+  *nf_out = nf;
+}
+
+// One butterfly stage of E2 between the lanes j and j ^ o of a quad: the
+// lane whose bit is clear holds a and keeps a + b, its partner holds b and
+// keeps a - b, computed as (-b) + a (IEEE subtraction is addition of the
+// negated operand, so the result is the same); neg is the sign bit for the
+// partner, 0 for the lane whose bit is clear.
+__device__ __forceinline__ float cross_butterfly(float z, int o, uint32_t neg) {
+  const float p = __shfl_xor_sync(kFull, z, o);
+  return __fadd_rn(__uint_as_float(__float_as_uint(z) ^ neg), p);
+}
+
+// Phase 1 for the 32 vectors of a warp (v0 .. v0 + 31), four lanes per
+// vector: in pass p the quad g = lane / 4 takes vector l = 8 p + g, and its
+// lane j holds the coordinates 32 m + 8 j + e in z[m][e]. E1 sign flip, E2
+// with the stages h = 1, 2, 4 in-lane, h = 8 and 16 between lanes j ^ 1 and
+// j ^ 2, h = 32 and 64 in-lane again (the seven stages in order, so the same
+// sums as a transform in one lane); E3 with the 32 partial sums of four
+// squares in-lane (lane j holds p_l for l = 8 j + e), offsets 16 and 8 from
+// lanes j ^ 2 and j ^ 1, then 4, 2, 1 in-lane; E4 by the three-step search.
+// Symbol i of vector l goes to byte i % 4 of W.syms[i / 4][l]; the norm and
+// the non-finite flag to W.n16[l] and W.nf[l].
+template <bool kBF16>
+__device__ __forceinline__ void quad_prepare(const AppendArgs &a, const StreamCtx &c, WarpArea &W, int64_t v0,
+                                             int lane) {
+  const int g = lane >> 2, j = lane & 3;
+#pragma unroll 1
+  for (int p = 0; p < 4; ++p) {
+    const int l = 8 * p + g;
+    const int64_t v = v0 + l;
+    const bool valid = v < c.nvec;  // quad-uniform
+    float z[4][8];
+    if (valid) {
+      const int h = c.head_of(a, v);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const uint32_t sb = __ldg(a.sign_bits + h * 4 + m) >> (8 * j);
+        const int64_t e0 = v * kD + 32 * m + 8 * j;
+        if constexpr (kBF16) {
+          const uint4 w = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(c.src) + e0));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            z[m][2 * t] = __uint_as_float((ww[t] << 16) ^ sign_bit(sb, 2 * t));
+            z[m][2 * t + 1] = __uint_as_float((ww[t] & 0xFFFF0000u) ^ sign_bit(sb, 2 * t + 1));
+          }
+        } else {
+          const uint4 *src4 = reinterpret_cast<const uint4 *>(static_cast<const float *>(c.src) + e0);
+          const uint4 w0 = __ldg(src4), w1 = __ldg(src4 + 1);
+          const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) z[m][e] = __uint_as_float(ww[e] ^ sign_bit(sb, e));
+        }
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) z[m][e] = 0.0f;
+    }
+    // E2, h = 1, 2, 4 (bits of e).
+#pragma unroll
+    for (int st = 0; st < 3; ++st) {
+      const int hh = 1 << st;
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int pr = 0; pr < 4; ++pr) {
+          const int e = ((pr >> st) << (st + 1)) | (pr & (hh - 1));
+          const float a0 = z[m][e], b0 = z[m][e + hh];
+          z[m][e] = __fadd_rn(a0, b0);
+          z[m][e + hh] = __fsub_rn(a0, b0);
+        }
+    }
+    // h = 8, 16 (bits of j).
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[m][e] = cross_butterfly(z[m][e], 1, (j & 1) ? 0x80000000u : 0u);
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) z[m][e] = cross_butterfly(z[m][e], 2, (j & 2) ? 0x80000000u : 0u);
+    // h = 32, 64 (bits of m).
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      const int hm = 1 << st;
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int m = ((pr >> st) << (st + 1)) | (pr & (hm - 1));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a0 = z[m][e], b0 = z[m + hm][e];
+          z[m][e] = __fadd_rn(a0, b0);
+          z[m + hm][e] = __fsub_rn(a0, b0);
+        }
+      }
+    }
+    // E3.
+    float pp[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      pp[e] = __fadd_rn(__fadd_rn(__fmul_rn(z[0][e], z[0][e]), __fmul_rn(z[1][e], z[1][e])),
+                        __fadd_rn(__fmul_rn(z[2][e], z[2][e]), __fmul_rn(z[3][e], z[3][e])));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pp[e] = __fadd_rn(pp[e], __shfl_xor_sync(kFull, pp[e], 2));  // lanes j = 0, 1
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pp[e] = __fadd_rn(pp[e], __shfl_xor_sync(kFull, pp[e], 1));  // lane j = 0
+#pragma unroll
+    for (int o = 4; o >= 1; o >>= 1)
+#pragma unroll
+      for (int e = 0; e < o; ++e) pp[e] = __fadd_rn(pp[e], pp[e + o]);
+    const float ss = __shfl_sync(kFull, pp[0], lane & ~3);
+    float sigma;
+    uint16_t n16;
+    bool nf;
+    norm_scale(ss, &sigma, &n16, &nf);
+    // E4 (u = 0 for the zero and the non-finite vector).
+    if (valid) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float u = nf ? 0.0f : __fmul_rn(z[m][4 * hf + e], sigma);
+            word |= quantize7(u, c.t) << (8 * e);
+          }
+          W.syms[8 * m + 2 * j + hf][l] = word;
+        }
+      if (j == 0) {
+        W.n16[l] = n16;
+        W.nf[l] = nf ? 1 : 0;
+      }
+    }
+  }
 }
 
 // Drift counters of one warp.
@@ -597,19 +672,13 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
   uint8_t *stk = W.stack + lane;
   uint16_t n16 = 0;
   bool nf = false, dropped = false, too_long = false, bad_page = false;
+  quad_prepare<kBF16>(a, c, W, v0, lane);
+  __syncwarp();
   if (valid) {
-    const int h = c.head_of(a, v);
-    uint32_t sw[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
-    {
-      uint32_t pk[32];
-      lane_prepare<kBF16>(c.src, v, sw, c.t, pk, &n16, &nf);
-#pragma unroll
-      for (int w2 = 0; w2 < kD / 4; ++w2) W.syms[w2][lane] = pk[w2];
-    }
-    // The encode loop reads the symbols back from shared memory so that it
-    // can stay rolled (a fully unrolled loop adds ~40 KB of code).
+    n16 = W.n16[lane];
+    nf = W.nf[lane] != 0;
+    // The encode loop reads the symbols from shared memory so that it can
+    // stay rolled (a fully unrolled loop adds ~40 KB of code).
     const uint8_t *sy = reinterpret_cast<const uint8_t *>(&W.syms[0][lane]);
     uint32_t x = 0;
     const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(sy[(i >> 2) * 128 + (i & 3)]); },
@@ -888,7 +957,7 @@ __global__ void __launch_bounds__(kDriftWarps * 32) append_drift_kernel(const Ap
 
 // One CTA = kAW warps of one stream (blockIdx.y: 0 = K, 1 = V).
 template <bool kBF16, bool kTwoK, bool kTwoV>
-__global__ void __launch_bounds__(kAW * 32, 3) append_lane_kernel(const AppendArgs a) {
+__global__ void __launch_bounds__(kAW * 32, 8) append_lane_kernel(const AppendArgs a) {
   __shared__ AppendTables T;
   __shared__ WarpArea W[kAW];
   const bool is_v = blockIdx.y == 1;
