@@ -131,19 +131,20 @@ __device__ __forceinline__ uint32_t sign_bit(uint32_t word, int b) { return (wor
 // go to stk[32 j]. Returns the total length 3 + #pushed; above `cap` the
 // container is too long (pushes past the stack wrap around and are never
 // stored). No lane branches, so all 32 lanes of a warp stay converged. kTwo:
-// the table has a symbol with f < 16, so a step can push two bytes.
+// the table has a symbol with f < 16, so a step can push two bytes. kStk:
+// push-stack slots per lane (a power of two, at least C - 4).
 // One encode step of encode_bf.
-template <bool kTwo>
+template <bool kTwo, int kStk = kStackSlots>
 __device__ __forceinline__ void encode_step(uint32_t s, const uint8_t *esb, uint8_t *stk, uint32_t &x, uint32_t &np) {
   const uint4 e0 = *reinterpret_cast<const uint4 *>(esb + s * sizeof(EncSym));  // {m, k, xmax, cum}
   const uint32_t g = *reinterpret_cast<const uint32_t *>(esb + s * sizeof(EncSym) + 16);
   bool push = x >= e0.z;
-  stk[32 * (np & (kStackSlots - 1))] = static_cast<uint8_t>(x);
+  stk[32 * (np & (kStk - 1))] = static_cast<uint8_t>(x);
   np += push ? 1u : 0u;
   x = push ? (x >> 8) : x;
   if constexpr (kTwo) {
     push = x >= e0.z;
-    stk[32 * (np & (kStackSlots - 1))] = static_cast<uint8_t>(x);
+    stk[32 * (np & (kStk - 1))] = static_cast<uint8_t>(x);
     np += push ? 1u : 0u;
     x = push ? (x >> 8) : x;
   }
@@ -153,17 +154,17 @@ __device__ __forceinline__ void encode_step(uint32_t s, const uint8_t *esb, uint
 
 // kRegs: symbols come from registers (the loop is unrolled completely so
 // that sym(i) indexes them statically); otherwise from shared memory.
-template <bool kTwo, bool kRegs, typename SymFn>
+template <bool kTwo, bool kRegs, typename SymFn, int kStk = kStackSlots>
 __device__ __forceinline__ int encode_bf(SymFn sym, const EncSym *es, uint8_t *stk, uint32_t *x_out) {
   uint32_t x = kL;
   uint32_t np = 0;
   const uint8_t *esb = reinterpret_cast<const uint8_t *>(es);
   if constexpr (kRegs) {
 #pragma unroll
-    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo>(sym(i), esb, stk, x, np);
+    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo, kStk>(sym(i), esb, stk, x, np);
   } else {
 #pragma unroll 4
-    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo>(sym(i), esb, stk, x, np);
+    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo, kStk>(sym(i), esb, stk, x, np);
   }
   *x_out = x;
   return 3 + static_cast<int>(np);
@@ -775,10 +776,15 @@ constexpr int kSlots = 8;
 constexpr int kWin = 4;
 static_assert(kSlots * kWin == 32, "one trial per lane");
 constexpr int kDriftWarps = 4;  // warps per drift CTA
+constexpr int kDriftCtas = 7;   // drift CTAs per SM the register budget is set for
 
+// kStk push-stack slots per lane: 32 when both containers hold at most 36
+// bytes (a string that fits pushes at most C - 5 <= 31 bytes; longer trials
+// wrap around and are never stored), else 64.
+template <int kStk>
 struct DriftArea {
-  uint8_t stack[kStackSlots * 32];
-  uint32_t sw[kD][kSlots];   // symbol i of slot c: q | tgt << 8 | rank << 16 (kNoRank: not ranked)
+  uint8_t stack[kStk * 32];
+  uint16_t sw[kD][kSlots];   // symbol i of slot c: q | tgt << 3 | rank << 6 (kNoRank: not ranked)
   float key[kSlots][4][32];  // key of the move of symbol l + 32 k, +inf once ranked or without a candidate
   int64_t vd[kSlots];
   int32_t ranked[kSlots], win[kSlots];
@@ -787,9 +793,9 @@ struct DriftArea {
 };
 
 // E6 for one stream's drift list: entries first, first + stride, ... .
-template <bool kTwo>
-__device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, bool is_v, int lane, uint32_t first,
-                                             uint32_t stride, DriftCount &dc) {
+template <bool kTwo, int kStk>
+__device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk> &A, bool is_v, int lane,
+                                             uint32_t first, uint32_t stride, DriftCount &dc) {
   __syncwarp();
   const StreamCtx c = stream_setup(a, A.T, is_v, lane);
   if (lane < kSlots) {
@@ -820,7 +826,8 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, 
       for (int k = 0; k < 4; ++k) {
         int tj;
         A.key[s][k][lane] = best_move(A.T, c.nl, static_cast<int>(qk[k]), u[k], &tj);
-        A.sw[lane + 32 * k][s] = qk[k] | (static_cast<uint32_t>(tj) << 8) | (static_cast<uint32_t>(kNoRank) << 16);
+        A.sw[lane + 32 * k][s] =
+            static_cast<uint16_t>(qk[k] | (static_cast<uint32_t>(tj) << 3) | (static_cast<uint32_t>(kNoRank) << 6));
       }
       if (lane == 0) {
         A.vd[s] = v;
@@ -864,7 +871,7 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, 
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             if (bi == lane + 32 * k) key[k] = INFINITY;
-          A.sw[bi][s] = (A.sw[bi][s] & 0xFFFFu) | (static_cast<uint32_t>(r) << 16);
+          A.sw[bi][s] = static_cast<uint16_t>((A.sw[bi][s] & 0x3Fu) | (static_cast<uint32_t>(r) << 6));
         }
       }
 #pragma unroll
@@ -879,7 +886,7 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, 
     // A lane whose slot is empty encodes a live slot's string (its words
     // were all written at refill, every symbol below nl); its result is
     // not used.
-    const uint32_t *swc = &A.sw[0][mine ? cs : __ffs(live) - 1];
+    const uint16_t *swc = &A.sw[0][mine ? cs : __ffs(live) - 1];
     const int win = A.win[cs], ranked = A.ranked[cs];
     const int km = win + jw;
     const bool trial = mine && km < ranked;
@@ -888,22 +895,20 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, 
     int len;
     if (__any_sync(kFull, fb)) {
       const uint32_t kmx = fb ? 254u : static_cast<uint32_t>(km);
-      len = encode_bf<kTwo, false>(
-          [&](int i) {
-            const uint32_t w = swc[i * kSlots];
-            uint32_t sy = ((w >> 16) <= kmx) ? ((w >> 8) & 0xFFu) : (w & 0xFFu);
-            if (fb) sy = sy >= hlf ? hlf : hlf - 1u;
-            return sy;
-          },
-          A.T.es, stk, &x);
+      auto sym = [&](int i) {
+        const uint32_t w = swc[i * kSlots];
+        uint32_t sy = ((w >> 6) <= kmx) ? ((w >> 3) & 7u) : (w & 7u);
+        if (fb) sy = sy >= hlf ? hlf : hlf - 1u;
+        return sy;
+      };
+      len = encode_bf<kTwo, false, decltype(sym), kStk>(sym, A.T.es, stk, &x);
     } else {
       const uint32_t kmx = static_cast<uint32_t>(km);
-      len = encode_bf<kTwo, false>(
-          [&](int i) {
-            const uint32_t w = swc[i * kSlots];
-            return ((w >> 16) <= kmx) ? ((w >> 8) & 0xFFu) : (w & 0xFFu);
-          },
-          A.T.es, stk, &x);
+      auto sym = [&](int i) {
+        const uint32_t w = swc[i * kSlots];
+        return ((w >> 6) <= kmx) ? ((w >> 3) & 7u) : (w & 7u);
+      };
+      len = encode_bf<kTwo, false, decltype(sym), kStk>(sym, A.T.es, stk, &x);
     }
     const bool ok = len <= c.P;
     const unsigned fit = __ballot_sync(kFull, trial && ok);
@@ -939,16 +944,16 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea &A, 
 
 // Every warp walks its share of the K list, then of the V list, so the two
 // streams' lists (often of very different lengths) spread over all warps.
-template <bool kTwoK, bool kTwoV>
-__global__ void __launch_bounds__(kDriftWarps * 32) append_drift_kernel(const AppendArgs a) {
-  __shared__ DriftArea A[kDriftWarps];
+template <bool kTwoK, bool kTwoV, int kStk>
+__global__ void __launch_bounds__(kDriftWarps * 32, kDriftCtas) append_drift_kernel(const AppendArgs a) {
+  __shared__ DriftArea<kStk> A[kDriftWarps];
   const int lane = threadIdx.x & 31;
-  DriftArea &w = A[threadIdx.x >> 5];
+  DriftArea<kStk> &w = A[threadIdx.x >> 5];
   const uint32_t first = blockIdx.x * kDriftWarps + (threadIdx.x >> 5);
   const uint32_t stride = gridDim.x * kDriftWarps;
   DriftCount dk, dv;
-  drift_stream<kTwoK>(a, w, false, lane, first, stride, dk);
-  drift_stream<kTwoV>(a, w, true, lane, first, stride, dv);
+  drift_stream<kTwoK, kStk>(a, w, false, lane, first, stride, dk);
+  drift_stream<kTwoV, kStk>(a, w, true, lane, first, stride, dv);
   if (lane == 0) {
     add_stats(a, false, dk, 0u, 0u);
     add_stats(a, true, dv, 0u, 0u);
@@ -984,6 +989,21 @@ __global__ void __launch_bounds__(kAW * 32) append_warp_kernel(const AppendArgs 
   }
 }
 
+template <bool kTwoK, bool kTwoV, int kStk>
+int launch_drift(const AppendArgs &a, int sms, cudaStream_t st) {
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV, kStk>, kDriftWarps * 32,
+                                                      0) != cudaSuccess ||
+        n < 1)
+      n = 1;
+    per_sm = n;
+  }
+  append_drift_kernel<kTwoK, kTwoV, kStk><<<static_cast<unsigned>(per_sm * sms), kDriftWarps * 32, 0, st>>>(a);
+  return static_cast<int>(cudaGetLastError());
+}
+
 template <bool kBF16, bool kTwoK, bool kTwoV>
 int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, int sms, cudaStream_t st) {
   const int64_t per_cta = lanes ? static_cast<int64_t>(kAW) * 32 : kAW;
@@ -1002,16 +1022,8 @@ int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, int sms, cudaStrea
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.drift_list) return static_cast<int>(e);
   // Drift: a persistent grid, as many CTAs as fit on the SMs at once.
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV>, kDriftWarps * 32, 0) !=
-            cudaSuccess || n < 1)
-      n = 1;
-    per_sm = n;
-  }
-  append_drift_kernel<kTwoK, kTwoV><<<static_cast<unsigned>(per_sm * sms), kDriftWarps * 32, 0, st>>>(a);
-  return static_cast<int>(cudaGetLastError());
+  if (a.ck <= 36 && a.cv <= 36) return launch_drift<kTwoK, kTwoV, 32>(a, sms, st);
+  return launch_drift<kTwoK, kTwoV, 64>(a, sms, st);
 }
 
 template <bool kBF16>
