@@ -111,6 +111,32 @@ __device__ __forceinline__ float best_move(const AppendTables &T, int nl, int s,
   return best;
 }
 
+// A float key as an unsigned integer with the same order (sign bit set:
+// all bits flipped; clear: the sign bit set). -0 is first made +0 (k + 0 in
+// round-to-nearest; the float order holds them equal), keys are never NaN,
+// so equal integers are equal keys; +inf (no candidate) maps to 0xFF800000,
+// above every finite key.
+__device__ __forceinline__ uint32_t order_bits(float k) {
+  const uint32_t b = __float_as_uint(__fadd_rn(k, 0.0f));
+  return b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
+}
+constexpr uint32_t kNoKey = 0xFF800000u;      // order_bits(+inf)
+constexpr uint32_t kRankedKey = 0xFFFFFFFFu;  // above kNoKey
+
+// Warp arg-min over the 128 keys of a vector (symbol lane + 32 k in key[k],
+// as order_bits): the least key, ties to the lowest symbol index. Returns
+// that index, or -1 when no key is below kNoKey (no candidate left).
+__device__ __forceinline__ int warp_argmin(const uint32_t (&key)[4], int lane) {
+  const uint32_t bk = __reduce_min_sync(kFull, min(min(key[0], key[1]), min(key[2], key[3])));
+  if (bk >= kNoKey) return -1;
+  const uint32_t mine = key[0] == bk   ? static_cast<uint32_t>(lane)
+                        : key[1] == bk ? static_cast<uint32_t>(lane + 32)
+                        : key[2] == bk ? static_cast<uint32_t>(lane + 64)
+                        : key[3] == bk ? static_cast<uint32_t>(lane + 96)
+                                       : 0xFFFFFFFFu;
+  return static_cast<int>(__reduce_min_sync(kFull, mine));
+}
+
 // E4: symbol = number of thresholds <= u (ties go up), by a three-step
 // search over the 7 sorted thresholds t0..t6 (padded with +inf).
 __device__ __forceinline__ uint32_t quantize7(float u, const float (&t)[7]) {
@@ -463,12 +489,12 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
                                           DriftCount &dc) {
   uint8_t *stk = stack + lane;
   // Best move and key of the 4 symbols this lane owns (i = lane + 32 k).
-  float key[4];
+  uint32_t key[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int i = lane + 32 * k;
     int tj;
-    key[k] = best_move(T, c.nl, q[i], u[k], &tj);
+    key[k] = order_bits(best_move(T, c.nl, q[i], u[k], &tj));
     rank[i] = kNoRank;
     tgt[i] = static_cast<uint8_t>(tj);
   }
@@ -482,22 +508,12 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
     const int batch = ranked == 0 ? first_batch : 32;
     int added = 0;
     for (; added < batch; ++added) {
-      float bk = key[0];
-      int bi = lane;
-#pragma unroll
-      for (int k = 1; k < 4; ++k)
-        if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const float ok = __shfl_xor_sync(kFull, bk, off);
-        const int oi = __shfl_xor_sync(kFull, bi, off);
-        if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-      }
-      if (bk == INFINITY) break;  // no candidate left
+      const int bi = warp_argmin(key, lane);
+      if (bi < 0) break;  // no candidate left
       if ((bi & 31) == lane) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-          if (bi == lane + 32 * k) key[k] = INFINITY;
+          if (bi == lane + 32 * k) key[k] = kRankedKey;
         rank[bi] = static_cast<uint8_t>(ranked + added);
       }
     }
@@ -570,7 +586,7 @@ template <bool kTwo>
 __device__ __forceinline__ int rd_fill(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
                                        uint8_t *stack, const uint8_t *q0, uint8_t *qd, int64_t v, uint16_t n16,
                                        const float (&u)[4], int lane) {
-  float key[4];
+  uint32_t key[4];
   uint8_t jn[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -587,36 +603,26 @@ __device__ __forceinline__ int rd_fill(const AppendArgs &a, const StreamCtx &c, 
     }
     const int s = qd[i];
     jn[k] = static_cast<uint8_t>(j);
-    key[k] = INFINITY;
+    key[k] = kNoKey;
     if (j != s && abs(j - s) == 1 && abs(j - static_cast<int>(q0[i])) <= 1) {
       const float dj = __fsub_rn(u[k], T.lev[j]);
       const float ds = __fsub_rn(u[k], T.lev[s]);
       const float dd = __fsub_rn(__fmul_rn(dj, dj), __fmul_rn(ds, ds));
       const float dr = __fsub_rn(T.cost[j], T.cost[s]);
-      if (dd < 0.0f && dr > 0.0f) key[k] = __fdiv_rn(dd, dr);
+      if (dd < 0.0f && dr > 0.0f) key[k] = order_bits(__fdiv_rn(dd, dr));
     }
   }
   uint8_t *stk = stack;  // lane 0's push stack
   int ups = 0;
   while (true) {
-    float bk = key[0];
-    int bi = lane;
-#pragma unroll
-    for (int k = 1; k < 4; ++k)
-      if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ok = __shfl_xor_sync(kFull, bk, off);
-      const int oi = __shfl_xor_sync(kFull, bi, off);
-      if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-    }
-    if (bk == INFINITY) break;
+    const int bi = warp_argmin(key, lane);
+    if (bi < 0) break;
     uint8_t old = 0;
     if ((bi & 31) == lane) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         if (bi == lane + 32 * k) {
-          key[k] = INFINITY;
+          key[k] = kRankedKey;
           old = qd[bi];
           qd[bi] = jn[k];
         }
@@ -784,8 +790,8 @@ constexpr int kDriftCtas = 7;   // drift CTAs per SM the register budget is set 
 template <int kStk>
 struct DriftArea {
   uint8_t stack[kStk * 32];
-  uint16_t sw[kD][kSlots];   // symbol i of slot c: q | tgt << 3 | rank << 6 (kNoRank: not ranked)
-  float key[kSlots][4][32];  // key of the move of symbol l + 32 k, +inf once ranked or without a candidate
+  uint16_t sw[kD][kSlots];      // symbol i of slot c: q | tgt << 3 | rank << 6 (kNoRank: not ranked)
+  uint32_t key[kSlots][4][32];  // order_bits of the move key of symbol l + 32 k; kRankedKey once ranked
   int64_t vd[kSlots];
   int32_t ranked[kSlots], win[kSlots];
   uint16_t n16[kSlots];
@@ -825,7 +831,7 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         int tj;
-        A.key[s][k][lane] = best_move(A.T, c.nl, static_cast<int>(qk[k]), u[k], &tj);
+        A.key[s][k][lane] = order_bits(best_move(A.T, c.nl, static_cast<int>(qk[k]), u[k], &tj));
         A.sw[lane + 32 * k][s] =
             static_cast<uint16_t>(qk[k] | (static_cast<uint32_t>(tj) << 3) | (static_cast<uint32_t>(kNoRank) << 6));
       }
@@ -841,36 +847,27 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
     if (!live) break;
     __syncwarp();
     // Every live slot with candidates left ranks its moves up to win + kWin
-    // by repeated arg-min over (key, index).
+    // by repeated arg-min over (key, index): the least key over the warp,
+    // then the lowest index holding it.
 #pragma unroll 1
     for (int s = 0; s < kSlots; ++s) {
       if (!(((live & ~exh) >> s) & 1u)) continue;
       int r = A.ranked[s];
       const int target = A.win[s] + kWin;
       if (r >= target) continue;
-      float key[4];
+      uint32_t key[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) key[k] = A.key[s][k][lane];
       for (; r < target; ++r) {
-        float bk = key[0];
-        int bi = lane;
-#pragma unroll
-        for (int k = 1; k < 4; ++k)
-          if (key[k] < bk) { bk = key[k]; bi = lane + 32 * k; }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          const float ok = __shfl_xor_sync(kFull, bk, off);
-          const int oi = __shfl_xor_sync(kFull, bi, off);
-          if (ok < bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-        }
-        if (bk == INFINITY) {
+        const int bi = warp_argmin(key, lane);
+        if (bi < 0) {
           exh |= 1u << s;
           break;
         }
         if ((bi & 31) == lane) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            if (bi == lane + 32 * k) key[k] = INFINITY;
+            if (bi == lane + 32 * k) key[k] = kRankedKey;
           A.sw[bi][s] = static_cast<uint16_t>((A.sw[bi][s] & 0x3Fu) | (static_cast<uint32_t>(r) << 6));
         }
       }
