@@ -68,7 +68,8 @@ struct WarpArea {
   uint8_t stack[kStackSlots * 32];
   uint32_t syms[kD / 4][32];
   uint8_t q[kD], rank[kD], tgt[kD];
-  uint16_t n16[32];  // fp16 norm of the warp's vector l (lane-per-vector kernel)
+  int32_t head[32];  // KV head of the warp's vector l (lane-per-vector kernel)
+  uint16_t n16[32];  // fp16 norm of the warp's vector l
   uint8_t nf[32];    // vector l was non-finite
 };
 
@@ -242,6 +243,20 @@ __device__ __forceinline__ void warp_prepare(const AppendArgs &a, const void *sr
   for (int k = 0; k < 4; ++k) q[lane + 32 * k] = static_cast<uint8_t>(qk[k]);
 }
 
+// v / d, with v % d in *rem, for 0 <= v and 0 < d; in 32-bit arithmetic
+// when both fit (the same quotient, far fewer instructions than a 64-bit
+// division).
+__device__ __forceinline__ int64_t div_rem(int64_t v, int64_t d, int64_t *rem) {
+  if (((v | d) >> 32) == 0) {
+    const uint32_t q = static_cast<uint32_t>(v) / static_cast<uint32_t>(d);
+    *rem = v - static_cast<int64_t>(q) * d;
+    return q;
+  }
+  const int64_t q = v / d;
+  *rem = v - q * d;
+  return q;
+}
+
 // Where the vectors of one append call come from and go to (one stream).
 struct StreamCtx {
   const void *src;
@@ -250,16 +265,26 @@ struct StreamCtx {
   int64_t per_seq, nvec;
   float t[7];
 
-  __device__ int head_of(const AppendArgs &a, int64_t v) const {
-    return static_cast<int>((v % per_seq) / a.n_new);
+  // Sequence b, KV head h and new-token index j of vector v
+  // (v = (b Hkv + h) n_new + j).
+  __device__ void split(const AppendArgs &a, int64_t v, int *b, int *h, int64_t *j) const {
+    int64_t rem, jj;
+    *b = static_cast<int>(div_rem(v, per_seq, &rem));
+    *h = static_cast<int>(div_rem(rem, a.n_new, &jj));
+    *j = jj;
   }
-  // Byte 0 of vector v's container (lane pos % 32 of the 32-token block
-  // holding position pos), or null when the position is outside the cache
-  // (dropped) or its page-table entry is out of range (also *bad_page).
-  __device__ uint8_t *dst_of(const AppendArgs &a, int64_t v, bool *dropped, bool *bad_page = nullptr) const {
-    const int b = static_cast<int>(v / per_seq);
-    const int h = head_of(a, v);
-    const int j = static_cast<int>(v % a.n_new);
+  __device__ int head_of(const AppendArgs &a, int64_t v) const {
+    int b, h;
+    int64_t j;
+    split(a, v, &b, &h, &j);
+    return h;
+  }
+  // Byte 0 of the container of token j of sequence b, KV head h (lane
+  // pos % 32 of the 32-token block holding position pos), or null when the
+  // position is outside the cache (dropped) or its page-table entry is out of
+  // range (also *bad_page).
+  __device__ uint8_t *dst_at(const AppendArgs &a, int b, int h, int64_t j, bool *dropped,
+                             bool *bad_page = nullptr) const {
     const int64_t pos = static_cast<int64_t>(a.start_pos[b]) + j;
     *dropped = pos < 0 || pos >= a.T_cap;
     if (*dropped) return nullptr;
@@ -276,6 +301,12 @@ struct StreamCtx {
       block = (static_cast<int64_t>(b) * a.Hkv + h) * (a.T_cap >> 5) + (pos >> 5);
     }
     return cache + block * 32 * C + (pos & 31);
+  }
+  __device__ uint8_t *dst_of(const AppendArgs &a, int64_t v, bool *dropped, bool *bad_page = nullptr) const {
+    int b, h;
+    int64_t j;
+    split(a, v, &b, &h, &j);
+    return dst_at(a, b, h, j, dropped, bad_page);
   }
 };
 
@@ -355,7 +386,8 @@ __device__ __forceinline__ float cross_butterfly(float z, int o, uint32_t neg) {
 // squares in-lane (lane j holds p_l for l = 8 j + e), offsets 16 and 8 from
 // lanes j ^ 2 and j ^ 1, then 4, 2, 1 in-lane; E4 by the three-step search.
 // Symbol i of vector l goes to byte i % 4 of W.syms[i / 4][l]; the norm and
-// the non-finite flag to W.n16[l] and W.nf[l].
+// the non-finite flag to W.n16[l] and W.nf[l]. W.head[l] holds the vector's
+// KV head on entry.
 template <bool kBF16>
 __device__ __forceinline__ void quad_prepare(const AppendArgs &a, const StreamCtx &c, WarpArea &W, int64_t v0,
                                              int lane) {
@@ -367,7 +399,7 @@ __device__ __forceinline__ void quad_prepare(const AppendArgs &a, const StreamCt
     const bool valid = v < c.nvec;  // quad-uniform
     float z[4][8];
     if (valid) {
-      const int h = c.head_of(a, v);
+      const int h = W.head[l];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const uint32_t sb = __ldg(a.sign_bits + h * 4 + m) >> (8 * j);
@@ -679,6 +711,11 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
   uint8_t *stk = W.stack + lane;
   uint16_t n16 = 0;
   bool nf = false, dropped = false, too_long = false, bad_page = false;
+  int vb = 0, vh = 0;
+  int64_t vj = 0;
+  if (valid) c.split(a, v, &vb, &vh, &vj);
+  W.head[lane] = vh;
+  __syncwarp();
   quad_prepare<kBF16>(a, c, W, v0, lane);
   __syncwarp();
   if (valid) {
@@ -691,7 +728,7 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
     const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(sy[(i >> 2) * 128 + (i & 3)]); },
                                            T.es, stk, &x);
     too_long = len > c.P;
-    uint8_t *dst = c.dst_of(a, v, &dropped, &bad_page);
+    uint8_t *dst = c.dst_at(a, vb, vh, vj, &dropped, &bad_page);
     if (!too_long && dst) store_container(dst, c.C, n16, x, stk, len);
   }
   unsigned drift_mask = __ballot_sync(kFull, too_long);
