@@ -612,12 +612,23 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
 // level j (least (u - y_j)^2 in fp32, ties to the lower level) is one level
 // from qd and at most one from q0, with dD = (u - y_j)^2 - (u - y_qd)^2 < 0 and
 // dR = cost_j - cost_qd > 0; candidates go in order of dD / dR (fp32, ties to
-// the lower index), each kept if lane 0's re-encode still fits. Stores the
-// container; returns the number of symbols moved.
+// the lower index), each kept if the string with it and every earlier kept
+// candidate still fits. Stores the container; returns the number of symbols
+// moved.
+//
+// The keys do not change while candidates are kept, so a pass tests 32 at
+// once: from the next untested rank p, lane m encodes the current string with
+// candidate p + m alone applied. Candidates p .. p + m* - 1 before the first
+// one that fits (m*) do not fit on the string they are tested on in the
+// one-at-a-time order either (nothing was kept between), so they are
+// dropped; p + m* is kept, lane m* stores its string (the container as
+// stored before the fill stands when nothing is kept) and the next pass
+// starts after it. cand[] (128 entries) holds the ranked candidates (symbol
+// index | target << 8).
 template <bool kTwo>
 __device__ __forceinline__ int rd_fill(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
-                                       uint8_t *stack, const uint8_t *q0, uint8_t *qd, int64_t v, uint16_t n16,
-                                       const float (&u)[4], int lane) {
+                                       uint8_t *stack, const uint8_t *q0, uint8_t *qd, uint16_t *cand, int64_t v,
+                                       uint16_t n16, const float (&u)[4], int lane) {
   uint32_t key[4];
   uint8_t jn[4];
 #pragma unroll
@@ -644,43 +655,53 @@ __device__ __forceinline__ int rd_fill(const AppendArgs &a, const StreamCtx &c, 
       if (dd < 0.0f && dr > 0.0f) key[k] = order_bits(__fdiv_rn(dd, dr));
     }
   }
-  uint8_t *stk = stack;  // lane 0's push stack
-  int ups = 0;
-  while (true) {
-    const int bi = warp_argmin(key, lane);
-    if (bi < 0) break;
-    uint8_t old = 0;
-    if ((bi & 31) == lane) {
+  uint8_t *stk = stack + lane;
+  bool dropped = false;
+  uint8_t *dst = c.dst_of(a, v, &dropped);
+  int ups = 0, ranked = 0, p = 0;
+  bool exhausted = false;
+  for (;;) {
+    // Ranks p .. p + 31 (as far as there are candidates).
+    while (!exhausted && ranked < p + 32) {
+      const int bi = warp_argmin(key, lane);
+      if (bi < 0) {
+        exhausted = true;
+        break;
+      }
+      if ((bi & 31) == lane) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (bi == lane + 32 * k) {
-          key[k] = kRankedKey;
-          old = qd[bi];
-          qd[bi] = jn[k];
-        }
+        for (int k = 0; k < 4; ++k)
+          if (bi == lane + 32 * k) {
+            key[k] = kRankedKey;
+            cand[ranked] = static_cast<uint16_t>(bi | (jn[k] << 8));
+          }
+      }
+      ++ranked;
     }
+    if (p >= ranked) break;
     __syncwarp();
-    int len = 0;
-    if (lane == 0) {
-      uint32_t x = 0;
-      len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(qd[i]); }, T.es, stk, &x);
-    }
-    len = __shfl_sync(kFull, len, 0);
-    if (len > c.P) {
-      if ((bi & 31) == lane) qd[bi] = old;
-    } else {
-      ++ups;
-    }
-    __syncwarp();
-  }
-  if (lane == 0) {
+    const bool has = p + lane < ranked;
+    const uint32_t cw = has ? cand[p + lane] : 0xFFFFu;
+    const int ci = static_cast<int>(cw & 0xFFu);  // 255: no candidate (matches no symbol)
+    const uint32_t ct = cw >> 8;
     uint32_t x = 0;
-    const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(qd[i]); }, T.es, stk, &x);
-    bool dr = false;
-    uint8_t *dst = c.dst_of(a, v, &dr);
-    if (dst && len <= c.P) store_container(dst, c.C, n16, x, stk, len);
+    const int len = encode_bf<kTwo, false>(
+        [&](int i) { return i == ci ? ct : static_cast<uint32_t>(qd[i]); }, T.es, stk, &x);
+    const unsigned fit = __ballot_sync(kFull, has && len <= c.P);
+    __syncwarp();
+    if (fit) {
+      const int m = __ffs(fit) - 1;
+      if (lane == m) {
+        qd[ci] = static_cast<uint8_t>(ct);
+        if (dst) store_container(dst, c.C, n16, x, stk, len);
+      }
+      ++ups;
+      p += m + 1;
+    } else {
+      p += 32;
+    }
+    __syncwarp();
   }
-  __syncwarp();
   return ups;
 }
 
@@ -800,7 +821,8 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
       W.tgt[i] = (r != kNoRank && static_cast<int>(r) < applied) ? W.tgt[i] : W.q[i];
     }
     __syncwarp();
-    const int ups = rd_fill<kTwo>(a, c, T, W.stack, W.q, W.tgt, v, n16, u, lane);
+    const int ups = rd_fill<kTwo>(a, c, T, W.stack, W.q, W.tgt, reinterpret_cast<uint16_t *>(&W.syms[0][0]), v, n16,
+                                  u, lane);
     if (lane == 0 && ups && a.stats)
       atomicAdd(is_v ? &a.stats->v_syms_filled : &a.stats->k_syms_filled, static_cast<unsigned long long>(ups));
   }
