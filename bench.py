@@ -468,7 +468,8 @@ def run_dq(args):
         }
         if ws == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(w, tab_seed=0, seconds=args.cpu_seconds,
-                                                  rate_offsets=(args.k_rate_offset, args.v_rate_offset))
+                                                  rate_offsets=(args.k_rate_offset, args.v_rate_offset),
+                                                  drift_mode=args.drift_mode)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -505,8 +506,8 @@ def oracle_sample_step(w, tabs, rows, cache_rows):
         from decode_attention_dq_b200 import synth
         k_new = synth.kv_row(w, "k", b, h, n=1, step=0)
         v_new = synth.kv_row(w, "v", b, h, n=1, step=0)
-        kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, np.array([h], np.int32))
-        vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, np.array([h], np.int32))
+        kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, np.array([h], np.int32), tabs.drift_mode)
+        vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, np.array([h], np.int32), tabs.drift_mode)
         kc[-1] = kk[0]
         vc[-1] = vv[0]
         q = synth.q_rows(w, b)[h * G:(h + 1) * G]
@@ -519,7 +520,7 @@ def oracle_sample_step(w, tabs, rows, cache_rows):
         o.attention_fp64(tabs, qb, kfull, vfull, [kc.shape[0]], rows=[(0, h)])
 
 
-def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0.0)):
+def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0.0), drift_mode=0):
     """The oracle, as it stands, on the host: a bounded sample of the step,
     once on one thread (BLAS limited to one thread too) and once on all host
     cores (a thread per (sequence, KV head) row; the oracle's C calls and
@@ -534,7 +535,7 @@ def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0
 
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
                     v_container_bytes=o.container_bytes(w.v_bits), sign_seed=tab_seed,
-                    k_rate_offset=rate_offsets[0], v_rate_offset=rate_offsets[1])
+                    k_rate_offset=rate_offsets[0], v_rate_offset=rate_offsets[1], drift_mode=drift_mode)
     ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
     with threadpool_limits(limits=1):
         # Containers for sampled rows, encoded by the oracle (setup, untimed).
@@ -545,8 +546,8 @@ def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0
             b, h = bh
             K = synth.kv_row(w, "k", b, h)
             V = synth.kv_row(w, "v", b, h)
-            kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
-            vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+            kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32), tabs.drift_mode)
+            vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32), tabs.drift_mode)
             return (bh, (kc, vc))
 
         prepared = []
@@ -635,7 +636,9 @@ def run_prefill(args):
         import torch.distributed as dist
     w = replica_workload(synth.WORKLOADS[args.workload], rank)
     dev = torch.device("cuda", torch.cuda.current_device())
-    tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
+    tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits,
+                             drift_mode=args.drift_mode, k_rate_offset=args.k_rate_offset,
+                             v_rate_offset=args.v_rate_offset)
     ck, cv = tab.k.container_bytes, tab.v.container_bytes
     T, n_q = w.T, args.prefill
     q_start = T - n_q
@@ -732,7 +735,8 @@ def run_prefill(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f16x2 tensor / f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
                        "context": T, "chunk": n_q, "q_start": q_start, "input_dtype": w.dtype,
-                       "k_container_bytes": ck, "v_container_bytes": cv,
+                       "k_container_bytes": ck, "v_container_bytes": cv, "drift_mode": args.drift_mode,
+                       "rate_offsets": [args.k_rate_offset, args.v_rate_offset],
                        "l2": "inputs larger than L2 (%.0f MB of containers, %.0f MB of queries and outputs)"
                              % (comp_bytes / 1e6, io_bytes / 1e6),
                        "parallelism": "replicas x%d" % ws},
@@ -753,7 +757,9 @@ def run_prefill(args):
             "integrity_errors": st["integrity_errors"], "wait_timeouts": st["wait_timeouts"],
         }
         if ws == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = prefill_cpu_baseline(w, n_q, seconds=args.cpu_seconds)
+            result["cpu_baseline"] = prefill_cpu_baseline(w, n_q, seconds=args.cpu_seconds,
+                                                          rate_offsets=(args.k_rate_offset, args.v_rate_offset),
+                                                          drift_mode=args.drift_mode)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -785,8 +791,8 @@ def oracle_prefill_row(w, tabs, bh, n_q, ctx, inputs):
     k_new, v_new, q = inputs
     T = kc.shape[0]
     hh = np.full(n_q, h, np.int32)
-    kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, hh)
-    vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, hh)
+    kk, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, k_new, hh, tabs.drift_mode)
+    vv, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, v_new, hh, tabs.drift_mode)
     kfull = np.zeros((1, w.Hkv, T, kc.shape[1]), np.uint8)
     vfull = np.zeros((1, w.Hkv, T, vc.shape[1]), np.uint8)
     kfull[0, h, :T - n_q] = kc[:T - n_q]
@@ -809,22 +815,23 @@ def prefill_contexts(w, tabs, n_rows, seconds, n_q=0):
     for b, h in rows:
         K = synth.kv_row(w, "k", b, h)
         V = synth.kv_row(w, "v", b, h)
-        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
-        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32), tabs.drift_mode)
+        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32), tabs.drift_mode)
         out.append(((b, h), (kc, vc), prefill_row_inputs(w, (b, h), n_q) if n_q else None))
         if time.time() - t0 > seconds:
             break
     return out
 
 
-def prefill_cpu_baseline(w, n_q, seconds=12.0):
+def prefill_cpu_baseline(w, n_q, seconds=12.0, rate_offsets=(0.0, 0.0), drift_mode=0):
     """The oracle's prefill step on one host thread (BLAS limited to one
     thread), on a bounded sample of (sequence, KV head) rows."""
     from threadpoolctl import threadpool_limits
 
     from oracle import oracle as o
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
-                    v_container_bytes=o.container_bytes(w.v_bits))
+                    v_container_bytes=o.container_bytes(w.v_bits), k_rate_offset=rate_offsets[0],
+                    v_rate_offset=rate_offsets[1], drift_mode=drift_mode)
     from concurrent.futures import ThreadPoolExecutor
     ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
     with threadpool_limits(limits=1):
@@ -858,7 +865,8 @@ def run_reference_prefill(args, w):
     from oracle import oracle as o
     n_q = args.prefill
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
-                    v_container_bytes=o.container_bytes(w.v_bits))
+                    v_container_bytes=o.container_bytes(w.v_bits), k_rate_offset=args.k_rate_offset,
+                    v_rate_offset=args.v_rate_offset, drift_mode=args.drift_mode)
     with threadpool_limits(limits=1):
         ctx = prefill_contexts(w, tabs, args.warmup + args.steps, 1e9, n_q)
         for i in range(args.warmup):
@@ -875,7 +883,8 @@ def run_reference_prefill(args, w):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
-                       "context": w.T, "chunk": n_q, "sample_per_step": "one (sequence, KV head) row"},
+                       "context": w.T, "chunk": n_q, "sample_per_step": "one (sequence, KV head) row",
+                       "drift_mode": args.drift_mode, "rate_offsets": [args.k_rate_offset, args.v_rate_offset]},
             "cpu_baseline": {"value": value, "unit": PREFILL_UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": PREFILL_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
@@ -892,14 +901,15 @@ def run_reference(args):
     import numpy as np
     from oracle import oracle as o
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
-                    v_container_bytes=o.container_bytes(w.v_bits))
+                    v_container_bytes=o.container_bytes(w.v_bits), k_rate_offset=args.k_rate_offset,
+                    v_rate_offset=args.v_rate_offset, drift_mode=args.drift_mode)
     rows = [(s % w.B, (s * 3) % w.Hkv) for s in range(args.warmup + args.steps)]
     prepared = []
     for b, h in rows:
         K = synth.kv_row(w, "k", b, h)
         V = synth.kv_row(w, "v", b, h)
-        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32))
-        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32))
+        kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32), tabs.drift_mode)
+        vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32), tabs.drift_mode)
         prepared.append(((b, h), (kc, vc)))
     from threadpoolctl import threadpool_limits
     with threadpool_limits(limits=1):  # one thread, BLAS included
@@ -916,7 +926,8 @@ def run_reference(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hkv": w.Hkv, "Hq": w.Hq, "head_dim": 128,
-                       "context": w.T, "sample_per_step": "one (sequence, KV head) row"},
+                       "context": w.T, "sample_per_step": "one (sequence, KV head) row",
+                       "drift_mode": args.drift_mode, "rate_offsets": [args.k_rate_offset, args.v_rate_offset]},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": "per step: one (sequence, KV head) row of %s, append 1 token "
                                        "+ fp64 attention over %d tokens, single thread" % (w.name, w.T)},
