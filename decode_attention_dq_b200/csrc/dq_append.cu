@@ -34,7 +34,8 @@
 //     The warp-per-vector kernel tries 32 move counts per pass. The separate
 //     drift kernel (lane-per-vector appends) keeps 8 containers per warp in
 //     flight and tries 4 move counts of each per encode pass, ranking 4 more
-//     moves of a container only when its window had no fit.
+//     moves of a container only when its window had no fit; in drift mode 1
+//     it also runs the rate-distortion fill of every container.
 #include "dq_device.cuh"
 
 namespace dqi {
@@ -507,7 +508,7 @@ __device__ __forceinline__ void quad_prepare(const AppendArgs &a, const StreamCt
 
 // Drift counters of one warp.
 struct DriftCount {
-  unsigned moves = 0, containers = 0, fallbacks = 0;
+  unsigned moves = 0, containers = 0, fallbacks = 0, filled = 0;
 };
 
 // E6 for one over-long container, by the whole warp. On entry q[] holds the
@@ -713,6 +714,8 @@ __device__ __forceinline__ void add_stats(const AppendArgs &a, bool is_v, const 
   if (dc.containers)
     atomicAdd(is_v ? &a.stats->v_cont_drifted : &a.stats->k_cont_drifted, (unsigned long long)dc.containers);
   if (dc.fallbacks) atomicAdd(&a.stats->overflow_fallbacks, (unsigned long long)dc.fallbacks);
+  if (dc.filled)
+    atomicAdd(is_v ? &a.stats->v_syms_filled : &a.stats->k_syms_filled, (unsigned long long)dc.filled);
   if (nf) atomicAdd(&a.stats->nonfinite_inputs, (unsigned long long)nf);
   if (drops) atomicAdd(&a.stats->dropped_writes, (unsigned long long)drops);
 }
@@ -759,12 +762,17 @@ __device__ __forceinline__ void lane_body(const AppendArgs &a, AppendTables &T, 
   DriftCount dc;
 
   if (a.drift_list) {
-    // List the over-long containers for the drift kernel (one atomic per warp).
+    // List the over-long containers for the drift kernel (one atomic per
+    // warp); in drift mode 1 every vector, over-long ones with bit 31 set,
+    // for the drift kernel's fill.
+    const bool listed = a.drift_mode == 1 ? valid : too_long;
+    const unsigned list_mask = __ballot_sync(kFull, listed);
     uint32_t base = 0;
-    if (lane == 0 && drift_mask) base = atomicAdd(&a.drift_count[is_v ? 1 : 0], static_cast<uint32_t>(__popc(drift_mask)));
+    if (lane == 0 && list_mask) base = atomicAdd(&a.drift_count[is_v ? 1 : 0], static_cast<uint32_t>(__popc(list_mask)));
     base = __shfl_sync(kFull, base, 0);
-    if (too_long)
-      a.drift_list[(is_v ? a.list_cap : 0) + base + __popc(drift_mask & ((1u << lane) - 1u))] = static_cast<uint32_t>(v);
+    if (listed)
+      a.drift_list[(is_v ? a.list_cap : 0) + base + __popc(list_mask & ((1u << lane) - 1u))] =
+          static_cast<uint32_t>(v) | (a.drift_mode == 1 && too_long ? 0x80000000u : 0u);
     drift_mask = 0;
   }
 
@@ -853,12 +861,56 @@ struct DriftArea {
   uint32_t key[kSlots][4][32];  // order_bits of the move key of symbol l + 32 k; kRankedKey once ranked
   int64_t vd[kSlots];
   int32_t ranked[kSlots], win[kSlots];
+  uint16_t pend[kSlots][kWin];  // fill phase: ranked, untested candidates (index | target << 8)
+  int32_t npend[kSlots];
   uint16_t n16[kSlots];
   AppendTables T;
 };
 
-// E6 for one stream's drift list: entries first, first + stride, ... .
-template <bool kTwo, int kStk>
+// Rate-distortion fill keys of the symbols this lane owns in slot s (drift
+// mode 1; the rule of rd_fill): q0 are the quantiser's symbols, qd the
+// symbols after drift. The slot's words become qd | nearest level << 3.
+template <int kStk>
+__device__ __forceinline__ void fill_keys(DriftArea<kStk> &A, int nl, int s, const float (&u)[4],
+                                          const uint32_t (&q0)[4], const uint32_t (&qd)[4], int lane) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    int j = 0;
+    float best = 0.0f;
+    for (int l = 0; l < nl; ++l) {
+      const float d = __fsub_rn(u[k], A.T.lev[l]);
+      const float e = __fmul_rn(d, d);
+      if (l == 0 || e < best) {
+        best = e;
+        j = l;
+      }
+    }
+    const int sd = static_cast<int>(qd[k]);
+    uint32_t key = kNoKey;
+    if (j != sd && abs(j - sd) == 1 && abs(j - static_cast<int>(q0[k])) <= 1) {
+      const float dj = __fsub_rn(u[k], A.T.lev[j]);
+      const float ds = __fsub_rn(u[k], A.T.lev[sd]);
+      const float dd = __fsub_rn(__fmul_rn(dj, dj), __fmul_rn(ds, ds));
+      const float dr = __fsub_rn(A.T.cost[j], A.T.cost[sd]);
+      if (dd < 0.0f && dr > 0.0f) key = order_bits(__fdiv_rn(dd, dr));
+    }
+    A.key[s][k][lane] = key;
+    A.sw[lane + 32 * k][s] =
+        static_cast<uint16_t>(qd[k] | (static_cast<uint32_t>(j) << 3) | (static_cast<uint32_t>(kNoRank) << 6));
+  }
+}
+
+// E6 (and, with kFill, the rate-distortion fill of drift mode 1) for one
+// stream's list: entries first, first + stride, ... . With kFill the list
+// holds every vector (bit 31: over-long); an over-long one drifts first and
+// goes on to the fill from its drifted symbols, the others go straight to
+// the fill. A fill pass tests up to kWin ranked candidates of a slot, each
+// applied alone to the current string (lane kWin c + j: candidate j of the
+// slot's queue); the first that fits is kept and stored by its lane, the
+// ones before it are dropped and the ones after it stay queued. The keys do
+// not change while candidates are kept, so this is the one-at-a-time order's
+// result.
+template <bool kTwo, int kStk, bool kFill>
 __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk> &A, bool is_v, int lane,
                                              uint32_t first, uint32_t stride, DriftCount &dc) {
   __syncwarp();
@@ -866,6 +918,7 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
   if (lane < kSlots) {
     A.ranked[lane] = 0;
     A.win[lane] = 0;
+    A.npend[lane] = 0;
   }
   __syncwarp();
   const uint32_t n = a.drift_count[is_v ? 1 : 0];
@@ -874,45 +927,83 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
   const int cs = lane / kWin, jw = lane % kWin;
   const uint32_t hlf = static_cast<uint32_t>(c.nl / 2);
   uint64_t cursor = first;
-  uint32_t live = 0, exh = 0;  // warp-uniform slot masks: holds a container; candidates ran out
+  // Warp-uniform slot masks: holds a container; candidates ran out; in the
+  // fill phase; drifted to a fit and waiting for its fill keys.
+  uint32_t live = 0, exh = 0, fil = 0, fsu = 0;
   for (;;) {
-    // Free slots take the next list entries: symbols, move targets and keys.
+    if constexpr (kFill) {
+      // Slots that drifted to a fit: fill keys from the drifted symbols
+      // (the first A.win[s] ranked moves applied).
+#pragma unroll 1
+      for (int s = 0; s < kSlots; ++s) {
+        if (!((fsu >> s) & 1u)) continue;
+        const int64_t v = A.vd[s];
+        const int applied = A.win[s];
+        float u[4];
+        uint32_t q0[4], qd[4];
+        uint16_t n16v;
+        bool nf;
+        warp_prepare_regs(a, c.src, v, c.head_of(a, v), c.t, lane, u, q0, &n16v, &nf);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w = A.sw[lane + 32 * k][s];
+          qd[k] = (static_cast<int>(w >> 6) < applied) ? ((w >> 3) & 7u) : (w & 7u);
+        }
+        __syncwarp();
+        fill_keys(A, c.nl, s, u, q0, qd, lane);
+        if (lane == 0) A.npend[s] = 0;
+        fsu &= ~(1u << s);
+        fil |= 1u << s;
+        exh &= ~(1u << s);
+      }
+    }
+    // Free slots take the next list entries.
 #pragma unroll 1
     for (int s = 0; s < kSlots && cursor < n; ++s) {
       if ((live >> s) & 1u) continue;
-      const int64_t v = list[cursor];
+      const uint32_t e = list[cursor];
       cursor += stride;
+      const int64_t v = kFill ? static_cast<int64_t>(e & 0x7FFFFFFFu) : static_cast<int64_t>(e);
+      const bool over = kFill ? (e >> 31) != 0 : true;
       float u[4];
       uint32_t qk[4];
       uint16_t n16v;
       bool nf;
       warp_prepare_regs(a, c.src, v, c.head_of(a, v), c.t, lane, u, qk, &n16v, &nf);
+      if (over) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        int tj;
-        A.key[s][k][lane] = order_bits(best_move(A.T, c.nl, static_cast<int>(qk[k]), u[k], &tj));
-        A.sw[lane + 32 * k][s] =
-            static_cast<uint16_t>(qk[k] | (static_cast<uint32_t>(tj) << 3) | (static_cast<uint32_t>(kNoRank) << 6));
+        for (int k = 0; k < 4; ++k) {
+          int tj;
+          A.key[s][k][lane] = order_bits(best_move(A.T, c.nl, static_cast<int>(qk[k]), u[k], &tj));
+          A.sw[lane + 32 * k][s] = static_cast<uint16_t>(qk[k] | (static_cast<uint32_t>(tj) << 3) |
+                                                         (static_cast<uint32_t>(kNoRank) << 6));
+        }
+        fil &= ~(1u << s);
+      } else {
+        fill_keys(A, c.nl, s, u, qk, qk, lane);
+        fil |= 1u << s;
       }
       if (lane == 0) {
         A.vd[s] = v;
         A.n16[s] = n16v;
         A.ranked[s] = 0;
         A.win[s] = 0;
+        A.npend[s] = 0;
       }
       live |= 1u << s;
       exh &= ~(1u << s);
     }
     if (!live) break;
     __syncwarp();
-    // Every live slot with candidates left ranks its moves up to win + kWin
-    // by repeated arg-min over (key, index): the least key over the warp,
-    // then the lowest index holding it.
+    // Ranking by repeated arg-min over (key, index): the least key over the
+    // warp, then the lowest index holding it. Drift slots rank their moves up
+    // to win + kWin; fill slots top their queue up to kWin candidates.
 #pragma unroll 1
     for (int s = 0; s < kSlots; ++s) {
       if (!(((live & ~exh) >> s) & 1u)) continue;
-      int r = A.ranked[s];
-      const int target = A.win[s] + kWin;
+      const bool fs = kFill && ((fil >> s) & 1u);
+      int r = fs ? A.npend[s] : A.ranked[s];
+      const int target = fs ? kWin : A.win[s] + kWin;
       if (r >= target) continue;
       uint32_t key[4];
 #pragma unroll
@@ -927,26 +1018,37 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             if (bi == lane + 32 * k) key[k] = kRankedKey;
-          A.sw[bi][s] = static_cast<uint16_t>((A.sw[bi][s] & 0x3Fu) | (static_cast<uint32_t>(r) << 6));
+          const uint32_t w = A.sw[bi][s];
+          if (fs) A.pend[s][r] = static_cast<uint16_t>(bi | (((w >> 3) & 7u) << 8));
+          else A.sw[bi][s] = static_cast<uint16_t>((w & 0x3Fu) | (static_cast<uint32_t>(r) << 6));
         }
       }
 #pragma unroll
       for (int k = 0; k < 4; ++k) A.key[s][k][lane] = key[k];
-      if (lane == 0) A.ranked[s] = r;
+      if (lane == 0) {
+        if (fs) A.npend[s] = r;
+        else A.ranked[s] = r;
+      }
     }
     __syncwarp();
-    // One encode pass. An exhausted slot has ranked < win + kWin, so the last
-    // lane of its window is free for the fallback string (all ranked moves,
-    // then every symbol to the innermost level of its side).
+    // One encode pass. An exhausted drift slot has ranked < win + kWin, so the
+    // last lane of its window is free for the fallback string (all ranked
+    // moves, then every symbol to the innermost level of its side).
     const bool mine = (live >> cs) & 1u;
     // A lane whose slot is empty encodes a live slot's string (its words
     // were all written at refill, every symbol below nl); its result is
     // not used.
-    const uint16_t *swc = &A.sw[0][mine ? cs : __ffs(live) - 1];
+    const int cr = mine ? cs : __ffs(live) - 1;
+    const uint16_t *swc = &A.sw[0][cr];
+    const bool lf = kFill && ((fil >> cr) & 1u);
     const int win = A.win[cs], ranked = A.ranked[cs];
     const int km = win + jw;
-    const bool trial = mine && km < ranked;
-    const bool fb = mine && ((exh >> cs) & 1u) && jw == kWin - 1;
+    const bool trial = mine && !lf && km < ranked;
+    const bool fb = mine && !lf && ((exh >> cs) & 1u) && jw == kWin - 1;
+    const bool has = mine && lf && jw < A.npend[cs];
+    const uint32_t cw = has ? A.pend[cs][jw] : 0xFFFFu;
+    const int ci = static_cast<int>(cw & 0xFFu);  // 255 (no candidate) matches no symbol
+    const uint32_t ct = cw >> 8;
     uint32_t x = 0;
     int len;
     if (__any_sync(kFull, fb)) {
@@ -954,6 +1056,9 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
       auto sym = [&](int i) {
         const uint32_t w = swc[i * kSlots];
         uint32_t sy = ((w >> 6) <= kmx) ? ((w >> 3) & 7u) : (w & 7u);
+        if constexpr (kFill) {
+          if (lf) sy = (i == ci) ? ct : (w & 7u);
+        }
         if (fb) sy = sy >= hlf ? hlf : hlf - 1u;
         return sy;
       };
@@ -962,45 +1067,73 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
       const uint32_t kmx = static_cast<uint32_t>(km);
       auto sym = [&](int i) {
         const uint32_t w = swc[i * kSlots];
-        return ((w >> 6) <= kmx) ? ((w >> 3) & 7u) : (w & 7u);
+        uint32_t sy = ((w >> 6) <= kmx) ? ((w >> 3) & 7u) : (w & 7u);
+        if constexpr (kFill) {
+          if (lf) sy = (i == ci) ? ct : (w & 7u);
+        }
+        return sy;
       };
       len = encode_bf<kTwo, false, decltype(sym), kStk>(sym, A.T.es, stk, &x);
     }
     const bool ok = len <= c.P;
-    const unsigned fit = __ballot_sync(kFull, trial && ok);
+    const unsigned fit = __ballot_sync(kFull, (trial || has) && ok);
     const unsigned fc = (fit >> (kWin * cs)) & ((1u << kWin) - 1u);
     const bool store = fc ? (jw == __ffs(fc) - 1) : (fb && ok);
+    __syncwarp();  // every lane has read the slot words of this pass
     if (store) {
       bool dr = false;
       uint8_t *dst = c.dst_of(a, A.vd[cs], &dr);
       if (dst) store_container(dst, c.C, A.n16[cs], x, stk, len);
+      if (kFill && lf) A.sw[ci][cs] = static_cast<uint16_t>((A.sw[ci][cs] & ~7u) | ct);  // kept: new string
     }
     // Slot bookkeeping (warp-uniform).
+    uint32_t drifting = 0;  // drift slots that go on to their next window
 #pragma unroll 1
     for (int s = 0; s < kSlots; ++s) {
       if (!((live >> s) & 1u)) continue;
       const unsigned f = (fit >> (kWin * s)) & ((1u << kWin) - 1u);
-      if (f) {
+      if (kFill && ((fil >> s) & 1u)) {
+        const int np = A.npend[s];
+        const int used = f ? __ffs(f) : np;  // tested candidates resolved by this pass
+        if (f) dc.filled += 1;
+        __syncwarp();
+        if (lane == 0) {
+          for (int t = used; t < np; ++t) A.pend[s][t - used] = A.pend[s][t];
+          A.npend[s] = np - used;
+        }
+        if (np - used == 0 && ((exh >> s) & 1u)) {
+          live &= ~(1u << s);
+          fil &= ~(1u << s);
+        }
+      } else if (f) {
         dc.moves += static_cast<unsigned>(A.win[s] + __ffs(f));
         dc.containers += 1;
-        live &= ~(1u << s);
+        if constexpr (kFill) {
+          __syncwarp();
+          if (lane == 0) A.win[s] = A.win[s] + __ffs(f);  // moves applied
+          fsu |= 1u << s;
+        } else {
+          live &= ~(1u << s);
+        }
       } else if ((exh >> s) & 1u) {
         const int r = A.ranked[s];
         dc.fallbacks += 1;
         dc.moves += static_cast<unsigned>(r);
         dc.containers += r > 0 ? 1u : 0u;
         live &= ~(1u << s);
+      } else {
+        drifting |= 1u << s;
       }
     }
     __syncwarp();
-    if (lane < kSlots && ((live >> lane) & 1u)) A.win[lane] += kWin;
+    if (lane < kSlots && ((drifting >> lane) & 1u)) A.win[lane] += kWin;
     __syncwarp();
   }
 }
 
 // Every warp walks its share of the K list, then of the V list, so the two
 // streams' lists (often of very different lengths) spread over all warps.
-template <bool kTwoK, bool kTwoV, int kStk>
+template <bool kTwoK, bool kTwoV, int kStk, bool kFill>
 __global__ void __launch_bounds__(kDriftWarps * 32, kDriftCtas) append_drift_kernel(const AppendArgs a) {
   __shared__ DriftArea<kStk> A[kDriftWarps];
   const int lane = threadIdx.x & 31;
@@ -1008,8 +1141,8 @@ __global__ void __launch_bounds__(kDriftWarps * 32, kDriftCtas) append_drift_ker
   const uint32_t first = blockIdx.x * kDriftWarps + (threadIdx.x >> 5);
   const uint32_t stride = gridDim.x * kDriftWarps;
   DriftCount dk, dv;
-  drift_stream<kTwoK, kStk>(a, w, false, lane, first, stride, dk);
-  drift_stream<kTwoV, kStk>(a, w, true, lane, first, stride, dv);
+  drift_stream<kTwoK, kStk, kFill>(a, w, false, lane, first, stride, dk);
+  drift_stream<kTwoV, kStk, kFill>(a, w, true, lane, first, stride, dv);
   if (lane == 0) {
     add_stats(a, false, dk, 0u, 0u);
     add_stats(a, true, dv, 0u, 0u);
@@ -1045,18 +1178,19 @@ __global__ void __launch_bounds__(kAW * 32) append_warp_kernel(const AppendArgs 
   }
 }
 
-template <bool kTwoK, bool kTwoV, int kStk>
+template <bool kTwoK, bool kTwoV, int kStk, bool kFill>
 int launch_drift(const AppendArgs &a, int sms, cudaStream_t st) {
   static int per_sm = 0;
   if (per_sm == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV, kStk>, kDriftWarps * 32,
-                                                      0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV, kStk, kFill>,
+                                                      kDriftWarps * 32, 0) != cudaSuccess ||
         n < 1)
       n = 1;
     per_sm = n;
   }
-  append_drift_kernel<kTwoK, kTwoV, kStk><<<static_cast<unsigned>(per_sm * sms), kDriftWarps * 32, 0, st>>>(a);
+  append_drift_kernel<kTwoK, kTwoV, kStk, kFill>
+      <<<static_cast<unsigned>(per_sm * sms), kDriftWarps * 32, 0, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 
@@ -1078,8 +1212,10 @@ int launch_two(const AppendArgs &a, bool lanes, int64_t nvec, int sms, cudaStrea
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || !a.drift_list) return static_cast<int>(e);
   // Drift: a persistent grid, as many CTAs as fit on the SMs at once.
-  if (a.ck <= 36 && a.cv <= 36) return launch_drift<kTwoK, kTwoV, 32>(a, sms, st);
-  return launch_drift<kTwoK, kTwoV, 64>(a, sms, st);
+  const bool small = a.ck <= 36 && a.cv <= 36;
+  if (a.drift_mode == 1)
+    return small ? launch_drift<kTwoK, kTwoV, 32, true>(a, sms, st) : launch_drift<kTwoK, kTwoV, 64, true>(a, sms, st);
+  return small ? launch_drift<kTwoK, kTwoV, 32, false>(a, sms, st) : launch_drift<kTwoK, kTwoV, 64, false>(a, sms, st);
 }
 
 template <bool kBF16>
@@ -1100,11 +1236,16 @@ int launch_append(const AppendArgs &a, void *stream) {
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // Lane per vector once every SM gets a few full CTAs of 128 vectors per
   // stream; below that, a warp per vector spreads the work wider.
-  // Drift mode 1 (rate-distortion fill) runs in the warp-per-vector kernel.
-  const bool lanes = a.drift_mode == 0 && nvec >= static_cast<int64_t>(sms) * kAW * 32 * 2;
+  bool lanes = nvec >= static_cast<int64_t>(sms) * kAW * 32 * 2;
   AppendArgs b = a;
   // The drift list holds 32-bit vector indices, one slot per vector.
   if (!lanes || b.list_cap < nvec || nvec > 0xFFFFFFFFll) b.drift_list = nullptr;
+  // Drift mode 1 needs the list (its fill runs in the drift kernel, with the
+  // over-long flag in bit 31); without it, the warp-per-vector kernel fills.
+  if (a.drift_mode == 1 && (!b.drift_list || nvec > 0x7FFFFFFFll)) {
+    lanes = false;
+    b.drift_list = nullptr;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return b.dtype == DQ_BF16 ? launch_dtype<true>(b, lanes, nvec, sms, st) : launch_dtype<false>(b, lanes, nvec, sms, st);
 }

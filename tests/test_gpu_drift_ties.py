@@ -107,3 +107,16 @@ def test_tied_keys_rate_distortion_fill():
     K, V = _tied_inputs(ref, 2, 2, 200, (1, 2, 8), (0.6, 0.3, 0.1), seed=4)
     kst, vst = _check(lib, ref, K, V, torch.float32, drift_mode=1)
     assert kst.cont_drifted > 50 and kst.syms_filled + vst.syms_filled > 0
+
+
+@pytest.mark.gpu
+def test_tied_keys_rate_distortion_fill_large():
+    # The lane-per-vector kernel, then the drift kernel's fill phase.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    B, Hkv = 4, 2
+    T = -(-(sms * 128 * 2 + 64) // (B * Hkv))
+    lib = dq.dq_build_tables(n_kv_heads=Hkv, drift_mode=1)
+    ref = o.Tables(Hkv, drift_mode=1)
+    K, V = _tied_inputs(ref, B, Hkv, T, (1, 2, 8), (0.6, 0.3, 0.1), seed=5)
+    kst, vst = _check(lib, ref, K, V, torch.float32, drift_mode=1)
+    assert kst.cont_drifted > B * Hkv * T // 10 and kst.syms_filled + vst.syms_filled > 0

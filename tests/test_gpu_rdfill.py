@@ -1,8 +1,9 @@
 """Drift mode 1 (drift, then the rate-distortion fill) on the GPU against the
 oracle: containers bit-identical to attention's input definition, the same
 drift and fill counts, at 1.96, 2.26 and 3.0 bits per value, for a small
-append (one token per sequence), a large one (which takes the lane-per-vector
-kernel in mode 0) and paged pools; attention over the filled caches matches
+append (one token per sequence, the warp-per-vector kernel with its fill), a
+large one (the lane-per-vector kernel, then the drift kernel's fill phase for
+every container) and paged pools; attention over the filled caches matches
 the fp64 oracle, and the fill lowers the reconstruction error of the
 synthetic rows as the oracle says it does.
 """
@@ -26,7 +27,8 @@ def _tables(Hkv, bits):
 
 
 @pytest.mark.parametrize("bits,B,T,dtype", [(2.26, 2, 300, torch.bfloat16), (1.96, 3, 100, torch.float32),
-                                            (3.0, 2, 64, torch.bfloat16), (2.26, 2, 4096, torch.bfloat16)])
+                                            (3.0, 2, 64, torch.bfloat16), (2.26, 2, 4096, torch.bfloat16),
+                                            (1.96, 2, 4096, torch.float32), (3.0, 2, 4096, torch.bfloat16)])
 def test_fill_containers_bit_exact(bits, B, T, dtype):
     Hkv = 8 if T == 4096 else 2
     w = synth.scaled(synth.WORKLOADS["qwen3_8b_b16_t8k"], B=B, Hkv=Hkv, Hq=4 * Hkv, T=T)
