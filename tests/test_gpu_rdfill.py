@@ -69,8 +69,10 @@ def test_fill_one_token_steps_and_attention():
     cm.assert_attention_close(got, o.attention_fp64(ref, q, rk, rv, lens), what="attention over filled caches")
 
 
-def test_fill_paged_matches_contiguous():
-    B, Hkv, T = 2, 2, 256
+@pytest.mark.parametrize("B,Hkv,T", [(2, 2, 256), (4, 8, 1280)])
+def test_fill_paged_matches_contiguous(B, Hkv, T):
+    # (4, 8, 1280): 40,960 vectors per stream take the lane kernel and the
+    # drift kernel's fill, writing through the page table.
     w = synth.scaled(synth.WORKLOADS["qwen3_8b_b16_t8k"], B=B, Hkv=Hkv, Hq=4 * Hkv, T=T)
     K, V, _ = cm.inputs(w)
     lib, ref = _tables(Hkv, 2.26)
