@@ -191,6 +191,51 @@ def dist_setup(args):
     return ws, rank, local
 
 
+def run_pipelined(nst, stream, n_in, n_out, h2d, compute, d2h, t_start=None, t_end=None):
+    """nst end-to-end steps with the copies on their own streams, pipelined
+    with the kernels on `stream`: step s+1's inputs go in (h2d(s) on an
+    upload stream) and step s's output comes back (d2h(s) on a read-back
+    stream) while kernels run. Events keep every dependency: compute(s)
+    waits for its inputs; input buffer s % n_in is refilled only after the
+    step that last read it has finished; output buffer s % n_out is rewritten
+    only after its read-back; t_end (on `stream`) follows the last
+    read-back, t_start precedes the first upload."""
+    import torch
+
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(nst)]
+    ev_done = [torch.cuda.Event() for _ in range(nst)]
+    ev_out = [torch.cuda.Event() for _ in range(nst)]
+    start = t_start if t_start is not None else torch.cuda.Event()
+    start.record(stream)
+    up.wait_event(start)
+    down.wait_event(start)
+
+    def upload(s):
+        if s >= n_in:
+            up.wait_event(ev_done[s - n_in])
+        with torch.cuda.stream(up):
+            h2d(s)
+        ev_in[s].record(up)
+
+    upload(0)
+    for s in range(nst):
+        if s + 1 < nst:
+            upload(s + 1)
+        stream.wait_event(ev_in[s])
+        if s >= n_out:
+            stream.wait_event(ev_out[s - n_out])
+        compute(s)
+        ev_done[s].record(stream)
+        down.wait_event(ev_done[s])
+        with torch.cuda.stream(down):
+            d2h(s)
+        ev_out[s].record(down)
+    stream.wait_event(ev_out[nst - 1])
+    if t_end is not None:
+        t_end.record(stream)
+
+
 def run_dq(args):
     import numpy as np
     import torch
@@ -271,12 +316,13 @@ def run_dq(args):
             dq.dq_append_kv_paged(tab, dev_k[i], dev_v[i], start, kl, vl, page_table, stats=stats,
                                   stream=st, workspace=app_ws)
 
-    def decode(i, layer, st):
+    def decode(i, layer, st, o=None):
         kl, vl = caches[layer]
+        o = out if o is None else o
         if page_table is None:
-            dq.dq_decode_attention(tab, dev_q[i], kl, vl, seq, T, out, wsp, stats=stats, stream=st)
+            dq.dq_decode_attention(tab, dev_q[i], kl, vl, seq, T, o, wsp, stats=stats, stream=st)
         else:
-            dq.dq_decode_attention_paged(tab, dev_q[i], kl, vl, page_table, seq, T, out, wsp, stats=stats,
+            dq.dq_decode_attention_paged(tab, dev_q[i], kl, vl, page_table, seq, T, o, wsp, stats=stats,
                                          stream=st)
 
     def step(s, ev=None, st=None):
@@ -340,26 +386,36 @@ def run_dq(args):
     value = whole_job_rate(kv_tokens_step, ws, ms_per_step)
 
     # ---- e2e: host buffers, copies inside the timed region ----
-    def step_e2e(s):
+    # Every step copies its new K/V and q in from pinned host memory and its
+    # output back, pipelined with the kernels (run_pipelined); the inputs
+    # cycle over nsteps_inputs device buffers, the outputs over two.
+    outs = [out, torch.empty_like(out)]
+    outs_host = [out_host, torch.empty_like(out_host).pin_memory()]
+
+    def e2e_h2d(s):
         i = s % nsteps_inputs
         dev_k[i].copy_(host_k[i], non_blocking=True)
         dev_v[i].copy_(host_v[i], non_blocking=True)
         dev_q[i].copy_(host_q[i], non_blocking=True)
+
+    def e2e_compute(s):
+        i = s % nsteps_inputs
         for layer in range(L):
             append(i, layer, stream)
-            decode(i, layer, stream)
-        out_host.copy_(out, non_blocking=True)
+            decode(i, layer, stream, outs[s % 2])
 
-    for s in range(2):
-        step_e2e(s)
+    def e2e_d2h(s):
+        outs_host[s % 2].copy_(outs[s % 2], non_blocking=True)
+
+    def run_e2e(nst, t_start=None, t_end=None):
+        run_pipelined(nst, stream, nsteps_inputs, 2, e2e_h2d, e2e_compute, e2e_d2h, t_start, t_end)
+
+    run_e2e(2)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for s in range(args.steps):
-        step_e2e(s)
-    f1.record(stream)
+    run_e2e(args.steps, f0, f1)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks([f0.elapsed_time(f1)], dist, dev)[0]
@@ -440,7 +496,9 @@ def run_dq(args):
                          "kernel_ms": dec_ms, "peak_source": "%s clock, %d SMs x 128 lanes" % (src, sm_count),
                          "hbm": {"achieved_gbs": hbm_gbs, "peak_gbs": peaks.get("hbm_gbs"),
                                  "frac": hbm_gbs / float(peaks.get("hbm_gbs", 6650.0))}},
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "copies": "every step's inputs in and output out, on upload and read-back streams "
+                              "pipelined with the kernels"},
             "gpu_launches": LAUNCHES_PER_STEP * L * args.steps,
             "clocks": clk,
             "drift": {"prefill_k_syms_filled_pct": 100.0 * pstats["k_syms_filled"] / (token_heads * 128),
@@ -700,21 +758,32 @@ def run_prefill(args):
     qtok = w.B * n_q
     value = whole_job_rate(qtok, ws, ms_per_step)
 
-    def step_e2e():
-        dk.copy_(host_k, non_blocking=True)
-        dv.copy_(host_v, non_blocking=True)
-        dqq.copy_(host_q, non_blocking=True)
-        step()
-        out_host.copy_(out, non_blocking=True)
+    # End to end: the chunk's K/V and q in from pinned host memory and the
+    # output back every step, pipelined with the kernels (run_pipelined) over
+    # two device buffer sets.
+    bufs = [(dk, dv, dqq, out), (torch.empty_like(dk), torch.empty_like(dv), torch.empty_like(dqq),
+                                 torch.empty_like(out))]
+    outs_host = [out_host, torch.empty_like(out_host).pin_memory()]
 
-    step_e2e()
+    def e2e_h2d(s):
+        bk, bv, bq, _ = bufs[s % 2]
+        bk.copy_(host_k, non_blocking=True)
+        bv.copy_(host_v, non_blocking=True)
+        bq.copy_(host_q, non_blocking=True)
+
+    def e2e_compute(s):
+        bk, bv, bq, bo = bufs[s % 2]
+        dq.dq_append_kv(tab, bk, bv, start, kc, vc, stats=stats, workspace=app_ws)
+        dq.dq_prefill_attention(tab, bq, kc, vc, start, bo, workspace=pf_ws, stats=stats)
+
+    def e2e_d2h(s):
+        outs_host[s % 2].copy_(bufs[s % 2][3], non_blocking=True)
+
+    run_pipelined(2, stream, 2, 2, e2e_h2d, e2e_compute, e2e_d2h)
     torch.cuda.synchronize()
     barrier()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(args.steps):
-        step_e2e()
-    f1.record(stream)
+    run_pipelined(args.steps, stream, 2, 2, e2e_h2d, e2e_compute, e2e_d2h, f0, f1)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks([f0.elapsed_time(f1)], dist, dev)[0]
@@ -751,7 +820,9 @@ def run_prefill(args):
                          "kernel_ms": attn_ms,
                          "peak_source": "%s bf16 dense GEMM (fp16 runs at the same rate)" % src},
             "e2e": {"value": whole_job_rate(qtok, ws, e2e_ms / args.steps), "unit": PREFILL_UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
+                    "copies": "every step's inputs in and output out, on upload and read-back streams "
+                              "pipelined with the kernels"},
             "gpu_launches": PREFILL_LAUNCHES_PER_STEP * args.steps,
             "clocks": clk,
             "integrity_errors": st["integrity_errors"], "wait_timeouts": st["wait_timeouts"],
