@@ -644,8 +644,13 @@ PREFILL_UNIT = "query tokens/s"
 # multiply-adds each.
 FLOPS_PER_PAIR = 4 * 128
 # Kernel launches of one prefill step: dq_append_kv of the chunk (encode +
-# drift kernels) and dq_prefill_attention (tile decode + attention kernels).
+# drift kernels; in drift mode 1 the drift kernel runs once per stream) and
+# dq_prefill_attention (tile decode + attention kernels).
 PREFILL_LAUNCHES_PER_STEP = 4
+
+
+def prefill_launches_per_step(drift_mode):
+    return PREFILL_LAUNCHES_PER_STEP + (1 if drift_mode == 1 else 0)
 
 
 # DRAM traffic of prefill_kernel (the dominant kernel of the prefill step)
@@ -823,7 +828,7 @@ def run_prefill(args):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_host.numel() * out_host.element_size(),
                     "copies": "every step's inputs in and output out, on upload and read-back streams "
                               "pipelined with the kernels"},
-            "gpu_launches": PREFILL_LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": prefill_launches_per_step(args.drift_mode) * args.steps,
             "clocks": clk,
             "integrity_errors": st["integrity_errors"], "wait_timeouts": st["wait_timeouts"],
         }

@@ -1133,7 +1133,10 @@ __device__ __forceinline__ void drift_stream(const AppendArgs &a, DriftArea<kStk
 
 // Every warp walks its share of the K list, then of the V list, so the two
 // streams' lists (often of very different lengths) spread over all warps.
-template <bool kTwoK, bool kTwoV, int kStk, bool kFill>
+// kWhich 0 or 1: the K or the V list only (drift mode 1, whose lists hold
+// every vector and so have equal lengths: one launch per stream keeps each
+// launch's code to one stream's body, which the fill phase makes large).
+template <bool kTwoK, bool kTwoV, int kStk, bool kFill, int kWhich>
 __global__ void __launch_bounds__(kDriftWarps * 32, kDriftCtas) append_drift_kernel(const AppendArgs a) {
   __shared__ DriftArea<kStk> A[kDriftWarps];
   const int lane = threadIdx.x & 31;
@@ -1141,8 +1144,8 @@ __global__ void __launch_bounds__(kDriftWarps * 32, kDriftCtas) append_drift_ker
   const uint32_t first = blockIdx.x * kDriftWarps + (threadIdx.x >> 5);
   const uint32_t stride = gridDim.x * kDriftWarps;
   DriftCount dk, dv;
-  drift_stream<kTwoK, kStk, kFill>(a, w, false, lane, first, stride, dk);
-  drift_stream<kTwoV, kStk, kFill>(a, w, true, lane, first, stride, dv);
+  if constexpr (kWhich != 1) drift_stream<kTwoK, kStk, kFill>(a, w, false, lane, first, stride, dk);
+  if constexpr (kWhich != 0) drift_stream<kTwoV, kStk, kFill>(a, w, true, lane, first, stride, dv);
   if (lane == 0) {
     add_stats(a, false, dk, 0u, 0u);
     add_stats(a, true, dv, 0u, 0u);
@@ -1178,20 +1181,28 @@ __global__ void __launch_bounds__(kAW * 32) append_warp_kernel(const AppendArgs 
   }
 }
 
-template <bool kTwoK, bool kTwoV, int kStk, bool kFill>
-int launch_drift(const AppendArgs &a, int sms, cudaStream_t st) {
+template <bool kTwoK, bool kTwoV, int kStk, bool kFill, int kWhich>
+int launch_drift_one(const AppendArgs &a, int sms, cudaStream_t st) {
   static int per_sm = 0;
   if (per_sm == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV, kStk, kFill>,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_drift_kernel<kTwoK, kTwoV, kStk, kFill, kWhich>,
                                                       kDriftWarps * 32, 0) != cudaSuccess ||
         n < 1)
       n = 1;
     per_sm = n;
   }
-  append_drift_kernel<kTwoK, kTwoV, kStk, kFill>
+  append_drift_kernel<kTwoK, kTwoV, kStk, kFill, kWhich>
       <<<static_cast<unsigned>(per_sm * sms), kDriftWarps * 32, 0, st>>>(a);
   return static_cast<int>(cudaGetLastError());
+}
+
+template <bool kTwoK, bool kTwoV, int kStk, bool kFill>
+int launch_drift(const AppendArgs &a, int sms, cudaStream_t st) {
+  if constexpr (!kFill) return launch_drift_one<kTwoK, kTwoV, kStk, false, -1>(a, sms, st);
+  const int e = launch_drift_one<kTwoK, kTwoV, kStk, true, 0>(a, sms, st);
+  if (e != 0) return e;
+  return launch_drift_one<kTwoK, kTwoV, kStk, true, 1>(a, sms, st);
 }
 
 template <bool kBF16, bool kTwoK, bool kTwoV>
