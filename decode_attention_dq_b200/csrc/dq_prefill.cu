@@ -73,6 +73,7 @@ constexpr int kSlotBytes = 2 * kTileBytes + 2 * kBlk * 4;  // K tile, V tile, K 
 constexpr int kChunkStride = kBlk / 8 * 128;               // bytes between 8-coordinate chunks of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kSpin = 1u << 24;  // bound on each mbarrier wait loop
+constexpr float kLazyLog2 = 8.0f;      // lazy rescaling: largest growth (log2) of the row maximum kept stale
 // Barrier slots of prefill_kernel.
 constexpr int kBarFull = 0, kBarEmpty = kMaxSlots, kBarSFull = 2 * kMaxSlots, kBarWFull = kBarSFull + 2,
               kBarPvDone = kBarSFull + 4, kBarQFull = kBarSFull + 6, kBarDrain = kBarSFull + 7,
@@ -109,7 +110,7 @@ __host__ __device__ inline TilesSmem tiles_smem_layout(int ck, int cv) {
 // flag, the row-max exchange [2 blocks][2 halves][128 rows] and the row-sum
 // exchange [2 halves][128 rows] of the softmax warp pairs, then the ring.
 struct AttnSmem {
-  size_t bars, misc, pmax, lsum, ring, total;
+  size_t bars, misc, pmax, lsum, pnv, ring, total;
 };
 
 __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
@@ -118,7 +119,8 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
   s.misc = s.bars + kNumBars * 8;
   s.pmax = align_up(s.misc + 16, 16);
   s.lsum = s.pmax + 2 * 2 * kRows * 4;
-  s.ring = align_up(s.lsum + 2 * kRows * 4, 128);
+  s.pnv = s.lsum + 2 * kRows * 4;
+  s.ring = align_up(s.pnv + 2 * 2 * kRows * 4, 128);
   s.total = s.ring + static_cast<size_t>(nslots) * kSlotBytes;
   return s;
 }
@@ -462,6 +464,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + L.misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 4);
   float *pmax = reinterpret_cast<float *>(smem + L.pmax);  // [2][2][128]
+  float *pnv = reinterpret_cast<float *>(smem + L.pnv);    // [2][2][128]: largest V norm of a row half
   float *lsum = reinterpret_cast<float *>(smem + L.lsum);  // [2][128]
   auto slot_base = [&](int d) { return smem + L.ring + static_cast<size_t>(d) * kSlotBytes; };
 
@@ -610,11 +613,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       for (int w2 = 16; w2 >= 1; w2 >>= 1)
 #pragma unroll
         for (int t = 0; t < w2; ++t) mu[t] = fmaxf(mu[t], mu[t + w2]);
-      // Row maximum over both halves: exchange through shared memory.
+      // Largest V norm of this half's tokens (bounds the weights below).
+      const float *nv = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + kBlk + 64 * half;
+      float mnv = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 64; t += 4) {
+        const float4 n4 = *reinterpret_cast<const float4 *>(nv + t);
+        mnv = fmaxf(mnv, fmaxf(fmaxf(n4.x, n4.y), fmaxf(n4.z, n4.w)));
+      }
+      // Row maximum and largest V norm over both halves: exchange through
+      // shared memory.
       pmax[(sb * 2 + half) * kRows + r] = mu[0];
+      pnv[(sb * 2 + half) * kRows + r] = mnv;
       pair_sync(pair_id);
       const float mrow = fmaxf(mu[0], pmax[(sb * 2 + (half ^ 1)) * kRows + r]);
-      const float mx = mrow == -INFINITY ? m_run : fmaxf(m_run, mrow * crow);
+      const float vmax = fmaxf(mnv, pnv[(sb * 2 + (half ^ 1)) * kRows + r]);
+      const float mcand = mrow == -INFINITY ? m_run : fmaxf(m_run, mrow * crow);
+      // Lazy rescaling: the running maximum stays while the block's is at most
+      // kLazyLog2 above it and the weights p ||v|| <= 2^(mcand - m_run) vmax
+      // stay within half the fp16 range; O, l and the weights all use the
+      // same maximum, so the result is the same. Both halves of a row decide
+      // alike (same inputs).
+      const float mx = (m_run != -INFINITY && mcand - m_run <= kLazyLog2 && ex2(mcand - m_run) * vmax <= 32768.0f)
+                           ? m_run
+                           : mcand;
       float alpha = 1.0f;
       uint32_t whi[32], wlo[32];
       float psum = 0.0f;
@@ -622,10 +644,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
         for (int p = 0; p < 32; ++p) whi[p] = wlo[p] = 0u;
       } else {
-        if (m_run != -INFINITY) alpha = ex2(m_run - mx);
+        if (m_run != -INFINITY && mx != m_run) alpha = ex2(m_run - mx);
         // p = 2^(logit - mx); w = p ||v|| (norms of tokens past the last
         // attended position are 0, so masked tokens give exactly 0).
-        const float *nv = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + kBlk + 64 * half;
         float ps[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int p = 0; p < 32; ++p) {
@@ -637,13 +658,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
         m_run = mx;
       }
       l_run = l_run * alpha + psum;
-      // O is current once P.V of the previous block is done.
-      ok = j == 0 ||
+      // Rescaling O needs P.V of the previous block done; W goes over this
+      // block's own score columns and needs nothing more. (The P.V-done
+      // barrier of block j - 1 cannot run a phase further before this warp
+      // writes W of block j + 1, so the parity wait is unambiguous.)
+      const bool resc = j > 0 && __any_sync(kFull, alpha != 1.0f);
+      ok = !resc ||
            mbar_wait(bars + kBarPvDone + ((j - 1) & 1), static_cast<uint32_t>(((j - 1) >> 1) & 1), abort_flag);
       ok = __all_sync(kFull, ok);
       if (ok) {
         tc_fence_after();
-        if (j > 0 && __any_sync(kFull, alpha != 1.0f)) {
+        if (resc) {
 #pragma unroll 1
           for (int c = 0; c < 64; c += 32) {
             float o[32];
