@@ -638,26 +638,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
                            ? m_run
                            : mcand;
       float alpha = 1.0f;
-      uint32_t whi[32], wlo[32];
-      float psum = 0.0f;
-      if (mx == -INFINITY) {
-#pragma unroll
-        for (int p = 0; p < 32; ++p) whi[p] = wlo[p] = 0u;
-      } else {
-        if (m_run != -INFINITY && mx != m_run) alpha = ex2(m_run - mx);
-        // p = 2^(logit - mx); w = p ||v|| (norms of tokens past the last
-        // attended position are 0, so masked tokens give exactly 0).
-        float ps[2] = {0.0f, 0.0f};
-#pragma unroll
-        for (int p = 0; p < 32; ++p) {
-          const float p0 = ex2(fmaf(u[2 * p], crow, -mx)), p1 = ex2(fmaf(u[2 * p + 1], crow, -mx));
-          ps[p & 1] += p0 + p1;
-          split_pair(p0 * nv[2 * p], p1 * nv[2 * p + 1], whi[p], wlo[p]);
-        }
-        psum = ps[0] + ps[1];
-        m_run = mx;
-      }
-      l_run = l_run * alpha + psum;
+      if (mx != -INFINITY && m_run != -INFINITY && mx != m_run) alpha = ex2(m_run - mx);
       // Rescaling O needs P.V of the previous block done; W goes over this
       // block's own score columns and needs nothing more. (The P.V-done
       // barrier of block j - 1 cannot run a phase further before this warp
@@ -666,6 +647,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       ok = !resc ||
            mbar_wait(bars + kBarPvDone + ((j - 1) & 1), static_cast<uint32_t>(((j - 1) >> 1) & 1), abort_flag);
       ok = __all_sync(kFull, ok);
+      float psum = 0.0f;
       if (ok) {
         tc_fence_after();
         if (resc) {
@@ -684,28 +666,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
             tmem_st16(oc + 16, w1);
           }
         }
-        // W in place of this warp's own score columns: hi in the first 32,
-        // lo in the next 32 (the scores were read above).
-        uint32_t w0[16], w1[16];
+        // W in place of this warp's own score columns (the scores were read
+        // above), 16 tokens at a time: p = 2^(logit - mx), w = p ||v|| as fp16
+        // hi (columns 0..31) and lo (32..63); norms of tokens past the last
+        // attended position are 0, so masked tokens give exactly 0.
+        float ps[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          w0[e] = whi[e];
-          w1[e] = whi[16 + e];
-        }
-        tmem_st16(scol, w0);
-        tmem_st16(scol + 16, w1);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t wh[8], wl[8];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          w0[e] = wlo[e];
-          w1[e] = wlo[16 + e];
+          for (int p = 0; p < 8; ++p) {
+            const int t = 16 * c + 2 * p;
+            float p0 = 0.0f, p1 = 0.0f;
+            if (mx != -INFINITY) {
+              p0 = ex2(fmaf(u[t], crow, -mx));
+              p1 = ex2(fmaf(u[t + 1], crow, -mx));
+            }
+            ps[p & 1] += p0 + p1;
+            split_pair(p0 * nv[t], p1 * nv[t + 1], wh[p], wl[p]);
+          }
+          tmem_st8(scol + 8 * c, wh);
+          tmem_st8(scol + 32 + 8 * c, wl);
         }
-        tmem_st16(scol + 32, w0);
-        tmem_st16(scol + 48, w1);
+        psum = ps[0] + ps[1];
         tmem_wait_st();
       } else {
         ++timeouts;
         alive = false;  // both warps stop at the next agreement
       }
+      if (mx != -INFINITY) m_run = mx;
+      l_run = l_run * alpha + psum;
       tc_fence_before();
       mbar_arrive(bars + kBarWFull + sb);  // always, so the MMA warp's count completes
     }
