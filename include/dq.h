@@ -179,8 +179,9 @@ int dq_get_signs(const dq_tables *t, int8_t *signs);
  * moving symbols one level up to their nearest level (at most one level from
  * the quantiser's symbol), best error reduction per bit first, each kept
  * only if the exact coded length still fits (none after a fallback). The
- * decoder is unchanged; encoding is several times slower (every append then
- * runs a warp per vector). */
+ * decoder is unchanged; encoding is about 15 times slower. Large appends
+ * with a workspace (dq_append_kv_ws) run the fill in the drift kernel, one
+ * launch per stream; the others run a warp per vector. */
 int dq_append_kv(const dq_tables *t, const void *k, const void *v, int dtype,
                  int B, int Hkv, int n_new, const int32_t *d_start_pos,
                  uint8_t *d_kcache, uint8_t *d_vcache, int64_t T_cap,
@@ -193,10 +194,10 @@ size_t dq_append_workspace_bytes(const dq_tables *t, int B, int Hkv, int n_new);
 
 /* dq_append_kv with a caller-provided device workspace (16-byte aligned, at
  * least dq_append_workspace_bytes; contents need not be initialised). Large
- * appends then list their over-long containers there and drift them ([news]
- * "Drift: Bending Variable Back to Fixed") in a separate kernel that runs
- * at higher occupancy than the encode kernel; the containers are the same
- * bytes as with dq_append_kv. d_workspace NULL gives dq_append_kv. Calls
+ * appends then list their over-long containers there (with drift_mode 1,
+ * every container) and drift them ([news] "Drift: Bending Variable Back to
+ * Fixed") in a separate kernel that runs at higher occupancy than the encode
+ * kernel; the containers are the same bytes as with dq_append_kv. d_workspace NULL gives dq_append_kv. Calls
  * sharing a workspace must not overlap on the GPU. DQ_ERR_WORKSPACE if
  * ws_bytes is too small, DQ_ERR_ALIGN if the workspace is misaligned. */
 int dq_append_kv_ws(const dq_tables *t, const void *k, const void *v, int dtype,
