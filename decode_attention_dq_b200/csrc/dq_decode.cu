@@ -271,6 +271,12 @@ __device__ __forceinline__ int64_t clamp_len(int32_t len, int64_t cap) {
 // [first(w), first(w + 1))).
 __host__ __device__ __forceinline__ int64_t warp_first(int64_t w, int64_t W, int64_t N) { return (w * N) / W; }
 
+// Warps that split N groups out of the grid's `total`: min(total, N). With
+// W <= N every warp owns at least one group, so the warps whose ranges meet
+// a (b, h) form one contiguous run with no empty warp in it; with W = N warp
+// w owns exactly group w.
+__host__ __device__ __forceinline__ int64_t active_warps(int64_t total, int64_t N) { return total < N ? total : N; }
+
 // Token groups per sequence and their prefix sums: prefix[b] = groups of
 // sequences 0..b-1, prefix[B] = total. One CTA of kPrefixThreads threads;
 // also counts the sequence lengths that had to be clamped.
@@ -358,8 +364,11 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
   const int64_t cap = a.T_max < a.T_cap ? a.T_max : a.T_cap;
   const int64_t Hkv = a.Hkv;
   const int64_t N = a.prefix[a.B] * Hkv;  // total token groups
-  const int64_t W = static_cast<int64_t>(gridDim.x) * nwarps;
+  // Warps that take part: all of them, or one per group when there are
+  // fewer groups than warps, so that no participating warp is empty.
+  const int64_t W = active_warps(static_cast<int64_t>(gridDim.x) * nwarps, N);
   const int64_t wid = static_cast<int64_t>(blockIdx.x) * nwarps + warp;
+  if (wid >= W) return;
   int64_t g = warp_first(wid, W, N);
   const int64_t g_end = warp_first(wid + 1, W, N);
   if (g >= g_end) return;
@@ -601,53 +610,95 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
   if (a.stats && lane == 0 && bad_pages) atomicAdd(&a.stats->bad_pages, static_cast<unsigned long long>(bad_pages));
 }
 
-__global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);  // b * Hq + hq
-  if (row >= static_cast<int64_t>(a.B) * a.Hq) return;
+// Combine: one CTA of kCombWarps warps per (b, query head). The warps split
+// the row's slots into contiguous chunks; a warp takes its chunk 32 slots at
+// a time (lane i reads slot i's (m, l), so the batch's weights come from one
+// load per lane and one max/sum over the warp; the partial o vectors of the
+// batch are then read with independent loads), merging batch after batch
+// with an online rescale. The warps' results meet in shared memory.
+constexpr int kCombWarps = 4;
+
+__global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(const DecodeArgs a) {
+  __shared__ float sh_m[kCombWarps], sh_l[kCombWarps];
+  __shared__ float sh_o[kCombWarps][kD];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row = blockIdx.x;  // b * Hq + hq
   const int b = static_cast<int>(row / a.Hq), hq = static_cast<int>(row % a.Hq);
   const int G = a.G;
   const int h = hq / G, gg = hq % G;
   const int64_t Hkv = a.Hkv;
-  const int64_t N = a.prefix[a.B] * Hkv;
-  const int64_t W = a.total_warps;
   const int64_t gb = a.prefix[b + 1] - a.prefix[b];
   const int64_t bh = static_cast<int64_t>(b) * Hkv + h;
-  float M = -INFINITY;
+  float M = -INFINITY, Ls = 0.0f;
   float v[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  float Ls = 0.0f;
   if (gb > 0) {
-    // Warps whose ranges cover groups [g0, g1) of (b, h): from the warp
-    // holding g0 to the warp holding g1 - 1 (the warp holding g is the
-    // largest w with first(w) <= g), skipping warps with empty ranges.
+    // The warps whose ranges meet groups [g0, g1) of (b, h) are the
+    // contiguous run from the owner of g0 to the owner of g1 - 1 (owner(g) =
+    // the largest w with first(w) <= g); none of them is empty (W <= N), and
+    // each wrote its partial state of (b, h) to slot bh + w.
+    const int64_t N = a.prefix[a.B] * Hkv;
+    const int64_t W = active_warps(a.total_warps, N);
     const int64_t g0 = a.prefix[b] * Hkv + h * gb, g1 = g0 + gb;
     const int64_t w_lo = ((g0 + 1) * W - 1) / N;
     const int64_t w_hi = (g1 * W - 1) / N;
-    auto covers = [&](int64_t w) {
-      const int64_t s = warp_first(w, W, N), e = warp_first(w + 1, W, N);
-      return s < e && s < g1 && e > g0;
-    };
-    for (int64_t w = w_lo; w <= w_hi; ++w)
-      if (covers(w)) M = fmaxf(M, a.ws_ml[((bh + w) * G + gg) * 2]);
-    if (M != -INFINITY)
-      for (int64_t w = w_lo; w <= w_hi; ++w) {
-        if (!covers(w)) continue;
-        const int64_t slot = bh + w;
-        const float ms = a.ws_ml[(slot * G + gg) * 2];
-        if (ms == -INFINITY) continue;
-        const float sc = exp2f(ms - M);
-        Ls = fmaf(sc, a.ws_ml[(slot * G + gg) * 2 + 1], Ls);
+    const int64_t S = w_hi - w_lo + 1;
+    const int64_t cs = (S + kCombWarps - 1) / kCombWarps;
+    const int64_t c0 = w_lo + warp * cs;
+    const int64_t c1 = (c0 + cs < w_hi + 1) ? c0 + cs : w_hi + 1;
+    const float2 *ml = reinterpret_cast<const float2 *>(a.ws_ml);
+    for (int64_t base = c0; base < c1; base += 32) {
+      const int64_t w = base + lane;
+      float2 s = make_float2(-INFINITY, 0.0f);
+      if (w < c1) s = ml[(bh + w) * G + gg];
+      const float bm = warp_max(s.x);
+      if (bm == -INFINITY) continue;  // all segments of the batch empty
+      const float m_new = fmaxf(M, bm);
+      const float r = exp2f(M - m_new);  // 0 while M is -inf
+      Ls *= r;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = fmaf(sc, a.ws_o[(slot * G + gg) * kD + lane + 32 * k], v[k]);
+      for (int k = 0; k < 4; ++k) v[k] *= r;
+      M = m_new;
+      const float sc = exp2f(s.x - M);  // 0 for lanes past the chunk or empty segments
+      Ls += warp_sum(sc * s.y);
+      const int nb = static_cast<int>((c1 - base) < 32 ? (c1 - base) : 32);
+#pragma unroll 8
+      for (int i = 0; i < nb; ++i) {
+        const float si = __shfl_sync(kFull, sc, i);
+        const float *o = a.ws_o + ((bh + base + i) * G + gg) * kD + lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = fmaf(si, o[32 * k], v[k]);
       }
+    }
   }
-  const float inv = (Ls > 0.0f) ? 1.0f / (Ls * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
-  wht128_warp(v, lane);
+  if (lane == 0) {
+    sh_m[warp] = M;
+    sh_l[warp] = Ls;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) sh_o[warp][lane + 32 * k] = v[k];
+  __syncthreads();
+  if (warp != 0) return;
+  float Mt = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kCombWarps; ++w) Mt = fmaxf(Mt, sh_m[w]);
+  float Lt = 0.0f;
+  float o[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (Mt != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < kCombWarps; ++w) {
+      const float r = exp2f(sh_m[w] - Mt);  // 0 for a warp without slots
+      Lt = fmaf(r, sh_l[w], Lt);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[k] = fmaf(r, sh_o[w][lane + 32 * k], o[k]);
+    }
+  }
+  const float inv = (Lt > 0.0f) ? 1.0f / (Lt * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
+  wht128_warp(o, lane);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const uint32_t sw = __ldg(a.sign_bits + h * 4 + k);
-    const float o = apply_sign(v[k] * inv, sw, lane);
-    store_elem(a.out, row * kD + lane + 32 * k, o, a.out_dtype);
+    const float y = apply_sign(o[k] * inv, sw, lane);
+    store_elem(a.out, row * kD + lane + 32 * k, y, a.out_dtype);
   }
 }
 
@@ -662,8 +713,8 @@ int launch_split(const DecodeArgs &a, cudaStream_t st) {
   const int nw = warps_for(G, a.ck, a.cv);
   if (static_cast<int64_t>(a.grid) * nw != a.total_warps) return static_cast<int>(cudaErrorInvalidValue);
   const SplitSmem L = split_smem_layout(G, a.ck, a.cv, nw);
-  auto kern = decode_split_kernel<G, kTwoK, kTwoV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  constexpr auto kern = decode_split_kernel<G, kTwoK, kTwoV>;
+  const cudaError_t e = ensure_max_dynamic_smem<kern>(static_cast<int>(L.total));
   if (e != cudaSuccess) return static_cast<int>(e);
   kern<<<a.grid, nw * 32, L.total, st>>>(a);
   return static_cast<int>(cudaGetLastError());
@@ -701,7 +752,8 @@ int launch_decode_attention(const DecodeArgs &a, void *stream) {
   }
   if (e) return e;
   const int64_t rows = static_cast<int64_t>(a.B) * a.Hq;
-  combine_kernel<<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(a);
+  if (rows > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidValue);
+  combine_kernel<<<static_cast<unsigned>(rows), kCombWarps * 32, 0, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 

@@ -5,6 +5,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "dq_internal.h"
@@ -67,6 +68,28 @@ __device__ __forceinline__ void wht128_warp(float (&v)[4], int lane) {
     v[1] = __fadd_rn(a1, a3);
     v[3] = __fsub_rn(a1, a3);
   }
+}
+
+// Raises kernel Kern's dynamic shared-memory limit to at least `bytes` on
+// the current device. The attribute call is made only when a larger size is
+// first needed on a device, so a launch sequence that repeats (a serving
+// loop, one call per layer) pays the host-side attribute call once.
+template <auto Kern>
+cudaError_t ensure_max_dynamic_smem(int bytes) {
+  constexpr int kDevs = 64;
+  static std::atomic<int> set_to[kDevs];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kDevs;
+  if (cached && set_to[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) {
+    int cur = set_to[dev].load(std::memory_order_relaxed);
+    while (cur < bytes && !set_to[dev].compare_exchange_weak(cur, bytes, std::memory_order_release)) {
+    }
+  }
+  return e;
 }
 
 // Sign of coordinate lane + 32 k for a KV head: bit `lane` of sign word k.

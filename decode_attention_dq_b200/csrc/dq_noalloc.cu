@@ -15,7 +15,13 @@
 // the library holds it (kScratchBytes) until the process exits, and every call
 // on a device shares it. Host code cannot use the array's name as a device
 // address (on the host it is only a stand-in symbol), so the device address
-// is looked up once per device with cudaGetSymbolAddress and cached.
+// is looked up with cudaGetSymbolAddress, with the device current, and cached
+// per device together with the id of the CUDA context it belongs to. A new
+// context on that device (after cudaDeviceReset, or once the primary context
+// has been released and created again) loads the module afresh, possibly at
+// another address; the id then differs and the address is looked up again,
+// so a stale address is never handed to a kernel.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -29,24 +35,71 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-std::mutex g_scratch_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void *ptr;
+};
 
-// Device address of g_scratch on the current device; looked up on the first
-// call per device (with that device current) and cached.
+std::mutex g_scratch_mutex;
+ScratchEntry g_scratch_entry[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Driver entry points for the current context and its id, resolved once
+// through the runtime (the library does not link the driver directly).
+bool driver_fns(CtxGetCurrentFn *get_current, CtxGetIdFn *get_id) {
+  static CtxGetCurrentFn s_current = nullptr;
+  static CtxGetIdFn s_id = nullptr;
+  static bool s_tried = false;
+  if (!s_tried) {
+    s_tried = true;
+    void *f0 = nullptr, *f1 = nullptr;
+    cudaDriverEntryPointQueryResult q0 = cudaDriverEntryPointSymbolNotFound, q1 = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f0, 12000, cudaEnableDefault, &q0) == cudaSuccess &&
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &f1, 12000, cudaEnableDefault, &q1) == cudaSuccess &&
+        q0 == cudaDriverEntryPointSuccess && q1 == cudaDriverEntryPointSuccess) {
+      s_current = reinterpret_cast<CtxGetCurrentFn>(f0);
+      s_id = reinterpret_cast<CtxGetIdFn>(f1);
+    }
+  }
+  *get_current = s_current;
+  *get_id = s_id;
+  return s_current && s_id;
+}
+
+// Id of the context current on this thread; false if there is none yet.
+bool current_ctx_id(CtxGetCurrentFn get_current, CtxGetIdFn get_id, unsigned long long *id) {
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || !c) return false;
+  return get_id(c, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_scratch in the current context of the current device:
+// looked up on the first call per device (with that device current) and
+// again whenever the device's context has changed since.
 int scratch_address(void **out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return DQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DQ_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scratch);
-    if (e != cudaSuccess || !p) return DQ_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+  if (!driver_fns(&get_current, &get_id)) return DQ_ERR_CUDA;
+  ScratchEntry &ent = g_scratch_entry[dev];
+  unsigned long long id = 0;
+  if (ent.ptr && current_ctx_id(get_current, get_id, &id) && id == ent.ctx_id) {
+    *out = ent.ptr;
+    return DQ_OK;
   }
-  *out = g_scratch_ptr[dev];
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_scratch);  // also makes the primary context current if needed
+  if (e != cudaSuccess || !p) return DQ_ERR_CUDA;
+  if (!current_ctx_id(get_current, get_id, &id)) return DQ_ERR_CUDA;
+  ent.ptr = p;
+  ent.ctx_id = id;
+  *out = p;
   return DQ_OK;
 }
 

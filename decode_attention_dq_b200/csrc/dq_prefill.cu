@@ -864,8 +864,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 template <bool kTwoK, bool kTwoV>
 int launch_tiles_t(const PrefillArgs &a, cudaStream_t st) {
   const TilesSmem L = tiles_smem_layout(a.ck, a.cv);
-  auto kern = prefill_tiles_kernel<kTwoK, kTwoV>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  constexpr auto kern = prefill_tiles_kernel<kTwoK, kTwoV>;
+  const cudaError_t e = ensure_max_dynamic_smem<kern>(static_cast<int>(L.total));
   if (e != cudaSuccess) return static_cast<int>(e);
   kern<<<a.tile_grid, kTileWarps * 32, L.total, st>>>(a);
   return static_cast<int>(cudaGetLastError());
@@ -906,8 +906,7 @@ int launch_prefill_attention(const PrefillArgs &a, void *stream) {
   else e = launch_tiles_t<false, false>(a, st);
   if (e) return e;
   const AttnSmem L = attn_smem_layout(a.nslots);
-  cudaError_t ce =
-      cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+  const cudaError_t ce = ensure_max_dynamic_smem<prefill_kernel>(static_cast<int>(L.total));
   if (ce != cudaSuccess) return static_cast<int>(ce);
   prefill_kernel<<<static_cast<unsigned>(grid), kAttnThreads, L.total, st>>>(a);
   return static_cast<int>(cudaGetLastError());

@@ -295,7 +295,10 @@ int dq_decode_attention_paged(const dq_tables *t, const void *q, int q_dtype,
  *   are rejected with DQ_ERR_WORKSPACE before anything is enqueued.
  *   Set-up: the first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, no allocation) with that device current; make that
- *   first call before any stream capture.
+ *   first call before any stream capture. The address is kept per device with
+ *   the id of its CUDA context; a call in a new context on that device (after
+ *   cudaDeviceReset, for example) looks the address up again, so that first
+ *   call after the reset should also come before any stream capture.
  *   Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents; nothing in it needs to start at zero. Calls whose work
  *   overlaps on the GPU (for example on two streams) race on the array and

@@ -191,6 +191,10 @@ ATTN_CASES = [
     # more token groups than warps in the grid: warp ranges cross (b, h) edges
     ("qwen3_8b_b16_t8k", 8, 8, 4, 3001, [3000, 33, 2900, 0, 2600, 2500, 40, 3001]),
     ("long_b4_t64k", 2, 8, 4, 20000, [20000, 12345]),
+    # far fewer token groups than warps: most warps are empty and the combine
+    # walks the few segments of each (b, h)
+    ("qwen3_8b_b16_t8k", 1, 1, 4, 64, [64]),
+    ("qwen3_8b_b16_t8k", 1, 8, 4, 64, [64]),
 ]
 
 
