@@ -57,13 +57,13 @@ ENCODE_OPS_PER_VECTOR = 2560
 LAUNCHES_PER_STEP = 4
 # DRAM traffic of decode_split_kernel from one ncu capture (dram__bytes_read
 # + dram__bytes_write) of the 32-sequence, 8192-token workload with 36-byte
-# containers: 151.37 MB + 3.62 MB per launch over 32*8*8192 token-heads. It
+# containers: 151.37 MB + 3.99 MB per launch over 32*8*8192 token-heads. It
 # scales with the token-heads a launch processes (reads are the containers,
 # writes the partial states). It belongs to one version of the kernel source:
 # for any other, or other container sizes, traffic is reported as null.
 DECODE_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_decode.cu",
-                  "sha256_16": "36f00627cfa3f944", "ck": 36, "cv": 36,
-                  "bytes_per_token_head": (151.368192e6 + 3.621888e6) / (32 * 8 * 8192)}
+                  "sha256_16": "c5c84b886abca60c", "ck": 36, "cv": 36,
+                  "bytes_per_token_head": (151.366912e6 + 3.988736e6) / (32 * 8 * 8192)}
 
 
 def decode_traffic(token_heads, ck, cv):
@@ -421,6 +421,22 @@ def run_dq(args):
     e2e_ms = max_over_ranks([f0.elapsed_time(f1)], dist, dev)[0]
     e2e_value = whole_job_rate(kv_tokens_step, ws, e2e_ms / args.steps)
 
+    # ---- small-batch decode latency: the first 1 and 8 sequences of the same
+    # cache, one dq_decode_attention call at a time with L2 flushed before
+    # each (the regime in which the pages find D-Quant slower than BF16) ----
+    small_batch = small_batch_latency(dq, tab, w, kc, vc, dev_q[0], seq, T, stream, dist, dev) \
+        if (L == 1 and page_table is None) else None
+
+    # ---- the long-context and low-budget workloads (device-timed, inputs
+    # larger than L2); the serving caches stay resident meanwhile ----
+    peaks, _src = measured_peaks()
+    alu_peak_all = (torch.cuda.get_device_properties(dev).multi_processor_count * 128
+                    * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12)
+    long_context = budget_sweep = None
+    if args.extra and L == 1 and page_table is None:
+        long_context = long_context_report(dq, args, dev, stream, dist, alu_peak_all, peaks)
+        budget_sweep = budget_sweep_report(dq, args, dev, stream, dist, alu_peak_all, peaks)
+
     # ---- chunked prefill over the same cache: the last n_q positions as a
     # chunk of queries (dq_prefill_attention), device-resident inputs ----
     prefill = None
@@ -509,6 +525,9 @@ def run_dq(args):
                       "prefill_v_cont_pct": 100.0 * pstats["v_cont_drifted"] / token_heads,
                       "fallbacks": pstats["overflow_fallbacks"]},
             "integrity_errors": st["integrity_errors"],
+            "small_batch": small_batch,
+            "long_context": long_context,
+            "budget_sweep": budget_sweep,
             "prefill_s": prefill_s,
             "encode": encode_report(enc_ms, enc_vectors, w, ck, cv, alu_peak, peaks),
             "chunked_prefill": None if prefill is None else dict(
@@ -532,6 +551,156 @@ def run_dq(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def decode_ms(dq, tab, w, kc, vc, T, stream, reps=5):
+    """Median device time (ms) of dq_decode_attention over the whole cache
+    (inputs larger than L2), after two untimed calls."""
+    import torch
+
+    from decode_attention_dq_b200 import synth
+    q = torch.from_numpy(synth.q_block(w)).to(device=kc.device, dtype=w.torch_dtype)
+    seq = torch.full((w.B,), T, dtype=torch.int32, device=kc.device)
+    ws = torch.empty(dq.dq_decode_workspace_bytes(tab, w.B, w.Hq, w.Hkv, T), dtype=torch.uint8, device=kc.device)
+    out = torch.empty((w.B, w.Hq, 128), dtype=torch.float32, device=kc.device)
+    stats = dq.new_stats(kc.device)
+    for _ in range(2):
+        dq.dq_decode_attention(tab, q, kc, vc, seq, T, out, ws, stream=stream)
+    evs = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dq.dq_decode_attention(tab, q, kc, vc, seq, T, out, ws, stats=stats, stream=stream)
+        b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs), dq.stats_dict(stats)["integrity_errors"]
+
+
+def decode_report(ms, w, T, ck, cv, alu_peak, peaks):
+    G = w.Hq // w.Hkv
+    token_heads = w.B * T * w.Hkv
+    achieved = token_heads * ops_per_token_head(G) / (ms * 1e-3) / 1e12
+    gbs = token_heads * (ck + cv) / (ms * 1e-3) / 1e9
+    return {"decode_ms": ms, "kv_tokens_per_s": w.B * T / (ms * 1e-3), "hbm_gbs": gbs,
+            "hbm_frac": gbs / float(peaks.get("hbm_gbs", 6650.0)),
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "Tlaneop/s",
+                         "frac": achieved / alu_peak}}
+
+
+def long_context_report(dq, args, dev, stream, dist, alu_peak, peaks):
+    """The long-context workload (4 sequences x 8 KV heads x 32 query heads,
+    2.26 bit/value): the full 65536-token prefill append of all 4 sequences
+    in one call (containers/s), then split-K decode attention over 65536 and
+    131072 tokens."""
+    import torch
+
+    from decode_attention_dq_b200 import synth
+    res = {"what": "4 sequences x 8 KV heads, 2.26 bit/value: one dq_append_kv of 65536 tokens per "
+                   "sequence (encode), and dq_decode_attention over 65536 and 131072 tokens"}
+    for name in ("long_b4_t64k", "long_b4_t128k"):
+        w = replica_workload(synth.WORKLOADS[name], int(os.environ.get("RANK", "0")))
+        tab = dq.dq_build_tables(n_kv_heads=w.Hkv, k_bits_per_value=w.k_bits, v_bits_per_value=w.v_bits)
+        ck, cv = tab.k.container_bytes, tab.v.container_bytes
+        kc = torch.zeros((w.B, w.Hkv, w.T, ck), dtype=torch.uint8, device=dev)
+        vc = torch.zeros((w.B, w.Hkv, w.T, cv), dtype=torch.uint8, device=dev)
+        timings = [] if w.T == 65536 else None
+        synth.prefill_cache(tab, w, kc, vc, w.T, seqs_per_call=w.B, threads=args.threads, timings=timings)
+        ms, bad = decode_ms(dq, tab, w, kc, vc, w.T, stream)
+        enc = None
+        if timings:
+            enc_ms = sum(a.elapsed_time(b) for a, b, _ in timings)
+            enc = max_over_ranks([enc_ms], dist, dev)[0]
+        ms = max_over_ranks([ms], dist, dev)[0]
+        r = dict(decode_report(ms, w, w.T, ck, cv, alu_peak, peaks), integrity_errors=bad)
+        if enc is not None:
+            n = sum(n for _, _, n in timings)
+            r["prefill_encode"] = {"ms": enc, "containers_per_s": 2 * n / (enc * 1e-3),
+                                   "tokens_per_sequence": w.T, "sequences": w.B}
+        res[name] = r
+        del kc, vc, tab
+    return res
+
+
+def budget_sweep_report(dq, args, dev, stream, dist, alu_peak, peaks):
+    """The Llama-3.1-8B-shaped workload (32 sequences x 8 KV heads x 32 query
+    heads x 32768 tokens) at 1.96, 2.26 and 3.0 bit/value: the same seeded
+    K/V encoded with each budget's tables (drift rate per stream), then
+    decode attention over the 32768 tokens."""
+    import torch
+
+    from decode_attention_dq_b200 import synth
+    base = replica_workload(synth.WORKLOADS["llama_b32_t32k_2p26"], int(os.environ.get("RANK", "0")))
+    budgets = (1.96, 2.26, 3.0)
+    tabs = [dq.dq_build_tables(n_kv_heads=base.Hkv, k_bits_per_value=b, v_bits_per_value=b) for b in budgets]
+    caches = [(torch.zeros((base.B, base.Hkv, base.T, t.k.container_bytes), dtype=torch.uint8, device=dev),
+               torch.zeros((base.B, base.Hkv, base.T, t.v.container_bytes), dtype=torch.uint8, device=dev))
+              for t in tabs]
+    stats = [dq.new_stats(dev) for _ in tabs]
+    # The same inputs for every budget: drawn once per batch of sequences.
+    for b0 in range(0, base.B, 8):
+        b1 = min(base.B, b0 + 8)
+        rows = [(b, h) for b in range(b0, b1) for h in range(base.Hkv)]
+        kt = torch.from_numpy(synth.kv_block(base, "k", rows, n=base.T, threads=args.threads)).to(
+            device=dev, dtype=base.torch_dtype).view(b1 - b0, base.Hkv, base.T, 128)
+        vt = torch.from_numpy(synth.kv_block(base, "v", rows, n=base.T, threads=args.threads)).to(
+            device=dev, dtype=base.torch_dtype).view(b1 - b0, base.Hkv, base.T, 128)
+        start = torch.zeros(b1 - b0, dtype=torch.int32, device=dev)
+        for t, (kc, vc), st in zip(tabs, caches, stats):
+            dq.dq_append_kv(t, kt, vt, start, kc[b0:b1], vc[b0:b1], stats=st)
+    torch.cuda.synchronize()
+    out = []
+    n_sym = base.B * base.Hkv * base.T * 128
+    n_cont = base.B * base.Hkv * base.T
+    for bits, t, (kc, vc), st in zip(budgets, tabs, caches, stats):
+        ms, bad = decode_ms(dq, t, base, kc, vc, base.T, stream)
+        ms = max_over_ranks([ms], dist, dev)[0]
+        sd = dq.stats_dict(st)
+        out.append(dict(decode_report(ms, base, base.T, t.k.container_bytes, t.v.container_bytes, alu_peak, peaks),
+                        bits_per_value=bits, k_container_bytes=t.k.container_bytes,
+                        v_container_bytes=t.v.container_bytes,
+                        k_drift_syms_pct=100.0 * sd["k_syms_drifted"] / n_sym,
+                        v_drift_syms_pct=100.0 * sd["v_syms_drifted"] / n_sym,
+                        k_drift_cont_pct=100.0 * sd["k_cont_drifted"] / n_cont,
+                        v_drift_cont_pct=100.0 * sd["v_cont_drifted"] / n_cont,
+                        fallbacks=sd["overflow_fallbacks"], integrity_errors=bad))
+    del caches
+    return {"what": "32 sequences x 8 KV heads x 32768 tokens, the same seeded K/V encoded at each budget; "
+                    "drift rates over the whole prefill, then dq_decode_attention over all tokens",
+            "budgets": out}
+
+
+def small_batch_latency(dq, tab, w, kc, vc, q, seq, T, stream, dist, dev, reps=20):
+    """Device time of one dq_decode_attention call (prefix, split and combine
+    kernels) over the first B sequences of the cache, B = 1 and 8, with L2
+    flushed (a 256 MB write) before every call; median over `reps` calls,
+    slowest rank."""
+    import torch
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+    for B in (1, 8):
+        if B > w.B:
+            continue
+        wsb = torch.empty(dq.dq_decode_workspace_bytes(tab, B, w.Hq, w.Hkv, T), dtype=torch.uint8, device=dev)
+        o = torch.empty((B, w.Hq, 128), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            dq.dq_decode_attention(tab, q[:B], kc[:B], vc[:B], seq[:B], T, o, wsb, stream=stream)
+        evs = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            dq.dq_decode_attention(tab, q[:B], kc[:B], vc[:B], seq[:B], T, o, wsb, stream=stream)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in evs) * 1e3
+        us = max_over_ranks([us], dist, dev)[0]
+        res["b%d" % B] = {"decode_us": us, "kv_tokens_per_s": B * T / (us * 1e-6),
+                          "sequences": B, "context": T}
+    res["what"] = ("one dq_decode_attention call over the first B sequences of the benchmark cache, "
+                   "L2 flushed before each call, median of %d" % reps)
+    return res
 
 
 def encode_report(enc_ms, enc_vectors, w, ck, cv, alu_peak, peaks):
@@ -578,11 +747,29 @@ def oracle_sample_step(w, tabs, rows, cache_rows):
         o.attention_fp64(tabs, qb, kfull, vfull, [kc.shape[0]], rows=[(0, h)])
 
 
+def host_cpu():
+    """Model string and usable core count of the host CPU."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    return model, ncores
+
+
 def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0.0), drift_mode=0):
     """The oracle, as it stands, on the host: a bounded sample of the step,
     once on one thread (BLAS limited to one thread too) and once on all host
     cores (a thread per (sequence, KV head) row; the oracle's C calls and
-    numpy's kernels release the GIL)."""
+    numpy's kernels release the GIL). Besides the step (append one token +
+    decode attention), the two halves of the path are timed on their own:
+    encode (containers/s over sampled rows' tokens) and fp64 decode
+    attention (KV tokens/s)."""
     from concurrent.futures import ThreadPoolExecutor
 
     import numpy as np
@@ -594,46 +781,91 @@ def cpu_baseline(w, tab_seed=0, seconds=15.0, max_rows=512, rate_offsets=(0.0, 0
     tabs = o.Tables(w.Hkv, k_container_bytes=o.container_bytes(w.k_bits),
                     v_container_bytes=o.container_bytes(w.v_bits), sign_seed=tab_seed,
                     k_rate_offset=rate_offsets[0], v_rate_offset=rate_offsets[1], drift_mode=drift_mode)
-    ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    model, ncores = host_cpu()
+    G = w.Hq // w.Hkv
     with threadpool_limits(limits=1):
-        # Containers for sampled rows, encoded by the oracle (setup, untimed).
+        # Sampled rows' inputs and their oracle containers (setup, untimed
+        # except for the encode measurement below, which re-encodes them).
         rng = np.random.default_rng(0)
         cand = [(int(b), int(h)) for b, h in zip(rng.integers(0, w.B, max_rows), rng.integers(0, w.Hkv, max_rows))]
 
-        def prepare(bh):
+        def inputs(bh):
             b, h = bh
-            K = synth.kv_row(w, "k", b, h)
-            V = synth.kv_row(w, "v", b, h)
-            kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, K, np.full(w.T, h, np.int32), tabs.drift_mode)
-            vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, V, np.full(w.T, h, np.int32), tabs.drift_mode)
-            return (bh, (kc, vc))
+            return synth.kv_row(w, "k", b, h), synth.kv_row(w, "v", b, h)
+
+        def encode(bh, kv):
+            h = bh[1]
+            kc, _, _, _ = o.encode_vectors(tabs.k, tabs.signs, kv[0], np.full(w.T, h, np.int32), tabs.drift_mode)
+            vc, _, _, _ = o.encode_vectors(tabs.v, tabs.signs, kv[1], np.full(w.T, h, np.int32), tabs.drift_mode)
+            return kc, vc
 
         prepared = []
         t_setup = time.time()
         with ThreadPoolExecutor(ncores) as ex:
             for i in range(0, len(cand), ncores):
-                prepared.extend(ex.map(prepare, cand[i:i + ncores]))
+                chunk = cand[i:i + ncores]
+                kvs = list(ex.map(inputs, chunk))
+                conts = list(ex.map(encode, chunk, kvs))
+                # The raw inputs (8 MB a row at 8K) are kept for the first 16
+                # rows only, for the encode measurement.
+                n0 = len(prepared)
+                prepared.extend((bh, cc, kv if n0 + i < 16 else None)
+                                for i, (bh, cc, kv) in enumerate(zip(chunk, conts, kvs)))
                 if time.time() - t_setup > seconds:
                     break
-        # One thread.
+        budget = seconds / 4
+        # Step (append one token + attention over the row), one thread.
         done = 0
         t0 = time.time()
-        for (bh, cc) in prepared:
+        for (bh, cc, _) in prepared:
             oracle_sample_step(w, tabs, [bh], [cc])
             done += 1
-            if time.time() - t0 > seconds / 2:
+            if time.time() - t0 > budget:
                 break
         dt = time.time() - t0
-        # All cores, over the same rows.
-        rows = prepared[:max(done, min(len(prepared), ncores))]
+        # Encode alone: the rows' T tokens of K and V, one thread.
+        enc_rows = 0
         t1 = time.time()
+        for (bh, _, kv) in prepared:
+            if kv is None:
+                break
+            encode(bh, kv)
+            enc_rows += 1
+            if time.time() - t1 > budget:
+                break
+        dt_enc = time.time() - t1
+        # Decode attention alone: G query heads over the row's T tokens, one thread.
+        dec_rows = 0
+        t2 = time.time()
+        for (bh, cc, _) in prepared:
+            b, h = bh
+            qb = np.zeros((1, w.Hq, 128))
+            qb[0, h * G:(h + 1) * G] = synth.q_rows(w, b)[h * G:(h + 1) * G]
+            kfull = np.zeros((1, w.Hkv) + cc[0].shape, np.uint8)
+            vfull = np.zeros((1, w.Hkv) + cc[1].shape, np.uint8)
+            kfull[0, h] = cc[0]
+            vfull[0, h] = cc[1]
+            o.attention_fp64(tabs, qb, kfull, vfull, [w.T], rows=[(0, h)])
+            dec_rows += 1
+            if time.time() - t2 > budget:
+                break
+        dt_dec = time.time() - t2
+        # All cores, the step over the same rows.
+        rows = prepared[:max(done, min(len(prepared), ncores))]
+        t3 = time.time()
         with ThreadPoolExecutor(ncores) as ex:
             list(ex.map(lambda p: oracle_sample_step(w, tabs, [p[0]], [p[1]]), rows))
-        dt_all = time.time() - t1
+        dt_all = time.time() - t3
     per_row = w.T / w.Hkv  # one KV token = one position across all KV heads
     return {"value": done * per_row / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_model": model, "nproc": ncores,
             "sample": "%d (sequence, KV head) rows of %s: append 1 token + fp64 decode attention over %d "
                       "tokens each, one thread, %.1f s" % (done, w.name, w.T, dt),
+            "encode": {"containers_per_s": enc_rows * 2 * w.T / dt_enc, "cores": 1,
+                       "sample": "%d rows x %d tokens, K and V, one thread, %.1f s" % (enc_rows, w.T, dt_enc)},
+            "decode": {"kv_tokens_per_s": dec_rows * per_row / dt_dec, "cores": 1,
+                       "sample": "%d rows: %d query heads over %d tokens, fp64, one thread, %.1f s"
+                                 % (dec_rows, G, w.T, dt_dec)},
             "all_cores": {"value": len(rows) * per_row / dt_all, "unit": UNIT, "cores": ncores,
                           "sample": "%d rows, one thread per row, %.1f s" % (len(rows), dt_all)}}
 
@@ -1020,6 +1252,8 @@ def main():
     ap.add_argument("--threads", type=int, default=max(4, min(32, os.cpu_count() or 8)))
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", dest="extra", action="store_false",
+                    help="skip the long-context and budget-sweep workloads")
     ap.add_argument("--paged", action="store_true", help="page pools and a shuffled page table")
     ap.add_argument("--layers", type=int, default=1, help="layers of the decode loop (one cache each)")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as a CUDA graph")

@@ -7,8 +7,8 @@ dq_decode_attention over the T tokens with the whole batch, as bench.py does.
 For a few sampled sequences the oracle encodes the same seeded K/V: their
 containers must be bit-identical and their attention rows (all query heads)
 within max-abs 2e-3 x RMS of the oracle's fp64 attention. The serving shape
-(128 x 8K), the long context (4 x 128K) and the low/high budgets of the
-32 x 32K sweep are covered.
+(128 x 8K), the Qwen3-8B-shaped decode step (16 x 8K), the long context
+(4 x 128K) and all three budgets of the 32 x 32K sweep are covered.
 """
 import numpy as np
 import pytest
@@ -23,8 +23,10 @@ pytestmark = pytest.mark.gpu
 
 FULL_CASES = [
     ("serve_b128_t8k", [0, 77, 127]),
+    ("qwen3_8b_b16_t8k", [3, 15]),
     ("long_b4_t128k", [2]),
     ("llama_b32_t32k_1p96", [5]),
+    ("llama_b32_t32k_2p26", [17]),
     ("llama_b32_t32k_3p0", [30]),
 ]
 
