@@ -27,20 +27,27 @@
 // one query token of the chunk with one of the G query heads of h (row r =
 // token r / G, head r % G). The CTAs of one (b, h) are launched together (the
 // longest causal ranges first) so that its tiles are read from L2. Warps:
-//   0-3  softmax: thread r owns row r = lane r of tensor memory. It rotates
-//        its query (q~ = H D q in fp32, times a power of two), splits it into
-//        fp16 hi + lo and stores both into tensor memory; per block j it reads
-//        its 32 scores, applies the key norms, the scale and the causal mask,
-//        runs the online softmax, rescales its row of O in tensor memory when
-//        the running maximum grows, and stores the weights w = p ||v|| as fp16
-//        hi + lo into tensor memory. At the end it applies 1 / (128 l kappa_V),
-//        the inverse rotation D H and writes the output row.
-//   4    owns the tensor memory; one lane issues the MMAs
-//          S_j = q~hi K_j^T + q~lo K_j^T        (M 128, N 32, K 128)
-//          O  += W_j,hi V_j + W_j,lo V_j         (M 128, N 128, K 32)
+//   0-15 softmax: the four warps w, w + 4, w + 8, w + 12 share rows
+//        32 (w % 4) .. + 31 (thread = row = lane of tensor memory); warp
+//        w + 4 q takes tokens 32 q .. 32 q + 31 of every block. The row's
+//        four threads rotate its query (q~ = H D q in fp32, times a power of
+//        two; stages h = 1 .. 16 on 32 coordinates each in registers, h = 32
+//        and 64 after an exchange through tensor memory), split it into fp16
+//        hi + lo and store both into tensor memory; per block j each reads
+//        its 32 scores, applies the key norms, the scale and the causal
+//        mask, and the four meet (shared memory, a named barrier per row
+//        group) on the row maximum; the online softmax rescales the row's O
+//        in tensor memory (32 columns per thread) when the running maximum
+//        grows, and each thread stores its tokens' weights w = p ||v|| as fp16
+//        hi + lo into tensor memory. At the end the four apply 1 / (128 l
+//        kappa_V), the inverse rotation D H (split as for q~) and write the
+//        output row.
+//   16   owns the tensor memory; one lane issues the MMAs
+//          S_j = q~hi K_j^T + q~lo K_j^T        (M 128, N 128, K 128)
+//          O  += W_j,hi V_j + W_j,lo V_j         (M 128, N 128, K 128)
 //        kind::f16 with fp32 accumulators, A from tensor memory, B (K tile
 //        K-major, V tile MN-major) from shared memory.
-//   5    one lane streams the slots into a ring in shared memory with bulk
+//   17   one lane streams the slots into a ring in shared memory with bulk
 //        copies counted on mbarriers.
 // Every wait is bounded; a CTA that gives up counts it in wait_timeouts,
 // skips the rest of its work and still frees its tensor memory after its MMAs
@@ -55,10 +62,11 @@ namespace {
 constexpr int kRows = 128;          // query rows per CTA (the MMA's M)
 constexpr int kGrp = 32;            // tokens per cache block (one decoder warp)
 constexpr int kBlk = 128;           // tokens per workspace slot / attention block (the score MMA's N)
-constexpr int kSoftWarps = 8;       // warps 0..7: warp w and w + 4 share rows 32 (w % 4) ..
-constexpr int kMmaWarp = 8;         // warp 8
-constexpr int kLoadWarp = 9;        // warp 9
-constexpr int kAttnThreads = 32 * 10;
+constexpr int kSoftWarps = 16;      // warps 0..15: warps w, w + 4, w + 8, w + 12 share rows 32 (w % 4) ..
+constexpr int kQuads = kSoftWarps / 4;  // softmax warps per row (each takes 32 tokens of a block)
+constexpr int kMmaWarp = 16;        // warp 16
+constexpr int kLoadWarp = 17;       // warp 17
+constexpr int kAttnThreads = 32 * 18;
 constexpr int kMaxSlots = 3;        // ring depth of prefill_kernel
 constexpr int kTileWarps = 20;      // warps per CTA of prefill_tiles_kernel
 constexpr uint32_t kTmemCols = 512;
@@ -107,10 +115,11 @@ __host__ __device__ inline TilesSmem tiles_smem_layout(int ck, int cv) {
 }
 
 // Shared memory of prefill_kernel: barriers, tensor-memory base and abort
-// flag, the row-max exchange [2 blocks][2 halves][128 rows] and the row-sum
-// exchange [2 halves][128 rows] of the softmax warp pairs, then the ring.
+// flag, the row-max, V-norm and go-on exchanges [2 blocks][4 quarters][128 rows],
+// the row-sum exchange [4 quarters][128 rows] of the softmax warps of a row,
+// then the ring.
 struct AttnSmem {
-  size_t bars, misc, pmax, lsum, pnv, ring, total;
+  size_t bars, misc, pmax, lsum, pnv, pgo, ring, total;
 };
 
 __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
@@ -118,9 +127,10 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
   s.bars = 0;
   s.misc = s.bars + kNumBars * 8;
   s.pmax = align_up(s.misc + 16, 16);
-  s.lsum = s.pmax + 2 * 2 * kRows * 4;
-  s.pnv = s.lsum + 2 * kRows * 4;
-  s.ring = align_up(s.pnv + 2 * 2 * kRows * 4, 128);
+  s.lsum = s.pmax + 2 * kQuads * kRows * 4;
+  s.pnv = s.lsum + kQuads * kRows * 4;
+  s.pgo = s.pnv + 2 * kQuads * kRows * 4;
+  s.ring = align_up(s.pgo + 2 * kQuads * kRows * 4, 128);
   s.total = s.ring + static_cast<size_t>(nslots) * kSlotBytes;
   return s;
 }
@@ -225,6 +235,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 8 consecutive fp32 columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&r)[4]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(r[0]),
@@ -453,7 +479,36 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   }
 }
 
-__device__ __forceinline__ void pair_sync(int id) { asm volatile("bar.sync %0, 64;\n" ::"r"(id) : "memory"); }
+// Barrier of the kQuads softmax warps that share a row group (ids 1..4).
+__device__ __forceinline__ void quad_sync(int id) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(32 * kQuads) : "memory");
+}
+
+// Stages h = 1, 2, 4, 8, 16 of the unnormalised Walsh-Hadamard transform on
+// 32 consecutive coordinates held in registers (butterfly (a, b) -> (a + b,
+// a - b), stages in that order).
+__device__ __forceinline__ void wht32_regs(float (&v)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if ((i & h) == 0) {
+        const float a0 = v[i], a1 = v[i + h];
+        v[i] = __fadd_rn(a0, a1);
+        v[i + h] = __fsub_rn(a0, a1);
+      }
+}
+
+// Stages h = 32 and 64 on the four coordinates i, i + 32, i + 64, i + 96
+// (z[m] is coordinate i + 32 m).
+__device__ __forceinline__ void wht_4(float (&z)[4]) {
+  const float a0 = __fadd_rn(z[0], z[1]), a1 = __fsub_rn(z[0], z[1]);
+  const float a2 = __fadd_rn(z[2], z[3]), a3 = __fsub_rn(z[2], z[3]);
+  z[0] = __fadd_rn(a0, a2);
+  z[2] = __fsub_rn(a0, a2);
+  z[1] = __fadd_rn(a1, a3);
+  z[3] = __fsub_rn(a1, a3);
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -463,9 +518,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + L.misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 4);
-  float *pmax = reinterpret_cast<float *>(smem + L.pmax);  // [2][2][128]
-  float *pnv = reinterpret_cast<float *>(smem + L.pnv);    // [2][2][128]: largest V norm of a row half
-  float *lsum = reinterpret_cast<float *>(smem + L.lsum);  // [2][128]
+  float *pmax = reinterpret_cast<float *>(smem + L.pmax);  // [2][kQuads][128]
+  float *pnv = reinterpret_cast<float *>(smem + L.pnv);    // [2][kQuads][128]: largest V norm of a row quarter
+  float *lsum = reinterpret_cast<float *>(smem + L.lsum);  // [kQuads][128]
+  int *pgo = reinterpret_cast<int *>(smem + L.pgo);        // [2][kQuads][128]: the warp's waits succeeded
   auto slot_base = [&](int d) { return smem + L.ring + static_cast<size_t>(d) * kSlotBytes; };
 
   // Work item: the query blocks of one (b, h) are consecutive, latest first.
@@ -500,7 +556,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       mbar_init(bars + kBarWFull + i, 32 * kSoftWarps);
       mbar_init(bars + kBarPvDone + i, 1);
     }
-    mbar_init(bars + kBarQFull, kRows);
+    mbar_init(bars + kBarQFull, kRows * kQuads);
     mbar_init(bars + kBarDrain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -512,35 +568,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   unsigned timeouts = 0, clamped = 0;
 
   if (warp < kSoftWarps) {
-    // ===== softmax: warps w and w + 4 own rows r = 32 (w % 4) + lane; warp w
-    // takes tokens 0..63 of each block, warp w + 4 tokens 64..127 =====
-    const int half = warp >> 2;
+    // ===== softmax: warps w, w + 4, w + 8, w + 12 own rows r = 32 (w % 4) +
+    // lane; warp w + 4 q takes tokens 32 q .. 32 q + 31 of each block =====
+    const int qt = warp >> 2;                    // token quarter of this warp
     const int r = (warp & 3) * 32 + lane;
     const uint32_t tl = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);  // this warp's lanes
     const int ti = i_lo + r / G, g = r % G;
     const bool in_chunk = ti <= i_hi;
     const int64_t pos = qs + ti;
     const bool row_ok = in_chunk && pos >= 0 && pos < a.T_cap;
-    if (half == 0 && in_chunk && !row_ok) ++clamped;
+    if (qt == 0 && in_chunk && !row_ok) ++clamped;
     const int hq = h * G + g;
     const int64_t qbase = ((static_cast<int64_t>(b) * a.n_q + (in_chunk ? ti : 0)) * a.Hq + hq) * kD;
-    // D1: q~ = H D q (unnormalised), times 2^e so that max |q~| is in [2^13, 2^14).
-    // Both warps of a pair need the row's scale; warp w alone stores q~.
+    const int quad_id = 1 + (warp & 3);
+    // D1: q~ = H D q (unnormalised), times 2^e so that max |q~| is in [2^13,
+    // 2^14). The four threads of a row share the work: thread qt rotates
+    // coordinates 32 qt .. 32 qt + 31 through stages h = 1 .. 16 in
+    // registers, passes them through tensor-memory columns (the score area,
+    // unused before the first MMA) and finishes stages h = 32, 64 on the
+    // coordinates i + 32 m, i in [8 qt, 8 qt + 8).
     float crow = 0.0f;
     {
-      float v[kD];
       uint32_t sw[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
+      float v[32];
 #pragma unroll
-      for (int c = 0; c < kD; ++c) {
-        const float x = in_chunk ? load_elem(a.q, qbase + c, a.q_dtype) : 0.0f;
-        v[c] = ((sw[c >> 5] >> (c & 31)) & 1u) ? -x : x;
+      for (int c = 0; c < 32; ++c) {
+        const float x = in_chunk ? load_elem(a.q, qbase + 32 * qt + c, a.q_dtype) : 0.0f;
+        v[c] = ((sw[qt] >> c) & 1u) ? -x : x;
       }
-      wht128_regs(v);
+      wht32_regs(v);
+      {
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 16) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(v[c + e]);
+          tmem_st16(tl + kColS + 32 * qt + c, w);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      quad_sync(quad_id);
+      tc_fence_after();
+      float z[4][8];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) tmem_ld8(tl + kColS + 32 * m + 8 * qt, z[m]);
       float amax = 0.0f;
 #pragma unroll
-      for (int c = 0; c < kD; ++c) amax = fmaxf(amax, fabsf(v[c]));
+      for (int i = 0; i < 8; ++i) {
+        float zz[4] = {z[0][i], z[1][i], z[2][i], z[3][i]};
+        wht_4(zz);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          z[m][i] = zz[m];
+          amax = fmaxf(amax, fabsf(zz[m]));
+        }
+      }
+      pmax[qt * kRows + r] = amax;
+      quad_sync(quad_id);
+#pragma unroll
+      for (int q2 = 0; q2 < kQuads; ++q2) amax = fmaxf(amax, pmax[q2 * kRows + r]);
       float sc = 1.0f;
       if (amax > 0.0f && amax < INFINITY) {
         int ex;
@@ -549,91 +638,92 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       }
       // logit (log2 units) = S * ||k|| * crow, with S = sum (q~ sc)(kappa_K y)
       crow = row_ok ? a.sm_scale * kLog2e / (static_cast<float>(kD) * sc * a.tabs->k.score_scale) : 0.0f;
-      if (half == 0) {
+      // Coordinates 32 m + 8 qt + 2 p, + 1 are packed fp16 column 16 m + 4 qt + p.
 #pragma unroll
-        for (int c16 = 0; c16 < kD; c16 += 16) {
-          uint32_t hi[8], lo[8];
+      for (int m = 0; m < 4; ++m) {
+        uint32_t hi[4], lo[4];
 #pragma unroll
-          for (int p = 0; p < 8; ++p) split_pair(v[c16 + 2 * p] * sc, v[c16 + 2 * p + 1] * sc, hi[p], lo[p]);
-          tmem_st8(tl + kColQh + c16 / 2, hi);
-          tmem_st8(tl + kColQl + c16 / 2, lo);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bars + kBarQFull);
+        for (int p2 = 0; p2 < 4; ++p2) split_pair(z[m][2 * p2] * sc, z[m][2 * p2 + 1] * sc, hi[p2], lo[p2]);
+        tmem_st4(tl + kColQh + 16 * m + 4 * qt, hi);
+        tmem_st4(tl + kColQl + 16 * m + 4 * qt, lo);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bars + kBarQFull);
+      quad_sync(quad_id);  // pmax is reused below; the score columns are the MMA's from here on
     }
 
     float m_run = -INFINITY, l_run = 0.0f;
     bool alive = true;
-    const int pair_id = 1 + (warp & 3);
     for (int64_t j = 0; j < nB; ++j) {
       const int sb = static_cast<int>(j & 1);
       const int rb = static_cast<int>(j % ns);
       bool ok = alive && mbar_wait(bars + kBarSFull + sb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) &&
                 mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag);
       ok = __all_sync(kFull, ok);
-      // The two warps of a pair leave the loop together (they meet at the
-      // pair barriers below): agree on going on, through shared memory.
-      pmax[(sb * 2 + half) * kRows + r] = ok ? 0.0f : 1.0f;
-      pair_sync(pair_id);
-      const bool go = ok && pmax[(sb * 2 + (half ^ 1)) * kRows + r] == 0.0f;
-      pair_sync(pair_id);
+      const uint32_t scol = tl + kColS + 128 * sb + 32 * qt;  // this warp's 32 score columns
+      const float *nv = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + kBlk + 32 * qt;
+      float u[32];
+      float mu0 = -INFINITY, mnv = 0.0f;
+      if (ok) {
+        tc_fence_after();
+        tmem_ld32(scol, u);
+        const float *nk = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + 32 * qt;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4) {
+          const float4 n4 = *reinterpret_cast<const float4 *>(nk + t);
+          u[t] *= n4.x;
+          u[t + 1] *= n4.y;
+          u[t + 2] *= n4.z;
+          u[t + 3] *= n4.w;
+        }
+        // u = S ||k|| (the logit divided by crow > 0); tokens past this row's
+        // position are masked, which only happens on the causal diagonal.
+        const int64_t rel = pos - j * kBlk - 32 * qt;
+        const int lim = (!row_ok || rel < 0) ? -1 : (rel > 31 ? 31 : static_cast<int>(rel));
+        if (!__all_sync(kFull, lim >= 31)) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
+        }
+        float mu[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          mu[t] = fmaxf(fmaxf(fmaxf(u[t], u[t + 4]), fmaxf(u[t + 8], u[t + 12])),
+                        fmaxf(fmaxf(u[t + 16], u[t + 20]), fmaxf(u[t + 24], u[t + 28])));
+        mu0 = fmaxf(fmaxf(mu[0], mu[1]), fmaxf(mu[2], mu[3]));
+        // Largest V norm of this quarter's tokens (bounds the weights below).
+#pragma unroll
+        for (int t = 0; t < 32; t += 4) {
+          const float4 n4 = *reinterpret_cast<const float4 *>(nv + t);
+          mnv = fmaxf(mnv, fmaxf(fmaxf(n4.x, n4.y), fmaxf(n4.z, n4.w)));
+        }
+      }
+      // One exchange per block among the four warps of the row: the row
+      // maximum, the largest V norm, and whether each warp could go on (its
+      // waits succeeded). The four leave the loop together when one cannot.
+      pmax[(sb * kQuads + qt) * kRows + r] = mu0;
+      pnv[(sb * kQuads + qt) * kRows + r] = mnv;
+      pgo[(sb * kQuads + qt) * kRows + r] = ok ? 1 : 0;
+      quad_sync(quad_id);
+      bool go = true;
+      float mrow = -INFINITY, vmax = 0.0f;
+#pragma unroll
+      for (int q2 = 0; q2 < kQuads; ++q2) {
+        go = go && pgo[(sb * kQuads + q2) * kRows + r] != 0;
+        mrow = fmaxf(mrow, pmax[(sb * kQuads + q2) * kRows + r]);
+        vmax = fmaxf(vmax, pnv[(sb * kQuads + q2) * kRows + r]);
+      }
       if (!go) {
         if (alive) ++timeouts;
         alive = false;
         break;
       }
-      tc_fence_after();
-      const uint32_t scol = tl + kColS + 128 * sb + 64 * half;  // this warp's 64 score columns
-      float u[64];
-      {
-        float s0[32], s1[32];
-        tmem_ld32(scol, s0);
-        tmem_ld32(scol + 32, s1);
-        const float *nk = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + 64 * half;
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          u[t] = s0[t] * nk[t];
-          u[32 + t] = s1[t] * nk[32 + t];
-        }
-      }
-      // u = S ||k|| (the logit divided by crow > 0); tokens past this row's
-      // position are masked, which only happens on the causal diagonal.
-      const int64_t rel = pos - j * kBlk - 64 * half;
-      const int lim = (!row_ok || rel < 0) ? -1 : (rel > 63 ? 63 : static_cast<int>(rel));
-      if (!__all_sync(kFull, lim >= 63)) {
-#pragma unroll
-        for (int t = 0; t < 64; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
-      }
-      float mu[32];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) mu[t] = fmaxf(u[t], u[t + 32]);
-#pragma unroll
-      for (int w2 = 16; w2 >= 1; w2 >>= 1)
-#pragma unroll
-        for (int t = 0; t < w2; ++t) mu[t] = fmaxf(mu[t], mu[t + w2]);
-      // Largest V norm of this half's tokens (bounds the weights below).
-      const float *nv = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + kBlk + 64 * half;
-      float mnv = 0.0f;
-#pragma unroll
-      for (int t = 0; t < 64; t += 4) {
-        const float4 n4 = *reinterpret_cast<const float4 *>(nv + t);
-        mnv = fmaxf(mnv, fmaxf(fmaxf(n4.x, n4.y), fmaxf(n4.z, n4.w)));
-      }
-      // Row maximum and largest V norm over both halves: exchange through
-      // shared memory.
-      pmax[(sb * 2 + half) * kRows + r] = mu[0];
-      pnv[(sb * 2 + half) * kRows + r] = mnv;
-      pair_sync(pair_id);
-      const float mrow = fmaxf(mu[0], pmax[(sb * 2 + (half ^ 1)) * kRows + r]);
-      const float vmax = fmaxf(mnv, pnv[(sb * 2 + (half ^ 1)) * kRows + r]);
       const float mcand = mrow == -INFINITY ? m_run : fmaxf(m_run, mrow * crow);
       // Lazy rescaling: the running maximum stays while the block's is at most
       // kLazyLog2 above it and the weights p ||v|| <= 2^(mcand - m_run) vmax
       // stay within half the fp16 range; O, l and the weights all use the
-      // same maximum, so the result is the same. Both halves of a row decide
-      // alike (same inputs).
+      // same maximum, so the result is the same. The four quarters of a row
+      // decide alike (same inputs).
       const float mx = (m_run != -INFINITY && mcand - m_run <= kLazyLog2 && ex2(mcand - m_run) * vmax <= 32768.0f)
                            ? m_run
                            : mcand;
@@ -651,28 +741,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       if (ok) {
         tc_fence_after();
         if (resc) {
-#pragma unroll 1
-          for (int c = 0; c < 64; c += 32) {
-            float o[32];
-            const uint32_t oc = tl + kColO + 64 * half + c;
-            tmem_ld32(oc, o);
-            uint32_t w0[16], w1[16];
+          // This warp rescales O's coordinate columns 32 qt .. 32 qt + 31.
+          float o[32];
+          const uint32_t oc = tl + kColO + 32 * qt;
+          tmem_ld32(oc, o);
+          uint32_t w0[16], w1[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              w0[e] = __float_as_uint(o[e] * alpha);
-              w1[e] = __float_as_uint(o[16 + e] * alpha);
-            }
-            tmem_st16(oc, w0);
-            tmem_st16(oc + 16, w1);
+          for (int e = 0; e < 16; ++e) {
+            w0[e] = __float_as_uint(o[e] * alpha);
+            w1[e] = __float_as_uint(o[16 + e] * alpha);
           }
+          tmem_st16(oc, w0);
+          tmem_st16(oc + 16, w1);
         }
         // W in place of this warp's own score columns (the scores were read
         // above), 16 tokens at a time: p = 2^(logit - mx), w = p ||v|| as fp16
-        // hi (columns 0..31) and lo (32..63); norms of tokens past the last
+        // hi (columns 0..15) and lo (16..31); norms of tokens past the last
         // attended position are 0, so masked tokens give exactly 0.
         float ps[2] = {0.0f, 0.0f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t wh[8], wl[8];
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
@@ -686,63 +774,91 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
             split_pair(p0 * nv[t], p1 * nv[t + 1], wh[p], wl[p]);
           }
           tmem_st8(scol + 8 * c, wh);
-          tmem_st8(scol + 32 + 8 * c, wl);
+          tmem_st8(scol + 16 + 8 * c, wl);
         }
         psum = ps[0] + ps[1];
         tmem_wait_st();
       } else {
         ++timeouts;
-        alive = false;  // both warps stop at the next agreement
+        alive = false;  // the whole row stops at the next agreement
       }
       if (mx != -INFINITY) m_run = mx;
       l_run = l_run * alpha + psum;
       tc_fence_before();
       mbar_arrive(bars + kBarWFull + sb);  // always, so the MMA warp's count completes
     }
-    // D7: o = D H o_rot / 128 with o_rot = O / (l kappa_V); l sums both halves.
-    lsum[half * kRows + r] = l_run;
-    pair_sync(pair_id);
-    const float l_all = l_run + lsum[(half ^ 1) * kRows + r];
-    if (half == 0) {
-      bool have_o = alive && nB > 0;
-      if (have_o) {
-        const int64_t jl = nB - 1;
-        const bool ok =
-            mbar_wait(bars + kBarPvDone + (jl & 1), static_cast<uint32_t>((jl >> 1) & 1), abort_flag);
-        if (!__all_sync(kFull, ok)) {
-          ++timeouts;
-          have_o = false;
-        }
+    // D7: o = D H o_rot / 128 with o_rot = O / (l kappa_V); l sums the four
+    // quarters. Thread qt takes O's coordinates 32 qt .. 32 qt + 31 through
+    // stages h = 1 .. 16, passes them through the (now idle) score columns
+    // and finishes stages h = 32, 64 on coordinates i + 32 m, i in [8 qt,
+    // 8 qt + 8).
+    lsum[qt * kRows + r] = l_run;
+    quad_sync(quad_id);
+    float l_all = 0.0f;
+#pragma unroll
+    for (int q2 = 0; q2 < kQuads; ++q2) l_all += lsum[q2 * kRows + r];
+    bool have_o = alive && nB > 0;
+    if (have_o) {
+      const int64_t jl = nB - 1;
+      const bool okw = mbar_wait(bars + kBarPvDone + (jl & 1), static_cast<uint32_t>((jl >> 1) & 1), abort_flag);
+      if (!__all_sync(kFull, okw)) {
+        ++timeouts;
+        have_o = false;
       }
-      float v[kD];
-      if (have_o) {
-        tc_fence_after();
+    }
+    // The row's four threads must agree (they exchange columns below).
+    pmax[qt * kRows + r] = have_o ? 0.0f : 1.0f;
+    quad_sync(quad_id);
 #pragma unroll
-        for (int c = 0; c < kD; c += 32) {
-          float o[32];
-          tmem_ld32(tl + kColO + c, o);
+    for (int q2 = 0; q2 < kQuads; ++q2) have_o = have_o && pmax[q2 * kRows + r] == 0.0f;
+    const float inv =
+        (have_o && row_ok && l_all > 0.0f) ? 1.0f / (l_all * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
+    // have_o is the same for the four warps of the row group (their
+    // agreement above), so they meet at the barrier below together. Without
+    // O (no block, or a wait that gave up) the output is zero and tensor
+    // memory is left alone.
+    float z[4][8];
+    if (have_o) {
+      float v[32];
+      tc_fence_after();
+      tmem_ld32(tl + kColO + 32 * qt, v);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[c + e] = o[e];
-        }
-      } else {
+      for (int c = 0; c < 32; ++c) v[c] *= inv;
+      wht32_regs(v);
+      uint32_t w[16];
 #pragma unroll
-        for (int c = 0; c < kD; ++c) v[c] = 0.0f;
+      for (int c = 0; c < 32; c += 16) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(v[c + e]);
+        tmem_st16(tl + kColS + 32 * qt + c, w);
       }
-      const float inv =
-          (have_o && row_ok && l_all > 0.0f) ? 1.0f / (l_all * static_cast<float>(kD) * a.tabs->v.tile_scale) : 0.0f;
+      tmem_wait_st();
+      tc_fence_before();
+      quad_sync(quad_id);
+      tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < kD; ++c) v[c] *= inv;
-      wht128_regs(v);
-      if (in_chunk) {
-        uint32_t sw[4];
+      for (int m = 0; m < 4; ++m) tmem_ld8(tl + kColS + 32 * m + 8 * qt, z[m]);
+      uint32_t sw[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
+      for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
 #pragma unroll
-        for (int c = 0; c < kD; ++c) {
-          const float o = ((sw[c >> 5] >> (c & 31)) & 1u) ? -v[c] : v[c];
-          store_elem(a.out, qbase + c, o, a.out_dtype);
-        }
+      for (int i = 0; i < 8; ++i) {
+        float zz[4] = {z[0][i], z[1][i], z[2][i], z[3][i]};
+        wht_4(zz);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) z[m][i] = ((sw[m] >> (8 * qt + i)) & 1u) ? -zz[m] : zz[m];
       }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[m][i] = 0.0f;
+    }
+    if (in_chunk) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) store_elem(a.out, qbase + 32 * m + 8 * qt + i, z[m][i], a.out_dtype);
     }
   } else if (warp == kMmaWarp) {
     // ===== MMA issue (one lane) =====
@@ -763,9 +879,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
         for (int ks = 0; ks < kBlk / 16; ++ks) {
           const uint64_t bd = smem_desc(vt + ks * 256, 128, kChunkStride);
-          const uint32_t wc = wb + (ks < 4 ? 0u : 64u) + (ks & 3) * 8;
+          // Tokens 16 ks .. 16 ks + 15 are in quarter ks / 2: fp16 hi pairs at
+          // its columns 8 (ks % 2) .., lo pairs 16 columns further.
+          const uint32_t wc = wb + 32 * static_cast<uint32_t>(ks >> 1) + (ks & 1) * 8;
           mma_ts(tbase + kColO, wc, bd, idO, (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_ts(tbase + kColO, wc + 32, bd, idO, 1u);
+          mma_ts(tbase + kColO, wc + 16, bd, idO, 1u);
         }
         tc_commit(bars + kBarPvDone + (jj & 1));
         tc_commit(bars + kBarEmpty + static_cast<int>(jj % ns));
