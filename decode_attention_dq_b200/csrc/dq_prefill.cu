@@ -42,13 +42,19 @@
 //        hi + lo into tensor memory. At the end the four apply 1 / (128 l
 //        kappa_V), the inverse rotation D H (split as for q~) and write the
 //        output row.
-//   16   owns the tensor memory; one lane issues the MMAs
+//   16   owns the tensor memory and issues the score MMAs
 //          S_j = q~hi K_j^T + q~lo K_j^T        (M 128, N 128, K 128)
+//   17   issues the P.V MMAs
 //          O  += W_j,hi V_j + W_j,lo V_j         (M 128, N 128, K 128)
 //        kind::f16 with fp32 accumulators, A from tensor memory, B (K tile
-//        K-major, V tile MN-major) from shared memory.
-//   17   one lane streams the slots into a ring in shared memory with bulk
+//        K-major, V tile MN-major) from shared memory. Two issuing warps on
+//        two schedulers: each shares its scheduler with four softmax warps,
+//        and one warp issuing all 32 MMAs of a block fell behind the tensor
+//        core. The barriers order the two streams.
+//   18   one lane streams the slots into a ring in shared memory with bulk
 //        copies counted on mbarriers.
+// The softmax arithmetic runs in packed fp32x2 operations (two tokens per
+// instruction) and three-input maxima.
 // Every wait is bounded; a CTA that gives up counts it in wait_timeouts,
 // skips the rest of its work and still frees its tensor memory after its MMAs
 // and copies have drained.
@@ -64,9 +70,10 @@ constexpr int kGrp = 32;            // tokens per cache block (one decoder warp)
 constexpr int kBlk = 128;           // tokens per workspace slot / attention block (the score MMA's N)
 constexpr int kSoftWarps = 16;      // warps 0..15: warps w, w + 4, w + 8, w + 12 share rows 32 (w % 4) ..
 constexpr int kQuads = kSoftWarps / 4;  // softmax warps per row (each takes 32 tokens of a block)
-constexpr int kMmaWarp = 16;        // warp 16
-constexpr int kLoadWarp = 17;       // warp 17
-constexpr int kAttnThreads = 32 * 18;
+constexpr int kMmaWarp = 16;        // warp 16: score MMAs; allocates tensor memory
+constexpr int kPvWarp = 17;         // warp 17: P.V MMAs
+constexpr int kLoadWarp = 18;       // warp 18: slot loader
+constexpr int kAttnThreads = 32 * 19;
 constexpr int kMaxSlots = 3;        // ring depth of prefill_kernel
 constexpr int kTileWarps = 20;      // warps per CTA of prefill_tiles_kernel
 constexpr uint32_t kTmemCols = 512;
@@ -85,7 +92,7 @@ constexpr float kLazyLog2 = 8.0f;      // lazy rescaling: largest growth (log2) 
 // Barrier slots of prefill_kernel.
 constexpr int kBarFull = 0, kBarEmpty = kMaxSlots, kBarSFull = 2 * kMaxSlots, kBarWFull = kBarSFull + 2,
               kBarPvDone = kBarSFull + 4, kBarQFull = kBarSFull + 6, kBarDrain = kBarSFull + 7,
-              kNumBars = kBarSFull + 8;
+              kBarDrainPv = kBarSFull + 8, kNumBars = kBarSFull + 9;
 static_assert(kSlotBytes % 16 == 0, "bulk copies move multiples of 16 bytes");
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -193,17 +200,25 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(smem_u32(bar))
-               : "memory");
-}
 // d (+)= a b^T: A (M 128 x K 16 fp16) from tensor memory, B from a shared
-// memory descriptor, fp32 accumulators in tensor memory.
+// memory descriptor, fp32 accumulators in tensor memory. Called by a whole
+// converged warp: every lane computes the operands and one elected lane (the
+// same one on every call, lane 0) issues, so the operands stay warp-uniform.
+// The issuing warp shares its scheduler with four softmax warps, and this
+// form issues an MMA in fewer slots than a lane-0 branch.
 __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "{\n.reg .pred p, e;\n.reg .b32 r;\nsetp.ne.b32 p, %4, 0;\nelect.sync r|e, 0xffffffff;\n"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
       "r"(a), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Commit of the elected lane's MMAs to an mbarrier (called by the same
+// converged warp as mma_ts).
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile(
+      "{\n.reg .pred e;\n.reg .b32 r;\nelect.sync r|e, 0xffffffff;\n"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
       : "memory");
 }
 // Shared-memory matrix descriptor, no swizzle: start address, leading and
@@ -275,6 +290,36 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Largest of 32 values: 16 three-input maxima, depth 4.
+__device__ __forceinline__ float max32(const float (&v)[32]) {
+  float m[12];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) m[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  m[10] = v[30];
+  m[11] = v[31];
+  const float a = fmax3(m[0], m[1], m[2]), b = fmax3(m[3], m[4], m[5]), c = fmax3(m[6], m[7], m[8]),
+              d = fmax3(m[9], m[10], m[11]);
+  return fmaxf(fmax3(a, b, c), d);
+}
+// fp16 hi + lo of a pair of non-negative fp32 values below 65504: hi is the
+// value with its 13 low mantissa bits cleared (exact in fp16 from 2^-14 up),
+// lo = w - hi (exact in fp32) rounded to fp16. Packed, first value low.
+__device__ __forceinline__ void split_pair_trunc(float2 w, uint32_t &hi, uint32_t &lo) {
+  const float2 hf = make_float2(__uint_as_float(__float_as_uint(w.x) & 0xFFFFE000u),
+                                __uint_as_float(__float_as_uint(w.y) & 0xFFFFE000u));
+  const float2 lf = __ffma2_rn(hf, make_float2(-1.0f, -1.0f), w);
+  const __half2 h = __floats2half2_rn(hf.x, hf.y);
+  const __half2 l = __floats2half2_rn(lf.x, lf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // fp16 hi + lo of a pair of fp32 values, packed (first value in the low half).
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo) {
   const __half2 h = __floats2half2_rn(x0, x1);
@@ -282,20 +327,6 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
   const __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
   hi = *reinterpret_cast<const uint32_t *>(&h);
   lo = *reinterpret_cast<const uint32_t *>(&l);
-}
-
-// Unnormalised Walsh-Hadamard transform of 128 values in registers (stages
-// h = 1, 2, ..., 64, butterfly (a, b) -> (a + b, a - b)).
-__device__ __forceinline__ void wht128_regs(float (&v)[kD]) {
-#pragma unroll
-  for (int h = 1; h < kD; h <<= 1)
-#pragma unroll
-    for (int i = 0; i < kD; ++i)
-      if ((i & h) == 0) {
-        const float a0 = v[i], a1 = v[i + h];
-        v[i] = __fadd_rn(a0, a1);
-        v[i + h] = __fsub_rn(a0, a1);
-      }
 }
 
 // ---- rANS decoding (one lane per token of a staged 32-token block) ------
@@ -558,6 +589,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
     }
     mbar_init(bars + kBarQFull, kRows * kQuads);
     mbar_init(bars + kBarDrain, 1);
+    mbar_init(bars + kBarDrainPv, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -672,10 +704,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
         for (int t = 0; t < 32; t += 4) {
           const float4 n4 = *reinterpret_cast<const float4 *>(nk + t);
-          u[t] *= n4.x;
-          u[t + 1] *= n4.y;
-          u[t + 2] *= n4.z;
-          u[t + 3] *= n4.w;
+          const float2 a0 = __fmul2_rn(make_float2(u[t], u[t + 1]), make_float2(n4.x, n4.y));
+          const float2 a1 = __fmul2_rn(make_float2(u[t + 2], u[t + 3]), make_float2(n4.z, n4.w));
+          u[t] = a0.x;
+          u[t + 1] = a0.y;
+          u[t + 2] = a1.x;
+          u[t + 3] = a1.y;
         }
         // u = S ||k|| (the logit divided by crow > 0); tokens past this row's
         // position are masked, which only happens on the causal diagonal.
@@ -685,17 +719,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
           for (int t = 0; t < 32; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
         }
-        float mu[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          mu[t] = fmaxf(fmaxf(fmaxf(u[t], u[t + 4]), fmaxf(u[t + 8], u[t + 12])),
-                        fmaxf(fmaxf(u[t + 16], u[t + 20]), fmaxf(u[t + 24], u[t + 28])));
-        mu0 = fmaxf(fmaxf(mu[0], mu[1]), fmaxf(mu[2], mu[3]));
+        mu0 = max32(u);
         // Largest V norm of this quarter's tokens (bounds the weights below).
+        {
+          float n[32];
 #pragma unroll
-        for (int t = 0; t < 32; t += 4) {
-          const float4 n4 = *reinterpret_cast<const float4 *>(nv + t);
-          mnv = fmaxf(mnv, fmaxf(fmaxf(n4.x, n4.y), fmaxf(n4.z, n4.w)));
+          for (int t = 0; t < 32; t += 4) {
+            const float4 n4 = *reinterpret_cast<const float4 *>(nv + t);
+            n[t] = n4.x;
+            n[t + 1] = n4.y;
+            n[t + 2] = n4.z;
+            n[t + 3] = n4.w;
+          }
+          mnv = max32(n);
         }
       }
       // One exchange per block among the four warps of the row: the row
@@ -758,25 +794,47 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
         // above), 16 tokens at a time: p = 2^(logit - mx), w = p ||v|| as fp16
         // hi (columns 0..15) and lo (16..31); norms of tokens past the last
         // attended position are 0, so masked tokens give exactly 0.
-        float ps[2] = {0.0f, 0.0f};
+        if (__all_sync(kFull, mx != -INFINITY)) {
+          // Packed pairs: x = u crow - mx, p = 2^x, w = p ||v||.
+          const float2 c2 = make_float2(crow, crow), m2 = make_float2(-mx, -mx);
+          float2 ps2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t wh[8], wl[8];
+          for (int c = 0; c < 2; ++c) {
+            uint32_t wh[8], wl[8];
 #pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const int t = 16 * c + 2 * p;
-            float p0 = 0.0f, p1 = 0.0f;
-            if (mx != -INFINITY) {
-              p0 = ex2(fmaf(u[t], crow, -mx));
-              p1 = ex2(fmaf(u[t + 1], crow, -mx));
+            for (int p = 0; p < 8; ++p) {
+              const int t = 16 * c + 2 * p;
+              const float2 x = __ffma2_rn(make_float2(u[t], u[t + 1]), c2, m2);
+              const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+              ps2 = __fadd2_rn(ps2, pp);
+              const float2 nn = *reinterpret_cast<const float2 *>(nv + t);
+              split_pair_trunc(__fmul2_rn(pp, nn), wh[p], wl[p]);
             }
-            ps[p & 1] += p0 + p1;
-            split_pair(p0 * nv[t], p1 * nv[t + 1], wh[p], wl[p]);
+            tmem_st8(scol + 8 * c, wh);
+            tmem_st8(scol + 16 + 8 * c, wl);
           }
-          tmem_st8(scol + 8 * c, wh);
-          tmem_st8(scol + 16 + 8 * c, wl);
+          psum = ps2.x + ps2.y;
+        } else {
+          float ps[2] = {0.0f, 0.0f};
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            uint32_t wh[8], wl[8];
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+              const int t = 16 * c + 2 * p;
+              float p0 = 0.0f, p1 = 0.0f;
+              if (mx != -INFINITY) {
+                p0 = ex2(fmaf(u[t], crow, -mx));
+                p1 = ex2(fmaf(u[t + 1], crow, -mx));
+              }
+              ps[p & 1] += p0 + p1;
+              split_pair(p0 * nv[t], p1 * nv[t + 1], wh[p], wl[p]);
+            }
+            tmem_st8(scol + 8 * c, wh);
+            tmem_st8(scol + 16 + 8 * c, wl);
+          }
+          psum = ps[0] + ps[1];
         }
-        psum = ps[0] + ps[1];
         tmem_wait_st();
       } else {
         ++timeouts;
@@ -860,43 +918,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
         for (int i = 0; i < 8; ++i) store_elem(a.out, qbase + 32 * m + 8 * qt + i, z[m][i], a.out_dtype);
     }
-  } else if (warp == kMmaWarp) {
-    // ===== MMA issue (one lane) =====
-    if (lane == 0 && nB > 0) {
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    // ===== MMA issue (one lane of each of two warps) =====
+    // Warp kMmaWarp issues the score MMAs, warp kPvWarp the P.V MMAs: two
+    // issuing threads on two schedulers. Each commits only its own MMAs;
+    // the order between the two streams comes from the barriers (S_j is
+    // written only after P.V of block j - 2 is done with its buffer; P.V of
+    // block j reads W_j, written after S_j was complete).
+    auto drain = [&](int bar) {
+      tc_commit(bars + bar);
+      const uint32_t da = smem_u32(bars + bar);
+      for (uint32_t it = 0; it < kSpin; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], 0;\nselp.u32 %0, 1, 0, P;\n}\n"
+            : "=r"(done)
+            : "r"(da)
+            : "memory");
+        if (done) break;
+      }
+    };
+    if (warp == kMmaWarp && nB > 0) {
       const uint32_t idS = instr_desc(kRows, kBlk, 0);
-      const uint32_t idO = instr_desc(kRows, kD, 1);
-      bool alive = mbar_wait(bars + kBarQFull, 0, abort_flag);
-      if (!alive) ++timeouts;
+      bool alive = __all_sync(kFull, mbar_wait(bars + kBarQFull, 0, abort_flag));
+      if (!alive && lane == 0) ++timeouts;
       tc_fence_after();
-      // O += W_jj V_jj: A = W (tensor memory; tokens 16 ks .. 16 ks + 15 of
-      // the hi or lo half), B = V tile, MN-major: token groups of 8 at 128
-      // bytes (LBO), coordinate chunks of 8 at kChunkStride bytes (SBO).
-      auto issue_pv = [&](int64_t jj) -> bool {
-        if (!mbar_wait(bars + kBarWFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vt = smem_u32(slot_base(static_cast<int>(jj % ns)) + kTileBytes);
-        const uint32_t wb = tbase + kColS + 128 * static_cast<uint32_t>(jj & 1);
-#pragma unroll
-        for (int ks = 0; ks < kBlk / 16; ++ks) {
-          const uint64_t bd = smem_desc(vt + ks * 256, 128, kChunkStride);
-          // Tokens 16 ks .. 16 ks + 15 are in quarter ks / 2: fp16 hi pairs at
-          // its columns 8 (ks % 2) .., lo pairs 16 columns further.
-          const uint32_t wc = wb + 32 * static_cast<uint32_t>(ks >> 1) + (ks & 1) * 8;
-          mma_ts(tbase + kColO, wc, bd, idO, (jj > 0 || ks > 0) ? 1u : 0u);
-          mma_ts(tbase + kColO, wc + 16, bd, idO, 1u);
-        }
-        tc_commit(bars + kBarPvDone + (jj & 1));
-        tc_commit(bars + kBarEmpty + static_cast<int>(jj % ns));
-        return true;
-      };
       for (int64_t j = 0; j < nB && alive; ++j) {
         const int rb = static_cast<int>(j % ns);
-        alive = mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag);
+        alive = __all_sync(kFull, mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag));
         // The score buffer j & 1 held W of block j - 2: wait until its P.V is done.
         if (alive && j >= 2)
-          alive = mbar_wait(bars + kBarPvDone + (j & 1), static_cast<uint32_t>(((j - 2) >> 1) & 1), abort_flag);
+          alive = __all_sync(kFull, mbar_wait(bars + kBarPvDone + (j & 1), static_cast<uint32_t>(((j - 2) >> 1) & 1), abort_flag));
         if (!alive) {
-          ++timeouts;
+          if (lane == 0) ++timeouts;
           break;
         }
         tc_fence_after();
@@ -911,24 +965,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
           mma_ts(sd, tbase + kColQl + ks * 8, bd, idS, 1u);
         }
         tc_commit(bars + kBarSFull + (j & 1));
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ++timeouts;
-          alive = false;
+      }
+      // Every MMA issued above has completed before tensor memory is freed.
+      drain(kBarDrain);
+    } else if (warp == kPvWarp && nB > 0) {
+      const uint32_t idO = instr_desc(kRows, kD, 1);
+      for (int64_t jj = 0; jj < nB; ++jj) {
+        if (!__all_sync(kFull, mbar_wait(bars + kBarWFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag))) {
+          if (lane == 0) ++timeouts;
+          break;
         }
+        tc_fence_after();
+        // O += W_jj V_jj: A = W (tensor memory; tokens 16 ks .. 16 ks + 15 of
+        // the hi or lo half), B = V tile, MN-major: token groups of 8 at 128
+        // bytes (LBO), coordinate chunks of 8 at kChunkStride bytes (SBO).
+        const uint32_t vt = smem_u32(slot_base(static_cast<int>(jj % ns)) + kTileBytes);
+        const uint32_t wb = tbase + kColS + 128 * static_cast<uint32_t>(jj & 1);
+#pragma unroll
+        for (int ks = 0; ks < kBlk / 16; ++ks) {
+          const uint64_t bd = smem_desc(vt + ks * 256, 128, kChunkStride);
+          // Tokens 16 ks .. 16 ks + 15 are in quarter ks / 2: fp16 hi pairs at
+          // its columns 8 (ks % 2) .., lo pairs 16 columns further.
+          const uint32_t wc = wb + 32 * static_cast<uint32_t>(ks >> 1) + (ks & 1) * 8;
+          mma_ts(tbase + kColO, wc, bd, idO, (jj > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tbase + kColO, wc + 16, bd, idO, 1u);
+        }
+        tc_commit(bars + kBarPvDone + (jj & 1));
+        // The slot is free once P.V is done: its score MMA completed before
+        // W_jj could be written.
+        tc_commit(bars + kBarEmpty + static_cast<int>(jj % ns));
       }
-      if (alive && !issue_pv(nB - 1)) ++timeouts;
-      // Drain: every MMA issued above has completed before tensor memory is freed.
-      tc_commit(bars + kBarDrain);
-      const uint32_t da = smem_u32(bars + kBarDrain);
-      for (uint32_t it = 0; it < kSpin; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n.reg .pred P;\nmbarrier.try_wait.parity.shared::cta.b64 P, [%1], 0;\nselp.u32 %0, 1, 0, P;\n}\n"
-            : "=r"(done)
-            : "r"(da)
-            : "memory");
-        if (done) break;
-      }
+      drain(kBarDrainPv);
     }
   } else if (warp == kLoadWarp) {
     // ===== slot loader (one lane) =====
