@@ -329,6 +329,60 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
   lo = *reinterpret_cast<const uint32_t *>(&l);
 }
 
+// 32 consecutive elements base[idx .. idx + 31] (fp32 or bf16) into v. With
+// vec (base 16-byte aligned; idx is a multiple of 32) as 16-byte loads: the
+// 32 lanes of a warp read 32 different rows, so every load instruction
+// touches 32 cache lines, and 4 (bf16) or 8 (fp32) of them replace 32.
+__device__ __forceinline__ void load_row32(const void *base, int64_t idx, int dtype, bool vec, float (&v)[32]) {
+  if (vec && dtype == DQ_BF16) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(base) + idx);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 u = __ldg(p + k);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[8 * k + 2 * e] = __uint_as_float(w[e] << 16);
+        v[8 * k + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      }
+    }
+  } else if (vec) {
+    const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + idx);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 f = __ldg(p + k);
+      v[4 * k] = f.x;
+      v[4 * k + 1] = f.y;
+      v[4 * k + 2] = f.z;
+      v[4 * k + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) v[c] = load_elem(base, idx + c, dtype);
+  }
+}
+// 8 consecutive elements base[idx .. idx + 7] = z (fp32, or bf16 rounded to
+// nearest even); with vec (base 16-byte aligned, idx a multiple of 8) as one
+// (bf16) or two (fp32) 16-byte stores.
+__device__ __forceinline__ void store_row8(void *base, int64_t idx, const float (&z)[8], int dtype, bool vec) {
+  if (vec && dtype == DQ_BF16) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(z[2 * e], z[2 * e + 1]);
+      w[e] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(base) + idx) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if (vec) {
+    float4 *p = reinterpret_cast<float4 *>(static_cast<float *>(base) + idx);
+    p[0] = make_float4(z[0], z[1], z[2], z[3]);
+    p[1] = make_float4(z[4], z[5], z[6], z[7]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) store_elem(base, idx + i, z[i], dtype);
+  }
+}
+
 // ---- rANS decoding (one lane per token of a staged 32-token block) ------
 
 struct RansLane {
@@ -625,11 +679,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
       for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
       float v[32];
+      if (in_chunk) {
+        load_row32(a.q, qbase + 32 * qt, a.q_dtype, (reinterpret_cast<uintptr_t>(a.q) & 15u) == 0, v);
+      } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float x = in_chunk ? load_elem(a.q, qbase + 32 * qt + c, a.q_dtype) : 0.0f;
-        v[c] = ((sw[qt] >> c) & 1u) ? -x : x;
+        for (int c = 0; c < 32; ++c) v[c] = 0.0f;
       }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) v[c] = ((sw[qt] >> c) & 1u) ? -v[c] : v[c];
       wht32_regs(v);
       {
         uint32_t w[16];
@@ -913,10 +970,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
         for (int i = 0; i < 8; ++i) z[m][i] = 0.0f;
     }
     if (in_chunk) {
+      const bool vec = (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) store_elem(a.out, qbase + 32 * m + 8 * qt + i, z[m][i], a.out_dtype);
+      for (int m = 0; m < 4; ++m) store_row8(a.out, qbase + 32 * m + 8 * qt, z[m], a.out_dtype, vec);
     }
   } else if (warp == kMmaWarp || warp == kPvWarp) {
     // ===== MMA issue (one lane of each of two warps) =====
