@@ -597,7 +597,7 @@ __device__ __forceinline__ void wht_4(float (&z)[4]) {
 
 __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int ns = a.nslots;
+  constexpr int ns = kMaxSlots;  // the host checks a.nslots against it
   const AttnSmem L = attn_smem_layout(ns);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
@@ -621,7 +621,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   const int i_hi = min(i_lo + Mt, a.n_q) - 1;
   const int64_t lo_pos = max(qs + i_lo, int64_t(0));
   const int64_t hi_pos = min(qs + i_hi, a.T_cap - 1);
-  const int64_t nB = lo_pos <= hi_pos ? hi_pos / kBlk + 1 : 0;  // 128-token blocks to attend
+  const int nB = lo_pos <= hi_pos ? static_cast<int>(hi_pos / kBlk) + 1 : 0;  // 128-token blocks to attend
   const int64_t gslots = (a.T_cap + kBlk - 1) / kBlk;
 
   // ---- set-up ----
@@ -744,7 +744,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 
     float m_run = -INFINITY, l_run = 0.0f;
     bool alive = true;
-    for (int64_t j = 0; j < nB; ++j) {
+    for (int j = 0; j < nB; ++j) {
       const int sb = static_cast<int>(j & 1);
       const int rb = static_cast<int>(j % ns);
       bool ok = alive && mbar_wait(bars + kBarSFull + sb, static_cast<uint32_t>((j >> 1) & 1), abort_flag) &&
@@ -770,7 +770,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
         }
         // u = S ||k|| (the logit divided by crow > 0); tokens past this row's
         // position are masked, which only happens on the causal diagonal.
-        const int64_t rel = pos - j * kBlk - 32 * qt;
+        const int64_t rel = pos - static_cast<int64_t>(j) * kBlk - 32 * qt;
         const int lim = (!row_ok || rel < 0) ? -1 : (rel > 31 ? 31 : static_cast<int>(rel));
         if (!__all_sync(kFull, lim >= 31)) {
 #pragma unroll
@@ -914,7 +914,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
     for (int q2 = 0; q2 < kQuads; ++q2) l_all += lsum[q2 * kRows + r];
     bool have_o = alive && nB > 0;
     if (have_o) {
-      const int64_t jl = nB - 1;
+      const int jl = nB - 1;
       const bool okw = mbar_wait(bars + kBarPvDone + (jl & 1), static_cast<uint32_t>((jl >> 1) & 1), abort_flag);
       if (!__all_sync(kFull, okw)) {
         ++timeouts;
@@ -999,7 +999,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       bool alive = __all_sync(kFull, mbar_wait(bars + kBarQFull, 0, abort_flag));
       if (!alive && lane == 0) ++timeouts;
       tc_fence_after();
-      for (int64_t j = 0; j < nB && alive; ++j) {
+      for (int j = 0; j < nB && alive; ++j) {
         const int rb = static_cast<int>(j % ns);
         alive = __all_sync(kFull, mbar_wait(bars + kBarFull + rb, static_cast<uint32_t>((j / ns) & 1), abort_flag));
         // The score buffer j & 1 held W of block j - 2: wait until its P.V is done.
@@ -1026,7 +1026,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       drain(kBarDrain);
     } else if (warp == kPvWarp && nB > 0) {
       const uint32_t idO = instr_desc(kRows, kD, 1);
-      for (int64_t jj = 0; jj < nB; ++jj) {
+      for (int jj = 0; jj < nB; ++jj) {
         if (!__all_sync(kFull, mbar_wait(bars + kBarWFull + (jj & 1), static_cast<uint32_t>((jj >> 1) & 1), abort_flag))) {
           if (lane == 0) ++timeouts;
           break;
@@ -1057,8 +1057,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
     // ===== slot loader (one lane) =====
     if (lane == 0 && nB > 0) {
       const uint8_t *src = a.tiles + static_cast<size_t>((bh - a.bh0) * gslots) * kSlotBytes;
-      int64_t issued = 0;
-      for (int64_t j = 0; j < nB; ++j) {
+      int issued = 0;
+      for (int j = 0; j < nB; ++j) {
         const int sl = static_cast<int>(j % ns);
         if (j >= ns && !mbar_wait(bars + kBarEmpty + sl, static_cast<uint32_t>(((j / ns) - 1) & 1), abort_flag)) {
           ++timeouts;
@@ -1070,7 +1070,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       }
       // Drain: the last copies into each slot have landed before the CTA
       // exits (bounded, whatever the abort flag says).
-      for (int64_t j = issued > ns ? issued - ns : 0; j < issued; ++j) {
+      for (int j = issued > ns ? issued - ns : 0; j < issued; ++j) {
         const uint32_t fa = smem_u32(bars + kBarFull + static_cast<int>(j % ns));
         const uint32_t par = static_cast<uint32_t>((j / ns) & 1);
         for (uint32_t it = 0; it < kSpin; ++it) {
@@ -1136,7 +1136,8 @@ bool prefill_supported(int ck, int cv) {
 
 int launch_prefill_attention(const PrefillArgs &a, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (a.nslots < 2 || a.nslots > kMaxSlots || a.tile_grid < 1 || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8))
+  if (a.nslots != kMaxSlots || a.tile_grid < 1 || (a.G != 1 && a.G != 2 && a.G != 4 && a.G != 8) ||
+      a.T_cap / kBlk >= 0x7FFFFFFF)
     return static_cast<int>(cudaErrorInvalidValue);
   const int64_t grid = prefill_grid(a.nbh, a.G, a.n_q);
   if (grid < 1 || grid > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidValue);
