@@ -84,7 +84,9 @@ constexpr uint32_t kColQl = 192;    // q~ lo: 64 columns
 constexpr uint32_t kColS = 256;     // 2 buffers x 128 columns: the scores S (fp32), then in place the
                                     // weights W: tokens 0..63 hi | lo, tokens 64..127 hi | lo (32 each)
 constexpr int kTileBytes = kBlk * kD * 2;                  // one fp16 tile: 128 tokens x 128 coordinates
-constexpr int kSlotBytes = 2 * kTileBytes + 2 * kBlk * 4;  // K tile, V tile, K norms, V norms
+constexpr int kQmaxOff = 2 * kTileBytes + 2 * kBlk * 4;    // after K tile, V tile, K norms, V norms: the
+                                                           // largest V norm of each 32-token quarter
+constexpr int kSlotBytes = kQmaxOff + 128;                 // (padded to 128 bytes)
 constexpr int kChunkStride = kBlk / 8 * 128;               // bytes between 8-coordinate chunks of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kSpin = 1u << 24;  // bound on each mbarrier wait loop
@@ -122,11 +124,11 @@ __host__ __device__ inline TilesSmem tiles_smem_layout(int ck, int cv) {
 }
 
 // Shared memory of prefill_kernel: barriers, tensor-memory base and abort
-// flag, the row-max, V-norm and go-on exchanges [2 blocks][4 quarters][128 rows],
+// flag, the row-max and go-on exchanges [2 blocks][4 quarters][128 rows],
 // the row-sum exchange [4 quarters][128 rows] of the softmax warps of a row,
 // then the ring.
 struct AttnSmem {
-  size_t bars, misc, pmax, lsum, pnv, pgo, ring, total;
+  size_t bars, misc, pmax, lsum, pgo, ring, total;
 };
 
 __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
@@ -135,8 +137,7 @@ __host__ __device__ inline AttnSmem attn_smem_layout(int nslots) {
   s.misc = s.bars + kNumBars * 8;
   s.pmax = align_up(s.misc + 16, 16);
   s.lsum = s.pmax + 2 * kQuads * kRows * 4;
-  s.pnv = s.lsum + kQuads * kRows * 4;
-  s.pgo = s.pnv + 2 * kQuads * kRows * 4;
+  s.pgo = s.lsum + kQuads * kRows * 4;
   s.ring = align_up(s.pgo + 2 * kQuads * kRows * 4, 128);
   s.total = s.ring + static_cast<size_t>(nslots) * kSlotBytes;
   return s;
@@ -540,7 +541,11 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
       // Tokens past the last attended position keep zero norms: their bytes
       // may be anything, and the softmax multiplies the weights by them.
       nrm[tl] = tok <= hi ? norm_of(kb) : 0.0f;
-      nrm[kBlk + tl] = tok <= hi ? norm_of(vb) : 0.0f;
+      const float nvt = tok <= hi ? norm_of(vb) : 0.0f;
+      nrm[kBlk + tl] = nvt;
+      // The quarter's largest V norm (bounds the softmax weights of a block).
+      const float qm = warp_max(nvt);
+      if (lane == 0) reinterpret_cast<float *>(dst + kQmaxOff)[q4] = qm;
       if (tok <= hi) bad += (rk.x != kL) + (rv.x != kL);
     } else {
       const uint4 z = make_uint4(0u, 0u, 0u, 0u);
@@ -551,6 +556,7 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
       }
       nrm[tl] = 0.0f;
       nrm[kBlk + tl] = 0.0f;
+      if (lane == 0) reinterpret_cast<float *>(dst + kQmaxOff)[q4] = 0.0f;
     }
     __syncwarp();  // the staging slot is refilled next iteration
     u = u_next;
@@ -604,7 +610,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + L.misc);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L.misc + 4);
   float *pmax = reinterpret_cast<float *>(smem + L.pmax);  // [2][kQuads][128]
-  float *pnv = reinterpret_cast<float *>(smem + L.pnv);    // [2][kQuads][128]: largest V norm of a row quarter
   float *lsum = reinterpret_cast<float *>(smem + L.lsum);  // [kQuads][128]
   int *pgo = reinterpret_cast<int *>(smem + L.pgo);        // [2][kQuads][128]: the warp's waits succeeded
   auto slot_base = [&](int d) { return smem + L.ring + static_cast<size_t>(d) * kSlotBytes; };
@@ -753,7 +758,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
       const uint32_t scol = tl + kColS + 128 * sb + 32 * qt;  // this warp's 32 score columns
       const float *nv = reinterpret_cast<const float *>(slot_base(rb) + 2 * kTileBytes) + kBlk + 32 * qt;
       float u[32];
-      float mu0 = -INFINITY, mnv = 0.0f;
+      float mu0 = -INFINITY, vmax = 0.0f;
       if (ok) {
         tc_fence_after();
         tmem_ld32(scol, u);
@@ -777,34 +782,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
           for (int t = 0; t < 32; ++t) u[t] = t <= lim ? u[t] : -INFINITY;
         }
         mu0 = max32(u);
-        // Largest V norm of this quarter's tokens (bounds the weights below).
-        {
-          float n[32];
-#pragma unroll
-          for (int t = 0; t < 32; t += 4) {
-            const float4 n4 = *reinterpret_cast<const float4 *>(nv + t);
-            n[t] = n4.x;
-            n[t + 1] = n4.y;
-            n[t + 2] = n4.z;
-            n[t + 3] = n4.w;
-          }
-          mnv = max32(n);
-        }
+        // Largest V norm of the block's tokens (bounds the weights below),
+        // from the slot's four quarter maxima.
+        const float4 qv = *reinterpret_cast<const float4 *>(slot_base(rb) + kQmaxOff);
+        vmax = fmaxf(fmax3(qv.x, qv.y, qv.z), qv.w);
       }
       // One exchange per block among the four warps of the row: the row
-      // maximum, the largest V norm, and whether each warp could go on (its
-      // waits succeeded). The four leave the loop together when one cannot.
+      // maximum and whether each warp could go on (its waits succeeded).
+      // The four leave the loop together when one cannot.
       pmax[(sb * kQuads + qt) * kRows + r] = mu0;
-      pnv[(sb * kQuads + qt) * kRows + r] = mnv;
       pgo[(sb * kQuads + qt) * kRows + r] = ok ? 1 : 0;
       quad_sync(quad_id);
       bool go = true;
-      float mrow = -INFINITY, vmax = 0.0f;
+      float mrow = -INFINITY;
 #pragma unroll
       for (int q2 = 0; q2 < kQuads; ++q2) {
         go = go && pgo[(sb * kQuads + q2) * kRows + r] != 0;
         mrow = fmaxf(mrow, pmax[(sb * kQuads + q2) * kRows + r]);
-        vmax = fmaxf(vmax, pnv[(sb * kQuads + q2) * kRows + r]);
       }
       if (!go) {
         if (alive) ++timeouts;

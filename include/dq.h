@@ -332,7 +332,7 @@ int dq_decode_attention_noalloc(const dq_tables *t, const void *q, int q_dtype,
  *               [0, T_cap) gets out = 0 and is counted in clamped_lengths
  *   out         device [B][n_q][Hq][128], out_dtype DQ_F32 or DQ_BF16
  *   d_workspace device, 16-byte aligned, contents need not be
- *               initialised: the decoded tiles (520 bytes per token and KV
+ *               initialised: the decoded tiles (521 bytes per token and KV
  *               head of the cache). dq_prefill_workspace_bytes(...) bytes
  *               hold the whole batch; any size down to one (b, KV head)
  *               row, dq_prefill_workspace_bytes(t, 1, 1, T_cap), works:
