@@ -90,6 +90,27 @@ __device__ __forceinline__ void store_container(uint8_t *dst, int C, uint16_t n1
   }
 }
 
+// store_container by a whole converged warp, one byte per lane: the string
+// is the one lane `src` encoded (its pushes at stack[src + 32 j]); every lane
+// passes that lane's x and len.
+__device__ __forceinline__ void store_container_warp(uint8_t *dst, int C, uint16_t n16, uint32_t x,
+                                                     const uint8_t *stack, int src, int len, int lane) {
+  const int np = len - 3;
+#pragma unroll
+  for (int k0 = 0; k0 < kMaxContainer; k0 += 32) {
+    const int k = k0 + lane;
+    if (k < C) {
+      uint8_t byte;
+      if (k == 0) byte = static_cast<uint8_t>(n16 & 0xFFu);
+      else if (k == 1) byte = static_cast<uint8_t>(n16 >> 8);
+      else if (k < 5) byte = static_cast<uint8_t>((x >> (8 * (k - 2))) & 0xFFu);
+      else if (k - 5 < np) byte = stack[src + 32 * (np - 1 - (k - 5))];
+      else byte = 0;
+      dst[32 * k] = byte;
+    }
+  }
+}
+
 // Best drift move of symbol i (one level toward a strictly cheaper neighbour):
 // key = ((u - y_j)^2 - (u - y_q)^2) / (cost_q - cost_j) in fp32, ties to the
 // lower j. Returns +inf when the symbol has no candidate.
@@ -161,18 +182,29 @@ __device__ __forceinline__ uint32_t sign_bit(uint32_t word, int b) { return (wor
 // stored). No lane branches, so all 32 lanes of a warp stay converged. kTwo:
 // the table has a symbol with f < 16, so a step can push two bytes. kStk:
 // push-stack slots per lane (a power of two, at least C - 4).
-// One encode step of encode_bf.
+//
+// A push is st.shared.u8 without a memory clobber, so that the compiler can
+// move the next steps' symbol and table loads ahead of it (as a C++ store it
+// could not tell the push stack from the tables and held every load back
+// behind the previous step's store). The stack is not read during the
+// encode; encode_bf has compiler barriers before and after the pushes.
+__device__ __forceinline__ void push_byte(uint32_t a, uint32_t v) {
+  asm volatile("st.shared.u8 [%0], %1;\n" ::"r"(a), "r"(v));
+}
+
+// One encode step of encode_bf (stk_s: the lane's stack as a shared-memory
+// address).
 template <bool kTwo, int kStk = kStackSlots>
-__device__ __forceinline__ void encode_step(uint32_t s, const uint8_t *esb, uint8_t *stk, uint32_t &x, uint32_t &np) {
+__device__ __forceinline__ void encode_step(uint32_t s, const uint8_t *esb, uint32_t stk_s, uint32_t &x, uint32_t &np) {
   const uint4 e0 = *reinterpret_cast<const uint4 *>(esb + s * sizeof(EncSym));  // {m, k, xmax, cum}
   const uint32_t g = *reinterpret_cast<const uint32_t *>(esb + s * sizeof(EncSym) + 16);
   bool push = x >= e0.z;
-  stk[32 * (np & (kStk - 1))] = static_cast<uint8_t>(x);
+  push_byte(stk_s + 32 * (np & (kStk - 1)), x & 0xFFu);
   np += push ? 1u : 0u;
   x = push ? (x >> 8) : x;
   if constexpr (kTwo) {
     push = x >= e0.z;
-    stk[32 * (np & (kStk - 1))] = static_cast<uint8_t>(x);
+    push_byte(stk_s + 32 * (np & (kStk - 1)), x & 0xFFu);
     np += push ? 1u : 0u;
     x = push ? (x >> 8) : x;
   }
@@ -187,13 +219,16 @@ __device__ __forceinline__ int encode_bf(SymFn sym, const EncSym *es, uint8_t *s
   uint32_t x = kL;
   uint32_t np = 0;
   const uint8_t *esb = reinterpret_cast<const uint8_t *>(es);
+  asm volatile("" ::: "memory");  // earlier stores (of the stack too) come before the pushes
+  const uint32_t stk_s = static_cast<uint32_t>(__cvta_generic_to_shared(stk));
   if constexpr (kRegs) {
 #pragma unroll
-    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo, kStk>(sym(i), esb, stk, x, np);
+    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo, kStk>(sym(i), esb, stk_s, x, np);
   } else {
-#pragma unroll 4
-    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo, kStk>(sym(i), esb, stk, x, np);
+#pragma unroll 8
+    for (int i = kD - 1; i >= 0; --i) encode_step<kTwo, kStk>(sym(i), esb, stk_s, x, np);
   }
+  asm volatile("" ::: "memory");  // the pushes above come before any read of the stack
   *x_out = x;
   return 3 + static_cast<int>(np);
 }
@@ -566,11 +601,12 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
     if (fit) {
       const int win = __ffs(fit) - 1;
       applied = ranked + win + 1;
-      if (lane == win) {
-        bool dr = false;
-        uint8_t *dst = c.dst_of(a, vd, &dr);
-        if (dst) store_container(dst, c.C, n16v, x, stk, len);
-      }
+      const uint32_t xw = __shfl_sync(kFull, x, win);
+      const int lw = __shfl_sync(kFull, len, win);
+      __syncwarp();  // lane win's pushes before the other lanes read them
+      bool dr = false;
+      uint8_t *dst = c.dst_of(a, vd, &dr);
+      if (dst) store_container_warp(dst, c.C, n16v, xw, stack, win, lw, lane);
     } else {
       ranked += added;
       exhausted = added < batch;
@@ -814,11 +850,14 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   DriftCount dc;
   int applied = 0;
   if (len <= c.P) {
-    if (lane == 0 && dst) store_container(dst, c.C, n16, x, stk, len);
+    // Every lane encoded the same string: lane k stores byte k from its own stack.
+    if (dst) store_container_warp(dst, c.C, n16, x, W.stack, lane, len, lane);
   } else {
     __syncwarp();
-    // One pass of 32 in most cases (latency of a small append).
-    applied = drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 32, dc);
+    // One pass in most cases (latency of a small append): most strings that
+    // miss need one to three moves, and ranking is a serial warp reduction
+    // per move.
+    applied = drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 16, dc);
   }
   if (a.drift_mode == 1 && applied >= 0) {
     // The symbols after drift (the first `applied` ranked moves) go to tgt[].
