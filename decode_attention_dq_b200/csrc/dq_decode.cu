@@ -615,9 +615,11 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
 // a time (lane i reads slot i's (m, l), so the batch's weights come from one
 // load per lane and one max/sum over the warp; the partial o vectors of the
 // batch are then read with independent loads), merging batch after batch
-// with an online rescale. The warps' results meet in shared memory.
-constexpr int kCombWarps = 4;
-
+// with an online rescale. The warps' results meet in shared memory. With a
+// small batch a row has hundreds of slots (one per split warp) and few rows
+// run at once, so the host takes 16 warps per CTA there (the merge is a
+// chain of load batches, latency-bound), 4 otherwise.
+template <int kCombWarps>
 __global__ void __launch_bounds__(kCombWarps * 32) combine_kernel(const DecodeArgs a) {
   __shared__ float sh_m[kCombWarps], sh_l[kCombWarps];
   __shared__ float sh_o[kCombWarps][kD];
@@ -753,7 +755,11 @@ int launch_decode_attention(const DecodeArgs &a, void *stream) {
   if (e) return e;
   const int64_t rows = static_cast<int64_t>(a.B) * a.Hq;
   if (rows > 0x7FFFFFFF) return static_cast<int>(cudaErrorInvalidValue);
-  combine_kernel<<<static_cast<unsigned>(rows), kCombWarps * 32, 0, st>>>(a);
+  // At least 64 slots per (b, KV head) possible: wide CTAs.
+  if (a.total_warps >= static_cast<int64_t>(64) * a.B * a.Hkv)
+    combine_kernel<16><<<static_cast<unsigned>(rows), 16 * 32, 0, st>>>(a);
+  else
+    combine_kernel<4><<<static_cast<unsigned>(rows), 4 * 32, 0, st>>>(a);
   return static_cast<int>(cudaGetLastError());
 }
 
