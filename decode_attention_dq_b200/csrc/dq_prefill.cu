@@ -629,6 +629,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   const int nB = lo_pos <= hi_pos ? static_cast<int>(hi_pos / kBlk) + 1 : 0;  // 128-token blocks to attend
   const int64_t gslots = (a.T_cap + kBlk - 1) / kBlk;
 
+  // A softmax thread's query row (thread = row r of the block). Its loads
+  // start before the set-up barrier, so that their latency overlaps the
+  // tensor-memory allocation and the barrier initialisation.
+  const int qt = warp >> 2;  // token quarter of a softmax warp
+  const int r = (warp & 3) * 32 + lane;
+  const int ti = i_lo + r / G, g = r % G;
+  const bool in_chunk = warp < kSoftWarps && ti <= i_hi;
+  const int64_t qbase = ((static_cast<int64_t>(b) * a.n_q + (in_chunk ? ti : 0)) * a.Hq + h * G + g) * kD;
+  float qrow[32];
+  if (in_chunk) {
+    load_row32(a.q, qbase + 32 * qt, a.q_dtype, (reinterpret_cast<uintptr_t>(a.q) & 15u) == 0, qrow);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 32; ++c) qrow[c] = 0.0f;
+  }
+
   // ---- set-up ----
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tslot)),
@@ -661,16 +677,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
   if (warp < kSoftWarps) {
     // ===== softmax: warps w, w + 4, w + 8, w + 12 own rows r = 32 (w % 4) +
     // lane; warp w + 4 q takes tokens 32 q .. 32 q + 31 of each block =====
-    const int qt = warp >> 2;                    // token quarter of this warp
-    const int r = (warp & 3) * 32 + lane;
     const uint32_t tl = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);  // this warp's lanes
-    const int ti = i_lo + r / G, g = r % G;
-    const bool in_chunk = ti <= i_hi;
     const int64_t pos = qs + ti;
     const bool row_ok = in_chunk && pos >= 0 && pos < a.T_cap;
     if (qt == 0 && in_chunk && !row_ok) ++clamped;
-    const int hq = h * G + g;
-    const int64_t qbase = ((static_cast<int64_t>(b) * a.n_q + (in_chunk ? ti : 0)) * a.Hq + hq) * kD;
     const int quad_id = 1 + (warp & 3);
     // D1: q~ = H D q (unnormalised), times 2^e so that max |q~| is in [2^13,
     // 2^14). The four threads of a row share the work: thread qt rotates
@@ -684,14 +694,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
       for (int k = 0; k < 4; ++k) sw[k] = __ldg(a.sign_bits + h * 4 + k);
       float v[32];
-      if (in_chunk) {
-        load_row32(a.q, qbase + 32 * qt, a.q_dtype, (reinterpret_cast<uintptr_t>(a.q) & 15u) == 0, v);
-      } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) v[c] = 0.0f;
-      }
-#pragma unroll
-      for (int c = 0; c < 32; ++c) v[c] = ((sw[qt] >> c) & 1u) ? -v[c] : v[c];
+      for (int c = 0; c < 32; ++c) v[c] = ((sw[qt] >> c) & 1u) ? -qrow[c] : qrow[c];
       wht32_regs(v);
       {
         uint32_t w[16];
