@@ -967,8 +967,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1) prefill_kernel(const PrefillA
 #pragma unroll
         for (int i = 0; i < 8; ++i) z[m][i] = 0.0f;
     }
-    if (in_chunk) {
-      const bool vec = (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
+    const bool vec = (reinterpret_cast<uintptr_t>(a.out) & 15u) == 0;
+    if (have_o && vec) {
+      // Through shared memory, so that a store instruction writes one whole
+      // output row (a warp's 32 lanes would otherwise write 32 rows). The
+      // ring is idle: every block's copies have landed and its MMAs are done
+      // (P.V of the last block, waited above). Rows 32 (w % 4) .. + 31 of
+      // the quad, 132 floats apart (no bank conflicts).
+      float *stg = reinterpret_cast<float *>(slot_base(0));
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float4 *p4 = reinterpret_cast<float4 *>(stg + r * 132 + 32 * m + 8 * qt);
+        p4[0] = make_float4(z[m][0], z[m][1], z[m][2], z[m][3]);
+        p4[1] = make_float4(z[m][4], z[m][5], z[m][6], z[m][7]);
+      }
+      quad_sync(quad_id);
+      // Warp qt of the quad stores rows 8 qt .. 8 qt + 7 of the quad's 32.
+#pragma unroll 2
+      for (int k = 0; k < 8; ++k) {
+        const int rr = (warp & 3) * 32 + 8 * qt + k;
+        const int ti2 = i_lo + rr / G;
+        if (ti2 > i_hi) continue;  // past the chunk (same for the whole warp)
+        const int64_t base2 = ((static_cast<int64_t>(b) * a.n_q + ti2) * a.Hq + h * G + rr % G) * kD;
+        const float4 val = reinterpret_cast<const float4 *>(stg + rr * 132)[lane];
+        if (a.out_dtype == DQ_BF16) {
+          const __nv_bfloat162 h0 = __floats2bfloat162_rn(val.x, val.y), h1 = __floats2bfloat162_rn(val.z, val.w);
+          reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(a.out) + base2)[lane] =
+              make_uint2(*reinterpret_cast<const uint32_t *>(&h0), *reinterpret_cast<const uint32_t *>(&h1));
+        } else {
+          reinterpret_cast<float4 *>(static_cast<float *>(a.out) + base2)[lane] = val;
+        }
+      }
+    } else if (in_chunk) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) store_row8(a.out, qbase + 32 * m + 8 * qt, z[m], a.out_dtype, vec);
     }
