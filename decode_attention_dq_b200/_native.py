@@ -12,7 +12,9 @@ from dataclasses import dataclass
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "lib", "libdq.so")
+# DQ_LIBRARY selects another build of the same ABI (lib/libdq_checked.so:
+# the attention kernels also count containers decoded past their bytes).
+LIB_PATH = os.environ.get("DQ_LIBRARY") or os.path.join(HERE, "lib", "libdq.so")
 
 DQ_OK = 0
 DQ_F32, DQ_BF16 = 0, 1
@@ -20,7 +22,7 @@ DQ_STREAM_K, DQ_STREAM_V = 0, 1
 STATS_FIELDS = ("k_syms_drifted", "v_syms_drifted", "k_cont_drifted", "v_cont_drifted",
                 "overflow_fallbacks", "integrity_errors", "nonfinite_inputs",
                 "dropped_writes", "clamped_lengths", "bad_pages", "wait_timeouts",
-                "k_syms_filled", "v_syms_filled")
+                "k_syms_filled", "v_syms_filled", "overreads")
 EXPORTED = ("dq_config_default", "dq_build_tables", "dq_free_tables", "dq_get_stream_table",
             "dq_get_stream_design", "dq_get_signs", "dq_append_kv", "dq_decode_workspace_bytes",
             "dq_decode_attention", "dq_decode_symbols", "dq_error_string", "dq_last_cuda_error",

@@ -117,6 +117,15 @@ __device__ __forceinline__ RansLane rans_open(const uint8_t *smem, uint32_t off)
   return r;
 }
 
+#ifdef DQ_CHECKED
+// Whether a lane's decoder consumed bytes past its container of C bytes at
+// cb (the cursor starts at byte 5 and moves 32 per byte consumed). Counted in
+// dq_stats.overreads by DQ_CHECKED builds.
+__device__ __forceinline__ bool overread(const RansLane &r, const uint8_t *cb, const uint8_t *smem, int C) {
+  return r.p > static_cast<uint32_t>(cb - smem) + static_cast<uint32_t>(C) * kTile;
+}
+#endif
+
 // One decode step. Table entry layout: bits 0..10 slot - c_s, bits 11..13 the
 // symbol s, bits 20..31 f_s. The state advances as x = f (x >> 12) + (slot -
 // c_s). Renormalisation has no branches: while x < 2^16 the next byte b is
@@ -373,6 +382,9 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
   const int64_t g_end = warp_first(wid + 1, W, N);
   if (g >= g_end) return;
   unsigned bad_count = 0;
+#ifdef DQ_CHECKED
+  unsigned over_count = 0;
+#endif
   unsigned bad_pages = 0;
 
   // Sequence holding flat group g: the largest b with prefix[b] * Hkv <= g
@@ -480,6 +492,9 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
       }
       const bool valid = group_t0(0) + lane < len;
       bad_count += __popc(__ballot_sync(kFull, valid && rk.x != kL));
+#ifdef DQ_CHECKED
+      over_count += __popc(__ballot_sync(kFull, valid && overread(rk, kb, smem, ck)));
+#endif
       softmax_update(acc, sc, norm_of(kb), valid, p, lane);
     }
     for (int64_t j = 0; j < n; ++j) {
@@ -564,10 +579,16 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
       {
         const bool vvalid = group_t0(j) + lane < len;
         bad_count += __popc(__ballot_sync(kFull, vvalid && rv.x != kL));
+#ifdef DQ_CHECKED
+        over_count += __popc(__ballot_sync(kFull, vvalid && overread(rv, vb, smem, cv)));
+#endif
       }
       if (has_next) {
         const bool valid = group_t0(j + 1) + lane < len;
         bad_count += __popc(__ballot_sync(kFull, valid && rk.x != kL));
+#ifdef DQ_CHECKED
+        over_count += __popc(__ballot_sync(kFull, valid && overread(rk, kb, smem, ck)));
+#endif
         softmax_update(acc, sc, norm_of(kb), valid, p, lane);
         // The next iteration needs V(j+1) (slot nxt) and K(j+2) (slot cur).
         cp_async_wait_0();
@@ -608,6 +629,9 @@ __global__ void __launch_bounds__(max_warps_for(G) * 32, 1) decode_split_kernel(
   }
   if (a.stats && lane == 0 && bad_count) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(bad_count));
   if (a.stats && lane == 0 && bad_pages) atomicAdd(&a.stats->bad_pages, static_cast<unsigned long long>(bad_pages));
+#ifdef DQ_CHECKED
+  if (a.stats && lane == 0 && over_count) atomicAdd(&a.stats->overreads, static_cast<unsigned long long>(over_count));
+#endif
 }
 
 // Combine: one CTA of kCombWarps warps per (b, query head). The warps split

@@ -462,6 +462,9 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   auto kslot = [&](int s) { return stg + s * L.kslot; };
   auto vslot = [&](int s) { return stg + 2 * L.kslot + s * L.vslot; };
   unsigned bad = 0, bad_pages = 0;
+#ifdef DQ_CHECKED
+  unsigned over = 0;  // containers decoded past their C bytes
+#endif
   auto last_of = [&](int64_t u) -> int64_t {
     return last_position(a.q_start[(a.bh0 + u / (gslots * kQuarters)) / a.Hkv], a.n_q, a.T_cap);
   };
@@ -547,6 +550,12 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
       const float qm = warp_max(nvt);
       if (lane == 0) reinterpret_cast<float *>(dst + kQmaxOff)[q4] = qm;
       if (tok <= hi) bad += (rk.x != kL) + (rv.x != kL);
+#ifdef DQ_CHECKED
+      // The cursor starts at byte 5 and moves 32 per byte consumed.
+      if (tok <= hi)
+        over += (rk.p > static_cast<uint32_t>(kb - smem) + static_cast<uint32_t>(ck) * kGrp) +
+                (rv.p > static_cast<uint32_t>(vb - smem) + static_cast<uint32_t>(cv) * kGrp);
+#endif
     } else {
       const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll 1
@@ -563,6 +572,10 @@ __global__ void __launch_bounds__(kTileWarps * 32, 1) prefill_tiles_kernel(const
   }
   cp_async_wait_0();
   if (a.stats) {
+#ifdef DQ_CHECKED
+    const unsigned o_w = __reduce_add_sync(kFull, over);
+    if (lane == 0 && o_w) atomicAdd(&a.stats->overreads, static_cast<unsigned long long>(o_w));
+#endif
     const unsigned b_w = __reduce_add_sync(kFull, bad);
     const unsigned p_w = __reduce_add_sync(kFull, bad_pages);
     if (lane == 0 && b_w) atomicAdd(&a.stats->integrity_errors, static_cast<unsigned long long>(b_w));

@@ -106,6 +106,14 @@ typedef struct {
   unsigned long long wait_timeouts;      /* bounded in-kernel waits given up */
   unsigned long long k_syms_filled;      /* K symbols moved up by the fill   */
   unsigned long long v_syms_filled;      /* V symbols moved up by the fill   */
+  unsigned long long overreads;          /* checked builds only (libdq_checked.so,
+                                          * compiled with DQ_CHECKED): containers
+                                          * whose decoder inside the attention
+                                          * kernels consumed bytes past the
+                                          * container (a corrupt container; the
+                                          * read stays in the kernel's shared
+                                          * memory and is counted, never
+                                          * trapped). Always 0 in libdq.so. */
 } dq_stats;
 
 typedef struct dq_tables dq_tables; /* opaque, library-owned */

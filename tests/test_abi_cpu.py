@@ -1,8 +1,10 @@
 """CPU checks of the C-ABI boundary (no GPU needed).
 
-libdq.so loads and exports every function include/dq.h declares; its
-host-side table design (dq_design_stream, the same code dq_build_tables
-uploads) is byte-identical to the oracle's independently written design.
+libdq.so (and the DQ_CHECKED build, libdq_checked.so) loads and exports
+every function include/dq.h declares; the binding's stats fields are the
+header's; the host-side table design (dq_design_stream, the same code
+dq_build_tables uploads) is byte-identical to the oracle's independently
+written design.
 """
 import ctypes
 import os
@@ -32,6 +34,28 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
         assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
     assert set(declared) == set(N.EXPORTED)
+
+
+def _stats_fields():
+    text = open(os.path.join(ROOT, "include", "dq.h")).read()
+    body = re.search(r"typedef struct \{([^}]*)\} dq_stats;", text, flags=re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    return tuple(re.findall(r"unsigned long long (\w+);", body))
+
+
+def test_stats_fields_match_the_header():
+    # new_stats() allocates one uint64 per STATS_FIELDS entry: the binding's
+    # names and order must be the C struct's.
+    assert _stats_fields() == N.STATS_FIELDS
+
+
+def test_checked_library_exports_every_declared_symbol():
+    from decode_attention_dq_b200 import build
+
+    path = build.build(checked=True)  # no-op when up to date
+    lib = ctypes.CDLL(path)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
 
 
 def test_error_strings():
