@@ -890,9 +890,9 @@ def prefill_launches_per_step(drift_mode):
 # pass) of `bench.py --prefill 512 --workload qwen3_8b_b16_t8k`: the decoded
 # tiles read once (545 MB) plus the queries, and the fp32 output. Reported
 # only for that workload and container size while the kernel source matches.
-PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "32b03172d79d0996",
+PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "ea5171e9edcc4ac1",
                    "workload": "qwen3_8b_b16_t8k", "chunk": 512, "ck": 36, "cv": 36,
-                   "bytes": 615.28e6 + 121.70e6}
+                   "bytes": 617.33e6 + 129.95e6}
 
 
 def prefill_traffic(workload, n_q, ck, cv):
