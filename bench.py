@@ -62,8 +62,8 @@ LAUNCHES_PER_STEP = 4
 # writes the partial states). It belongs to one version of the kernel source:
 # for any other, or other container sizes, traffic is reported as null.
 DECODE_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_decode.cu",
-                  "sha256_16": "5ea9de2e196cf75f", "ck": 36, "cv": 36,
-                  "bytes_per_token_head": (151.373312e6 + 3.464960e6) / (32 * 8 * 8192)}
+                  "sha256_16": "5f062cef3d424eb2", "ck": 36, "cv": 36,
+                  "bytes_per_token_head": (151.369216e6 + 3.344896e6) / (32 * 8 * 8192)}
 
 
 def decode_traffic(token_heads, ck, cv):
