@@ -551,10 +551,14 @@ struct DriftCount {
 // scratch, stack the warp's push stacks. Returns the number of moves applied
 // (the ranked moves 0 .. n - 1, in rank[] / tgt[]), or -1 after a fallback.
 template <bool kTwo>
+// zero_first: the string without moves has not been encoded yet; the first
+// pass ranks 31 moves and lane m encodes the string with m of them (lane 0:
+// none), so that the first count that fits, zero included, comes out of one
+// encode pass. Later passes are as without it.
 __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c, const AppendTables &T,
                                           uint8_t *stack, const uint8_t *q, uint8_t *rank, uint8_t *tgt, int64_t vd,
                                           uint16_t n16v, const float (&u)[4], int lane, int first_batch,
-                                          DriftCount &dc) {
+                                          DriftCount &dc, bool zero_first = false) {
   uint8_t *stk = stack + lane;
   // Best move and key of the 4 symbols this lane owns (i = lane + 32 k).
   uint32_t key[4];
@@ -573,7 +577,8 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
   while (applied < 0 && !exhausted) {
     // Rank the next moves by repeated arg-min over (key, index):
     // first_batch on the first pass, then up to 32 per pass.
-    const int batch = ranked == 0 ? first_batch : 32;
+    const bool zf = zero_first && ranked == 0;  // this pass includes the string without moves
+    const int batch = zf ? 31 : (ranked == 0 ? first_batch : 32);
     int added = 0;
     for (; added < batch; ++added) {
       const int bi = warp_argmin(key, lane);
@@ -587,8 +592,9 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
     }
     __syncwarp();
     // Lane m encodes the string with moves 0 .. ranked + m applied (lanes
-    // m >= added too, with all ranked moves; their result is not used).
-    const int m_moves = ranked + lane;  // highest rank applied by this lane
+    // m >= added too, with all ranked moves; their result is not used); in
+    // a zero-first pass, moves 0 .. m - 1 (lanes m > added: not used).
+    const int m_moves = zf ? lane - 1 : ranked + lane;  // highest rank applied by this lane
     uint32_t x = 0;
     const int len = encode_bf<kTwo, false>(
         [&](int i) {
@@ -597,10 +603,10 @@ __device__ __forceinline__ int drift_one(const AppendArgs &a, const StreamCtx &c
                                                                   : static_cast<uint32_t>(q[i]);
         },
         T.es, stk, &x);
-    const unsigned fit = __ballot_sync(kFull, lane < added && len <= c.P);
+    const unsigned fit = __ballot_sync(kFull, (zf ? lane <= added : lane < added) && len <= c.P);
     if (fit) {
       const int win = __ffs(fit) - 1;
-      applied = ranked + win + 1;
+      applied = zf ? win : ranked + win + 1;
       const uint32_t xw = __shfl_sync(kFull, x, win);
       const int lw = __shfl_sync(kFull, len, win);
       __syncwarp();  // lane win's pushes before the other lanes read them
@@ -842,29 +848,45 @@ __device__ __forceinline__ void warp_body(const AppendArgs &a, AppendTables &T, 
   bool nf;
   warp_prepare(a, c.src, v, c.head_of(a, v), c.t, lane, u, W.q, &n16, &nf);
   __syncwarp();
-  uint8_t *stk = W.stack + lane;
-  uint32_t x = 0;
-  const int len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(W.q[i]); }, T.es, stk, &x);
   bool dropped = false, bad_page = false;
   uint8_t *dst = c.dst_of(a, v, &dropped, &bad_page);
   DriftCount dc;
   int applied = 0;
-  if (len <= c.P) {
-    // Every lane encoded the same string: lane k stores byte k from its own stack.
-    if (dst) store_container_warp(dst, c.C, n16, x, W.stack, lane, len, lane);
+  // The string's ideal length, the sum of its symbols' costs in bits. An
+  // encoded string pushes at most that + a fraction of a bit, so a string
+  // that ends up too long (more than P - 3 pushes) costs nearly 8 (P - 2)
+  // bits or more. Above 8 (P - 3) + 4 bits the warp ranks its moves before
+  // encoding and tries 0 .. 31 moves in one pass (the greedy result as
+  // before, without a first encode that would fail); below it, one encode,
+  // and drift after it in the rare case that the string is still too long.
+  float cbits = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) cbits += T.cost[W.q[lane + 32 * k]];
+  cbits = warp_sum(cbits);
+  const bool spec = __shfl_sync(kFull, cbits > 8.0f * static_cast<float>(c.P - 3) + 4.0f, 0);
+  bool drifted = spec;
+  int len = 0;
+  if (spec) {
+    applied = drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 32, dc, true);
   } else {
-    __syncwarp();
-    // One pass in most cases (latency of a small append): most strings that
-    // miss need one to three moves, and ranking is a serial warp reduction
-    // per move.
-    applied = drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 16, dc);
+    uint8_t *stk = W.stack + lane;
+    uint32_t x = 0;
+    len = encode_bf<kTwo, false>([&](int i) { return static_cast<uint32_t>(W.q[i]); }, T.es, stk, &x);
+    if (len <= c.P) {
+      // Every lane encoded the same string: lane k stores byte k from its own stack.
+      if (dst) store_container_warp(dst, c.C, n16, x, W.stack, lane, len, lane);
+    } else {
+      __syncwarp();
+      drifted = true;
+      applied = drift_one<kTwo>(a, c, T, W.stack, W.q, W.rank, W.tgt, v, n16, u, lane, 16, dc);
+    }
   }
   if (a.drift_mode == 1 && applied >= 0) {
     // The symbols after drift (the first `applied` ranked moves) go to tgt[].
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int i = lane + 32 * k;
-      const uint32_t r = (len <= c.P) ? kNoRank : W.rank[i];
+      const uint32_t r = drifted ? W.rank[i] : kNoRank;
       W.tgt[i] = (r != kNoRank && static_cast<int>(r) < applied) ? W.tgt[i] : W.q[i];
     }
     __syncwarp();
