@@ -1,9 +1,10 @@
 """Pins for the oracle's rANS coder.
 
 Round trips on random strings (including frequency-1 symbols and constant
-strings), the decoder's final state returning to L, and the code length of a
+strings), the decoder's final state returning to L, the code length of a
 long stream within 1% of the information-theoretic cross-entropy of the
-integer model.
+integer model, and a 128-symbol string's pushed bits within [-8.5, +1] of
+its ideal length.
 """
 import numpy as np
 import pytest
@@ -75,3 +76,28 @@ def test_decoder_flags_corruption():
         rc, dq, xf, used = o.rans_decode(st, b2, 128)
         flagged += (rc != 0) or (not np.array_equal(dq, q))
     assert flagged == 200
+
+
+@pytest.mark.parametrize("n,cb", [(8, 36), (6, 36), (8, 31), (6, 48)])
+def test_pushed_bits_track_the_ideal_length(n, cb):
+    # A 128-symbol string's pushed bytes carry its ideal length, the sum of
+    # the symbols' costs -log2(f / 4096), less what stays in the final state
+    # (up to 8 bits above the initial 2^16) and at most a fraction of a bit
+    # more (the integer model's rounding). The decode-step append uses the
+    # upper bound to rank moves before the first encode of a string that may
+    # not fit; its result does not depend on it.
+    st = o.Stream(n, cb)
+    rng = np.random.default_rng(n * 1000 + cb)
+    p = st.freq / 4096.0
+    for trial in range(1500):
+        mode = trial % 3
+        if mode == 0:
+            q = rng.choice(n, size=128, p=p)
+        elif mode == 1:
+            q = rng.integers(0, n, 128)  # rare symbols often
+        else:
+            q = np.where(rng.random(128) < 0.5, 0, n - 1)
+        q = q.astype(np.uint8)
+        length, _ = o.rans_encode(st, q)
+        resid = (length - 3) * 8 - float(st.cost[q].astype(np.float64).sum())
+        assert -8.5 <= resid <= 1.0, (trial, resid)
