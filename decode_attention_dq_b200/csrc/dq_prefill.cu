@@ -82,7 +82,8 @@ constexpr uint32_t kColO = 0;       // O: 128 fp32 columns
 constexpr uint32_t kColQh = 128;    // q~ hi: 64 columns of packed fp16 pairs
 constexpr uint32_t kColQl = 192;    // q~ lo: 64 columns
 constexpr uint32_t kColS = 256;     // 2 buffers x 128 columns: the scores S (fp32), then in place the
-                                    // weights W: tokens 0..63 hi | lo, tokens 64..127 hi | lo (32 each)
+                                    // weights W: per 32-token quarter, 16 columns of fp16 hi pairs,
+                                    // then 16 of lo pairs
 constexpr int kTileBytes = kBlk * kD * 2;                  // one fp16 tile: 128 tokens x 128 coordinates
 constexpr int kQmaxOff = 2 * kTileBytes + 2 * kBlk * 4;    // after K tile, V tile, K norms, V norms: the
                                                            // largest V norm of each 32-token quarter
