@@ -31,7 +31,11 @@
 //     arithmetic), ranks the candidate moves by repeated arg-min (least key
 //     first, ties to the lower index), and lane m encodes the string with the
 //     first m+1 moves applied; the smallest m that fits is the greedy result.
-//     The warp-per-vector kernel tries 32 move counts per pass. The separate
+//     The warp-per-vector kernel (small appends) tries up to 32 move counts
+//     per pass; a string whose symbol costs add up to near the budget is
+//     ranked before its first encode, so that one pass tries 0 .. 31 moves
+//     (lane m: m moves) instead of an encode that fails and a second one;
+//     it stores a container with the whole warp, a byte per lane. The separate
 //     drift kernel (lane-per-vector appends) keeps 8 containers per warp in
 //     flight and tries 4 move counts of each per encode pass, ranking 4 more
 //     moves of a container only when its window had no fit; in drift mode 1
