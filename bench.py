@@ -57,12 +57,14 @@ ENCODE_OPS_PER_VECTOR = 2560
 LAUNCHES_PER_STEP = 4
 # DRAM traffic of decode_split_kernel from one ncu capture (dram__bytes_read
 # + dram__bytes_write) of the 32-sequence, 8192-token workload with 36-byte
-# containers: 151.37 MB + 3.99 MB per launch over 32*8*8192 token-heads. It
+# containers: 151.37 MB + 3.34 MB per launch over 32*8*8192 token-heads. It
 # scales with the token-heads a launch processes (reads are the containers,
 # writes the partial states). It belongs to one version of the kernel source:
 # for any other, or other container sizes, traffic is reported as null.
+# (Captured at source hash 5f062cef3d424eb2; the file has changed since in
+# one comment only.)
 DECODE_TRAFFIC = {"source": "decode_attention_dq_b200/csrc/dq_decode.cu",
-                  "sha256_16": "5f062cef3d424eb2", "ck": 36, "cv": 36,
+                  "sha256_16": "2e1b65131b495877", "ck": 36, "cv": 36,
                   "bytes_per_token_head": (151.369216e6 + 3.344896e6) / (32 * 8 * 8192)}
 
 

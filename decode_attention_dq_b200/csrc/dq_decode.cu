@@ -37,7 +37,8 @@
 //       levels are stored as fp16(kappa y) with a per-table kappa that makes
 //       them exact to a few 1e-5 (relative), undone in the combine
 //   D6  at the end of a segment the warp writes (m, l, o_rot) to its slot
-// Combine kernel, one warp per (b, query head):
+// Combine kernel, one CTA per (b, query head), of 16 warps for small batches
+// (hundreds of slots per row) and 4 otherwise:
 //   D7  log-sum-exp merge of the slots of (b, h), o = D H o_rot / (128 l)
 #include <type_traits>
 
