@@ -100,3 +100,40 @@ def test_host_design_rejects_bad_configs():
     assert e.value.code == -2
     with pytest.raises(N.DqError):
         N.dq_design_stream(10, 36)  # the decoder supports at most 8 levels
+
+
+def test_argument_errors_are_codes_before_any_device_work():
+    # Host-side fault injection: null pointers and invalid configurations
+    # come back as error codes from the argument checks, which run before
+    # any CUDA call (so this needs no GPU), and size queries without tables
+    # return 0.
+    lib = N.load()
+    vp, i32, i64, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    null_calls = {
+        "dq_append_kv": ([vp, vp, vp, i32, i32, i32, i32, vp, vp, vp, i64, vp, vp],
+                         [None, None, None, 0, 1, 1, 1, None, None, None, 32, None, None]),
+        "dq_decode_attention": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, i64, i64, f32, vp, i32, vp, sz, vp, vp],
+                                [None, None, 0, None, None, None, 1, 4, 1, 32, 32, 0.0, None, 0, None, 0, None, None]),
+        "dq_prefill_attention": ([vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, i64, f32, vp, i32, vp, sz, vp, vp],
+                                 [None, None, 0, None, None, None, 1, 1, 4, 1, 32, 0.0, None, 0, None, 0, None, None]),
+        "dq_get_signs": ([vp, vp], [None, None]),
+        "dq_build_tables": ([vp, vp], [None, None]),
+    }
+    for name, (argt, args) in null_calls.items():
+        f = getattr(lib, name)
+        f.argtypes, f.restype = argt, ctypes.c_int
+        assert f(*args) == -1, name  # DQ_ERR_NULL
+    for name, argt, args in (("dq_decode_workspace_bytes", [vp, i32, i32, i32, i64], [None, 1, 4, 1, 32]),
+                             ("dq_prefill_workspace_bytes", [vp, i32, i32, i64], [None, 1, 1, 32]),
+                             ("dq_append_workspace_bytes", [vp, i32, i32, i32], [None, 1, 1, 1])):
+        f = getattr(lib, name)
+        f.argtypes, f.restype = argt, sz
+        assert f(*args) == 0, name
+    out = ctypes.c_void_p()
+    for fields, code in (({"head_dim": 64}, -2), ({"prob_bits": 11}, -2), ({"k_levels": 9}, -2),
+                         ({"n_kv_heads": 0}, -2), ({"k_container_bytes": 8}, -3)):
+        cfg = N.DqConfig()
+        lib.dq_config_default(ctypes.byref(cfg))
+        for k, v in fields.items():
+            setattr(cfg, k, v)
+        assert lib.dq_build_tables(ctypes.byref(cfg), ctypes.byref(out)) == code, fields
